@@ -40,7 +40,7 @@ _STREAMS = {"keys": 0, "values": 1, "clusters": 2, "queries": 3, "append": 4, "q
 # strength) were calibrated with the oracle on the 1M workload so that the
 # fraction of the cache read lands in the 1-6 % band.
 SHIFT = 3.0
-RUN = 1024
+RUN = 8192
 BETA = 48.0
 ZIPF_S = 1.1
 

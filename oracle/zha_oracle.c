@@ -178,7 +178,10 @@ static int cmp_i64(const void *a, const void *b) {
  *
  * Outputs: sel[0..count) = kept level-1 block ids, ascending (capacity n_1);
  * per level l (index l-1): n_cand[l-1], n_kept[l-1], margin[l-1] with
- * margin = min(c_m - p, p - c_{m-1}, P_(m) - P_(m+1)) (absent terms = +inf).
+ * margin = min(c_m - p, p - c_{m-1}, s_(m) - s_(m+1)): the distance of the
+ * cumulative normalised mass from p on both sides of the cut, and the score
+ * gap (log-mass units) between the last kept and the first dropped candidate
+ * (absent terms = +inf).
  * Returns the count.
  */
 int64_t oracle_route(const double *q, int d, int R, int B, int b, int64_t N, int L,
@@ -232,7 +235,7 @@ int64_t oracle_route(const double *q, int d, int R, int B, int b, int64_t N, int
             }
             double t1 = cum - p[l - 1];
             double t2 = p[l - 1] - prev;
-            double t3 = m < nc ? (exp(cand[m - 1].s - smax) - exp(cand[m].s - smax)) / total : INFINITY;
+            double t3 = m < nc ? cand[m - 1].s - cand[m].s : INFINITY;
             mg = t1 < t2 ? t1 : t2;
             if (t3 < mg) mg = t3;
         }

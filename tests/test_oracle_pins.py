@@ -273,17 +273,18 @@ def _children_scores_level(tree, l, x):
 
 
 def test_margin_is_the_distance_of_the_cut_from_p():
-    """For a flat one-level case the margin equals min(c_m - p, p - c_{m-1}, P_(m) - P_(m+1))
-    computed here from brute-force sorted probabilities."""
+    """For a flat one-level case the margin equals min(c_m - p, p - c_{m-1}, s_(m) - s_(m+1))
+    computed here from brute-force sorted probabilities and scores."""
     d, N = 16, 12
     r = rng(400)
     K = (r.standard_normal((N, d)) * 1.5).astype(np.float32)
     x = r.standard_normal(d) * 2
     tree, _ = _tree(K, N, 1, 16)
-    probs = np.sort(softmax(tree.scale * K.astype(np.float64) @ x))[::-1]
+    z = np.sort(tree.scale * K.astype(np.float64) @ x)[::-1]
+    probs = softmax(z)
     c = np.cumsum(probs)
     m = int(np.argmax(c >= 0.8)) + 1
-    expect = min(c[m - 1] - 0.8, 0.8 - (c[m - 2] if m >= 2 else 0.0), probs[m - 1] - probs[m])
+    expect = min(c[m - 1] - 0.8, 0.8 - (c[m - 2] if m >= 2 else 0.0), z[m - 1] - z[m])
     assert abs(O.route(x, tree, 0.8).margin[0] - expect) < 1e-12
 
 
