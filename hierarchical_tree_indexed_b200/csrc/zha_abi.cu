@@ -1,0 +1,509 @@
+// zha_abi.cu -- the C ABI (include/zha.h): argument checks, buffer layouts and
+// kernel launches.  Every step of the path runs in the kernels included below;
+// this file only validates, lays out the caller's buffers and launches.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "zha.h"
+#include "zha_common.cuh"
+#include "zha_build.cuh"
+#include "zha_route.cuh"
+#include "zha_attend.cuh"
+
+using namespace zha;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+#define ZHA_CUDA(call)                                                                   \
+    do {                                                                                 \
+        cudaError_t e_ = (call);                                                         \
+        if (e_ != cudaSuccess) return fail(ZHA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+    } while (0)
+
+#define ZHA_TRY(expr)               \
+    do {                            \
+        int r_ = (expr);            \
+        if (r_ != ZHA_OK) return r_; \
+    } while (0)
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct TreeLayout {
+    int Lcap;
+    int64_t ncap[kMaxLevels];
+    size_t off_ntree, off_qref, off_khat[kMaxLevels], off_bhat[kMaxLevels], total;
+};
+
+struct WsLayout {
+    int64_t cand_cap, par_cap, sel_cap, item_cap, words;
+    size_t off_scores, off_parents, off_sel, off_count, off_items, off_nitems, off_ml, off_acc, off_counters;
+    size_t total;
+};
+
+
+int validate(const zha_config* c) {
+    if (!c) return fail(ZHA_ERR_INVALID_ARG, "cfg is null");
+    if (c->d != 64 && c->d != 128) return fail(ZHA_ERR_UNSUPPORTED, "d=%d: head dim must be 64 or 128", c->d);
+    if (c->Hq < 1 || c->Hkv < 1 || c->Hq % c->Hkv) return fail(ZHA_ERR_INVALID_ARG, "Hq=%d must be a positive multiple of Hkv=%d", c->Hq, c->Hkv);
+    const int G = c->Hq / c->Hkv;
+    if (G != 1 && G != 2 && G != 4) return fail(ZHA_ERR_UNSUPPORTED, "Hq/Hkv=%d: groups of 1, 2 or 4 query heads", G);
+    if (c->Hkv > 32) return fail(ZHA_ERR_UNSUPPORTED, "Hkv=%d > 32", c->Hkv);
+    if (c->B < 1) return fail(ZHA_ERR_INVALID_ARG, "B=%d", c->B);
+    if (c->B > 64) return fail(ZHA_ERR_UNSUPPORTED, "B=%d > 64", c->B);
+    if (c->b < 2 || c->b > 32) return fail(c->b < 2 ? ZHA_ERR_INVALID_ARG : ZHA_ERR_UNSUPPORTED, "b=%d: branching must be 2..32", c->b);
+    if (c->R < 1) return fail(ZHA_ERR_INVALID_ARG, "R=%d", c->R);
+    if (c->R != 1) return fail(ZHA_ERR_UNSUPPORTED, "R=%d: the GPU path keeps one reference query per node", c->R);
+    if (c->dtype != ZHA_F32 && c->dtype != ZHA_BF16) return fail(ZHA_ERR_INVALID_ARG, "dtype=%d", c->dtype);
+    if (c->batch < 1) return fail(ZHA_ERR_INVALID_ARG, "batch=%d", c->batch);
+    if (c->N_cap < 1 || c->N_cap > (int64_t{1} << 31) - 128) return fail(ZHA_ERR_INVALID_ARG, "N_cap=%lld", (long long)c->N_cap);
+    if (c->L_fixed < 0 || c->L_fixed > ZHA_MAX_LEVELS) return fail(ZHA_ERR_INVALID_ARG, "L_fixed=%d", c->L_fixed);
+    if (!(c->scale >= 0.f) || !std::isfinite(c->scale)) return fail(ZHA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+    int64_t n[kMaxLevels];
+    const int L = tree_levels(c->N_cap, c->B, c->b, c->L_fixed, n);
+    if (L < 0) return fail(ZHA_ERR_UNSUPPORTED, "tree deeper than %d levels", ZHA_MAX_LEVELS);
+    for (int l = 0; l < L; ++l)
+        if (!(c->p[l] > 0.f) || !std::isfinite(c->p[l])) return fail(ZHA_ERR_INVALID_ARG, "p[%d]=%g must be in (0, inf)", l, c->p[l]);
+    return ZHA_OK;
+}
+
+float scale_of(const zha_config* c) { return c->scale > 0.f ? c->scale : 1.0f / std::sqrt(static_cast<float>(c->d)); }
+
+int tree_layout(const zha_config* c, TreeLayout* t) {
+    ZHA_TRY(validate(c));
+    int64_t n[kMaxLevels];
+    t->Lcap = tree_levels(c->N_cap, c->B, c->b, c->L_fixed, n);
+    const int64_t slices = static_cast<int64_t>(c->batch) * c->Hkv;
+    size_t off = 0;
+    t->off_ntree = off;
+    off = align256(off + sizeof(int32_t) * c->batch);
+    t->off_qref = off;
+    off = align256(off + sizeof(float) * static_cast<size_t>(c->Hkv) * t->Lcap * c->R * c->d);
+    for (int l = 0; l < kMaxLevels; ++l) {
+        t->ncap[l] = l < t->Lcap ? std::max<int64_t>(n[l], 1) : 0;
+        t->off_khat[l] = off;
+        off = align256(off + sizeof(float) * static_cast<size_t>(slices) * t->ncap[l] * c->R * c->d);
+        t->off_bhat[l] = off;
+        off = align256(off + sizeof(float) * static_cast<size_t>(slices) * t->ncap[l] * c->R);
+    }
+    t->total = off;
+    return ZHA_OK;
+}
+
+TreeDev tree_view(const TreeLayout& t, void* tree) {
+    TreeDev v{};
+    char* base = static_cast<char*>(tree);
+    v.n_tree = reinterpret_cast<int32_t*>(base + t.off_ntree);
+    v.qref = reinterpret_cast<float*>(base + t.off_qref);
+    for (int l = 0; l < kMaxLevels; ++l) {
+        v.khat[l] = reinterpret_cast<float*>(base + t.off_khat[l]);
+        v.bhat[l] = reinterpret_cast<float*>(base + t.off_bhat[l]);
+        v.ncap[l] = t.ncap[l];
+    }
+    v.Lcap = t.Lcap;
+    return v;
+}
+
+int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
+    if (n_q != 1) return fail(ZHA_ERR_UNSUPPORTED, "n_q=%d: decode takes one query per sequence", n_q);
+    const int64_t groups = static_cast<int64_t>(c->batch) * c->Hkv;
+    const int64_t ctas = static_cast<int64_t>(c->batch) * c->Hq * n_q;
+    const int G = c->Hq / c->Hkv;
+    w->cand_cap = t.ncap[0] + c->b;
+    w->par_cap = std::max<int64_t>(t.ncap[0], 1);
+    w->sel_cap = std::max<int64_t>(t.ncap[0], 1);
+    w->item_cap = t.ncap[0] + 2 + (c->N_cap + kAttRows - 1) / kAttRows;
+    w->words = (t.ncap[0] + 31) / 32;
+    size_t off = 0;
+    w->off_scores = off;   off = align256(off + sizeof(float) * ctas * w->cand_cap);
+    w->off_parents = off;  off = align256(off + sizeof(int32_t) * ctas * 2 * w->par_cap);
+    w->off_sel = off;      off = align256(off + sizeof(int32_t) * ctas * w->sel_cap);
+    w->off_count = off;    off = align256(off + sizeof(int32_t) * ctas);
+    w->off_items = off;    off = align256(off + sizeof(int2) * groups * w->item_cap);
+    w->off_nitems = off;   off = align256(off + sizeof(int32_t) * groups);
+    w->off_ml = off;       off = align256(off + sizeof(float2) * groups * kSplitMax * G);
+    w->off_acc = off;      off = align256(off + sizeof(float) * groups * kSplitMax * G * c->d);
+    w->off_counters = off; off = align256(off + sizeof(uint32_t) * groups);
+    w->total = off;
+    if (static_cast<size_t>(G) * w->words * 4 > 200 * 1024)
+        return fail(ZHA_ERR_UNSUPPORTED, "N_cap too large for the on-chip union bitmap");
+    return ZHA_OK;
+}
+
+template <typename P>
+P* at(void* base, size_t off) { return reinterpret_cast<P*>(static_cast<char*>(base) + off); }
+
+struct DevInfo {
+    int sms = 0;
+    int smem_optin = 0;
+};
+
+int dev_info(DevInfo* info) {
+    static std::mutex mu;
+    static DevInfo cache[64];
+    int dev = 0;
+    ZHA_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(ZHA_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev].sms == 0) {
+        ZHA_CUDA(cudaDeviceGetAttribute(&cache[dev].sms, cudaDevAttrMultiProcessorCount, dev));
+        ZHA_CUDA(cudaDeviceGetAttribute(&cache[dev].smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    }
+    *info = cache[dev];
+    return ZHA_OK;
+}
+
+// Lets `kernel` use the device's opt-in shared memory (once per kernel and device).
+template <typename Kern>
+int allow_smem(Kern kernel, size_t need) {
+    static std::mutex mu;
+    static std::set<std::pair<const void*, int>> done;
+    DevInfo di;
+    ZHA_TRY(dev_info(&di));
+    cudaFuncAttributes fa;
+    ZHA_CUDA(cudaFuncGetAttributes(&fa, kernel));
+    const size_t dyn_max = static_cast<size_t>(di.smem_optin) - fa.sharedSizeBytes;
+    if (need > dyn_max)
+        return fail(ZHA_ERR_UNSUPPORTED, "kernel needs %zu B of dynamic shared memory (device max %zu)", need, dyn_max);
+    int dev = 0;
+    ZHA_CUDA(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lk(mu);
+    auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+    if (!done.count(key)) {
+        ZHA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn_max)));
+        done.insert(key);
+    }
+    return ZHA_OK;
+}
+
+int check_launch(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ZHA_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    return ZHA_OK;
+}
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------- build / append
+template <typename T, int D>
+int run_build(const zha_config* c, const TreeLayout& lay, const void* K, const int32_t* N, void* tree,
+              cudaStream_t st) {
+    BuildArgs a{};
+    a.tree = tree_view(lay, tree);
+    a.K = K;
+    a.N = N;
+    a.batch = c->batch; a.Hkv = c->Hkv; a.B = c->B; a.b = c->b; a.L_fixed = c->L_fixed;
+    a.N_cap = c->N_cap;
+    a.scale = scale_of(c);
+    const int64_t slices = static_cast<int64_t>(c->batch) * c->Hkv;
+    build_set_count_kernel<<<static_cast<unsigned>(cdiv(c->batch, 128)), 128, 0, st>>>(a.tree, N, c->batch, c->N_cap);
+    ZHA_TRY(check_launch("build_set_count"));
+    build_leaf_kernel<T, D><<<static_cast<unsigned>(cdiv(slices * lay.ncap[0] * 32, 256)), 256, 0, st>>>(a);
+    ZHA_TRY(check_launch("build_leaf"));
+    for (int l = 2; l <= lay.Lcap; ++l) {
+        build_upper_kernel<D><<<static_cast<unsigned>(cdiv(slices * lay.ncap[l - 1] * 32, 256)), 256, 0, st>>>(a, l);
+        ZHA_TRY(check_launch("build_upper"));
+    }
+    return ZHA_OK;
+}
+
+template <typename T, int D>
+int run_append(const zha_config* c, const TreeLayout& lay, void* K, void* V, const void* kn, const void* vn,
+               int32_t* N, void* tree, cudaStream_t st) {
+    AppendArgs a{};
+    a.tree = tree_view(lay, tree);
+    a.K = K; a.V = V; a.k_new = kn; a.v_new = vn; a.N = N;
+    a.batch = c->batch; a.Hkv = c->Hkv; a.B = c->B; a.b = c->b; a.L_fixed = c->L_fixed;
+    a.N_cap = c->N_cap;
+    a.scale = scale_of(c);
+    append_kernel<T, D><<<c->batch, 32 * c->Hkv, 0, st>>>(a);
+    return check_launch("append");
+}
+
+// ---------------------------------------------------------------- route
+template <typename T, int D, int NVR>
+int run_route_t(const RouteArgs& a, int ctas, cudaStream_t st) {
+    auto kern = route_decode_kernel<T, D, NVR>;
+    ZHA_TRY(allow_smem(kern, sizeof(RouteSmem)));
+    kern<<<ctas, kRouteThreads, sizeof(RouteSmem), st>>>(a);
+    return check_launch("route");
+}
+
+template <typename T, int D>
+int run_route(const zha_config* c, const TreeLayout& lay, const WsLayout& wl, const void* tree, const void* Q,
+              const int32_t* N, int32_t* sel, int32_t* cnt, int32_t sel_cap, void* ws, cudaStream_t st) {
+    RouteArgs a{};
+    a.tree = tree_view(lay, const_cast<void*>(tree));
+    a.Q = Q; a.N = N; a.sel = sel; a.sel_count = cnt;
+    a.ws_scores = at<float>(ws, wl.off_scores);
+    a.ws_parents = at<int32_t>(ws, wl.off_parents);
+    a.cand_cap = wl.cand_cap; a.par_cap = wl.par_cap; a.N_cap = c->N_cap;
+    a.sel_cap = sel_cap; a.batch = c->batch; a.Hq = c->Hq; a.Hkv = c->Hkv; a.B = c->B; a.b = c->b;
+    a.L_fixed = c->L_fixed; a.n_q = 1;
+    a.scale = scale_of(c);
+    for (int l = 0; l < kMaxLevels; ++l) a.p[l] = c->p[l];
+    const int ctas = c->batch * c->Hq;
+    if (c->b <= 4) return run_route_t<T, D, 4>(a, ctas, st);
+    if (c->b <= 8) return run_route_t<T, D, 8>(a, ctas, st);
+    if (c->b <= 16) return run_route_t<T, D, 16>(a, ctas, st);
+    return run_route_t<T, D, 32>(a, ctas, st);
+}
+
+// ---------------------------------------------------------------- attend
+template <typename T, int D, int G>
+int run_attend_t(const AttendArgs& a, cudaStream_t st) {
+    auto kern = attend_kernel<T, D, G>;
+    const size_t smem = sizeof(AttSmem<T, D, G>) + sizeof(int) * (a.groups + 1);
+    ZHA_TRY(allow_smem(kern, smem));
+    DevInfo di;
+    ZHA_TRY(dev_info(&di));
+    kern<<<2 * di.sms, kAttThreads, smem, st>>>(a);
+    return check_launch("attend");
+}
+
+template <typename T, int D>
+int run_attend(const zha_config* c, const WsLayout& wl, const void* K, const void* V, const void* Q, float* O,
+               void* ws, cudaStream_t st) {
+    AttendArgs a{};
+    a.K = K; a.V = V; a.Q = Q; a.O = O;
+    a.items = at<int2>(ws, wl.off_items);
+    a.n_items = at<int32_t>(ws, wl.off_nitems);
+    a.part_ml = at<float2>(ws, wl.off_ml);
+    a.part_acc = at<float>(ws, wl.off_acc);
+    a.counters = at<uint32_t>(ws, wl.off_counters);
+    a.item_cap = wl.item_cap; a.N_cap = c->N_cap;
+    a.groups = c->batch * c->Hkv; a.Hq = c->Hq; a.Hkv = c->Hkv; a.n_q = 1;
+    a.qscale = scale_of(c) * 1.4426950408889634f;
+    switch (c->Hq / c->Hkv) {
+        case 1: return run_attend_t<T, D, 1>(a, st);
+        case 2: return run_attend_t<T, D, 2>(a, st);
+        default: return run_attend_t<T, D, 4>(a, st);
+    }
+}
+
+int run_plan(const zha_config* c, const WsLayout& wl, const TreeLayout& lay, const void* tree, const int32_t* N,
+             const int32_t* sel, const int32_t* cnt, int32_t sel_cap, void* ws, cudaStream_t st) {
+    PlanArgs a{};
+    a.sel = sel; a.sel_count = cnt; a.N = N;
+    a.n_tree = tree_view(lay, const_cast<void*>(tree)).n_tree;
+    a.items = at<int2>(ws, wl.off_items);
+    a.n_items = at<int32_t>(ws, wl.off_nitems);
+    a.item_cap = wl.item_cap; a.N_cap = c->N_cap;
+    a.sel_cap = sel_cap; a.Hq = c->Hq; a.Hkv = c->Hkv; a.G = c->Hq / c->Hkv; a.B = c->B; a.n_q = 1;
+    a.words = std::max<int64_t>(wl.words, 1);
+    const size_t smem = sizeof(uint32_t) * a.G * a.words;
+    ZHA_TRY(allow_smem(plan_decode_kernel, smem));
+    plan_decode_kernel<<<c->batch * c->Hkv, kPlanThreads, smem, st>>>(a);
+    return check_launch("plan");
+}
+
+// Dispatch on (dtype, d).
+#define ZHA_DISPATCH(c, FN, ...)                                                          \
+    ((c)->dtype == ZHA_BF16 ? ((c)->d == 128 ? FN<uint16_t, 128>(__VA_ARGS__) : FN<uint16_t, 64>(__VA_ARGS__)) \
+                            : ((c)->d == 128 ? FN<float, 128>(__VA_ARGS__) : FN<float, 64>(__VA_ARGS__)))
+
+int need(const void* p, const char* name) {
+    return p ? ZHA_OK : fail(ZHA_ERR_INVALID_ARG, "%s is null", name);
+}
+
+int check_ws(const WsLayout& wl, const void* ws, size_t ws_bytes) {
+    ZHA_TRY(need(ws, "ws"));
+    if (ws_bytes < wl.total) return fail(ZHA_ERR_WORKSPACE, "workspace of %zu B < %zu B needed", ws_bytes, wl.total);
+    return ZHA_OK;
+}
+
+}  // namespace
+
+// ======================================================================== C ABI
+extern "C" {
+
+int zha_levels_cap(const zha_config* cfg, int32_t* levels) {
+    TreeLayout t;
+    ZHA_TRY(need(levels, "levels"));
+    ZHA_TRY(tree_layout(cfg, &t));
+    *levels = t.Lcap;
+    return ZHA_OK;
+}
+
+int zha_tree_bytes(const zha_config* cfg, size_t* bytes) {
+    TreeLayout t;
+    ZHA_TRY(need(bytes, "bytes"));
+    ZHA_TRY(tree_layout(cfg, &t));
+    *bytes = t.total;
+    return ZHA_OK;
+}
+
+int zha_tree_level(const zha_config* cfg, int32_t level, size_t* khat_offset, size_t* bhat_offset,
+                   int64_t* nodes_cap) {
+    TreeLayout t;
+    ZHA_TRY(need(khat_offset, "khat_offset"));
+    ZHA_TRY(need(bhat_offset, "bhat_offset"));
+    ZHA_TRY(need(nodes_cap, "nodes_cap"));
+    ZHA_TRY(tree_layout(cfg, &t));
+    if (level < 1 || level > t.Lcap) return fail(ZHA_ERR_INVALID_ARG, "level=%d outside 1..%d", level, t.Lcap);
+    *khat_offset = t.off_khat[level - 1];
+    *bhat_offset = t.off_bhat[level - 1];
+    *nodes_cap = t.ncap[level - 1];
+    return ZHA_OK;
+}
+
+int zha_tree_count_offset(const zha_config* cfg, size_t* offset) {
+    TreeLayout t;
+    ZHA_TRY(need(offset, "offset"));
+    ZHA_TRY(tree_layout(cfg, &t));
+    *offset = t.off_ntree;
+    return ZHA_OK;
+}
+
+int zha_workspace_bytes(const zha_config* cfg, int32_t n_q, size_t* bytes) {
+    TreeLayout t;
+    WsLayout w;
+    ZHA_TRY(need(bytes, "bytes"));
+    ZHA_TRY(tree_layout(cfg, &t));
+    ZHA_TRY(ws_layout(cfg, n_q, t, &w));
+    *bytes = w.total;
+    return ZHA_OK;
+}
+
+int zha_workspace_init(const zha_config* cfg, void* ws, size_t ws_bytes, zha_stream_t stream) {
+    TreeLayout t;
+    WsLayout w;
+    ZHA_TRY(tree_layout(cfg, &t));
+    ZHA_TRY(ws_layout(cfg, 1, t, &w));
+    ZHA_TRY(check_ws(w, ws, ws_bytes));
+    ZHA_CUDA(cudaMemsetAsync(ws, 0, w.total, stream));
+    return ZHA_OK;
+}
+
+int zha_build(const zha_config* cfg, const void* K, const float* Qref, const int32_t* N, void* tree,
+              zha_stream_t stream) {
+    TreeLayout t;
+    ZHA_TRY(tree_layout(cfg, &t));
+    ZHA_TRY(need(K, "K"));
+    ZHA_TRY(need(Qref, "Qref"));
+    ZHA_TRY(need(N, "N"));
+    ZHA_TRY(need(tree, "tree"));
+    const size_t qbytes = sizeof(float) * static_cast<size_t>(cfg->Hkv) * t.Lcap * cfg->R * cfg->d;
+    ZHA_CUDA(cudaMemcpyAsync(static_cast<char*>(tree) + t.off_qref, Qref, qbytes, cudaMemcpyDeviceToDevice, stream));
+    return ZHA_DISPATCH(cfg, run_build, cfg, t, K, N, tree, stream);
+}
+
+int zha_append(const zha_config* cfg, void* K, void* V, const void* k_new, const void* v_new, int32_t* N,
+               void* tree, zha_stream_t stream) {
+    TreeLayout t;
+    ZHA_TRY(tree_layout(cfg, &t));
+    ZHA_TRY(need(K, "K"));
+    ZHA_TRY(need(V, "V"));
+    ZHA_TRY(need(k_new, "k_new"));
+    ZHA_TRY(need(v_new, "v_new"));
+    ZHA_TRY(need(N, "N"));
+    ZHA_TRY(need(tree, "tree"));
+    return ZHA_DISPATCH(cfg, run_append, cfg, t, K, V, k_new, v_new, N, tree, stream);
+}
+
+int zha_route(const zha_config* cfg, const void* tree, const void* Q, int32_t n_q, const int32_t* N, int32_t* sel,
+              int32_t* sel_count, int32_t sel_cap, void* ws, size_t ws_bytes, zha_stream_t stream) {
+    TreeLayout t;
+    WsLayout w;
+    ZHA_TRY(tree_layout(cfg, &t));
+    ZHA_TRY(ws_layout(cfg, n_q, t, &w));
+    ZHA_TRY(check_ws(w, ws, ws_bytes));
+    ZHA_TRY(need(tree, "tree"));
+    ZHA_TRY(need(Q, "Q"));
+    ZHA_TRY(need(N, "N"));
+    ZHA_TRY(need(sel, "sel"));
+    ZHA_TRY(need(sel_count, "sel_count"));
+    if (sel_cap < 1) return fail(ZHA_ERR_INVALID_ARG, "sel_cap=%d", sel_cap);
+    return ZHA_DISPATCH(cfg, run_route, cfg, t, w, tree, Q, N, sel, sel_count, sel_cap, ws, stream);
+}
+
+int zha_attend(const zha_config* cfg, const void* K, const void* V, const void* tree, const void* Q, int32_t n_q,
+               const int32_t* N, const int32_t* sel, const int32_t* sel_count, int32_t sel_cap, float* O, void* ws,
+               size_t ws_bytes, zha_stream_t stream) {
+    TreeLayout t;
+    WsLayout w;
+    ZHA_TRY(tree_layout(cfg, &t));
+    ZHA_TRY(ws_layout(cfg, n_q, t, &w));
+    ZHA_TRY(check_ws(w, ws, ws_bytes));
+    ZHA_TRY(need(K, "K"));
+    ZHA_TRY(need(V, "V"));
+    ZHA_TRY(need(tree, "tree"));
+    ZHA_TRY(need(Q, "Q"));
+    ZHA_TRY(need(N, "N"));
+    ZHA_TRY(need(sel, "sel"));
+    ZHA_TRY(need(sel_count, "sel_count"));
+    ZHA_TRY(need(O, "O"));
+    if (sel_cap < 1) return fail(ZHA_ERR_INVALID_ARG, "sel_cap=%d", sel_cap);
+    ZHA_TRY(run_plan(cfg, w, t, tree, N, sel, sel_count, sel_cap, ws, stream));
+    return ZHA_DISPATCH(cfg, run_attend, cfg, w, K, V, Q, O, ws, stream);
+}
+
+int zha_decode(const zha_config* cfg, void* K, void* V, void* tree, const void* q, const void* k_new,
+               const void* v_new, int32_t* N, float* O, void* ws, size_t ws_bytes, zha_stream_t stream) {
+    TreeLayout t;
+    WsLayout w;
+    ZHA_TRY(tree_layout(cfg, &t));
+    ZHA_TRY(ws_layout(cfg, 1, t, &w));
+    ZHA_TRY(check_ws(w, ws, ws_bytes));
+    ZHA_TRY(need(q, "q"));
+    ZHA_TRY(need(O, "O"));
+    ZHA_TRY(zha_append(cfg, K, V, k_new, v_new, N, tree, stream));
+    int32_t* sel = at<int32_t>(ws, w.off_sel);
+    int32_t* cnt = at<int32_t>(ws, w.off_count);
+    const int32_t sel_cap = static_cast<int32_t>(w.sel_cap);
+    ZHA_TRY(ZHA_DISPATCH(cfg, run_route, cfg, t, w, tree, q, N, sel, cnt, sel_cap, ws, stream));
+    ZHA_TRY(run_plan(cfg, w, t, tree, N, sel, cnt, sel_cap, ws, stream));
+    return ZHA_DISPATCH(cfg, run_attend, cfg, w, K, V, q, O, ws, stream);
+}
+
+int zha_dense(const zha_config* cfg, const void* K, const void* V, const void* Q, int32_t n_q, const int32_t* N,
+              float* O, void* ws, size_t ws_bytes, zha_stream_t stream) {
+    TreeLayout t;
+    WsLayout w;
+    ZHA_TRY(tree_layout(cfg, &t));
+    ZHA_TRY(ws_layout(cfg, n_q, t, &w));
+    ZHA_TRY(check_ws(w, ws, ws_bytes));
+    ZHA_TRY(need(K, "K"));
+    ZHA_TRY(need(V, "V"));
+    ZHA_TRY(need(Q, "Q"));
+    ZHA_TRY(need(N, "N"));
+    ZHA_TRY(need(O, "O"));
+    plan_dense_kernel<<<cfg->batch * cfg->Hkv, 256, 0, stream>>>(N, at<int2>(ws, w.off_items), at<int32_t>(ws, w.off_nitems),
+                                                                w.item_cap, cfg->N_cap, cfg->Hkv, cfg->Hq / cfg->Hkv);
+    ZHA_TRY(check_launch("plan_dense"));
+    return ZHA_DISPATCH(cfg, run_attend, cfg, w, K, V, Q, O, ws, stream);
+}
+
+int zha_get_status(int32_t* status_bits, int32_t clear, zha_stream_t stream) {
+    ZHA_TRY(need(status_bits, "status_bits"));
+    ZHA_CUDA(cudaStreamSynchronize(stream));
+    int v = 0;
+    ZHA_CUDA(cudaMemcpyFromSymbol(&v, g_status, sizeof v));
+    if (clear) {
+        const int z = 0;
+        ZHA_CUDA(cudaMemcpyToSymbol(g_status, &z, sizeof z));
+    }
+    *status_bits = v;
+    return ZHA_OK;
+}
+
+const char* zha_last_error(void) { return g_err; }
+
+}  // extern "C"

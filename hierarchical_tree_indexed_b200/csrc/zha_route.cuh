@@ -1,0 +1,366 @@
+// zha_route.cuh -- top-down top-p routing of decode queries.
+//
+// Page: [HTI] "Subquadratic Attention with a Hierarchical Tree-Structured
+// Indexer", Methodology / Routing: at each level keep the smallest prefix of
+// the candidates, ordered by score, whose normalised mass
+//   sum_{i<=m} exp(s_i) / sum_{i<=n} exp(s_i)  reaches p  (the cut m_l(q)),
+// then pass the kept nodes' children to the next level, down to the leaf
+// blocks.  Scores are the tangent estimates s = scale * q.khat + bhat.
+//
+// One CTA walks the levels for one (sequence, query head), with no host round
+// trip.  Per level:
+//   scan   -- one warp per kept parent reads its b contiguous children (b*d fp32,
+//             float4 per lane) and reduces b dot products at once with a
+//             transpose-reduce over the warp;
+//   top-p  -- exact and deterministic: masses exp(s - s_max) become 64-bit
+//             fixed-point integers (2^-40 units), so sums are order-free; a
+//             radix select over the order-preserving 32-bit score keys finds the
+//             cut score, equal scores are taken in ascending id order (ties to
+//             the lower id), and a block scan compacts the kept ids, which stay
+//             ascending because children of ascending parents are ascending.
+#pragma once
+
+#include "zha_common.cuh"
+
+namespace zha {
+
+constexpr int kRouteThreads = 512;
+constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kScoresSmem = 16384;   // candidate scores kept in shared memory up to this count
+constexpr int kParentsSmem = 4096;   // per buffer; larger lists live in the workspace
+
+struct RouteArgs {
+    TreeDev tree;
+    const void* Q;          // [batch][n_q][Hq][d]
+    const int32_t* N;       // [batch]
+    int32_t* sel;           // [batch][n_q][Hq][sel_cap]
+    int32_t* sel_count;     // [batch][n_q][Hq]
+    float* ws_scores;       // [batch*Hq][cand_cap]
+    int32_t* ws_parents;    // [batch*Hq][2][par_cap]
+    int64_t cand_cap, par_cap, N_cap;
+    int sel_cap, batch, Hq, Hkv, B, b, L_fixed, n_q;
+    float scale;
+    float p[kMaxLevels];
+};
+
+struct RouteSmem {
+    float scores[kScoresSmem];
+    int32_t parents[2][kParentsSmem];
+    unsigned long long hist_mass[256];
+    uint32_t hist_cnt[256];
+    float q[128];
+    int scan[kRouteWarps + 1];
+    float redf[kRouteWarps];
+    unsigned long long redu[kRouteWarps];
+    uint32_t redk[2][kRouteWarps];
+    int digit;
+    uint32_t digit_cnt;
+    unsigned long long digit_above, digit_mass;
+};
+
+// Order-preserving key of a finite float (larger score -> larger key); -0 == +0.
+__device__ __forceinline__ uint32_t score_key(float s) {
+    const uint32_t u = __float_as_uint(s + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ unsigned long long score_mass(float s, float smax) {
+    return __float2ull_rn(expf(s - smax) * 1099511627776.0f);   // 2^40
+}
+
+// Top-p over sc[0..nc) (invalid slots hold -inf).  Writes the kept node ids,
+// ascending, to out and returns their count.  node_of(i) maps a slot to its id.
+template <typename NodeOf>
+__device__ int top_p_select(const float* sc, int nc, float p, int32_t* out, RouteSmem& sm, NodeOf node_of) {
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    // 1. max score and key range
+    float mx = -INFINITY;
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int i = tid; i < nc; i += kRouteThreads) {
+        const float s = sc[i];
+        if (s != -INFINITY) {
+            mx = fmaxf(mx, s);
+            const uint32_t k = score_key(s);
+            kmin = min(kmin, k);
+            kmax = max(kmax, k);
+        }
+    }
+    mx = warp_max(mx);
+    kmin = warp_min_u32(kmin);
+    kmax = warp_max_u32(kmax);
+    if (lane == 0) { sm.redf[w] = mx; sm.redk[0][w] = kmin; sm.redk[1][w] = kmax; }
+    __syncthreads();
+    mx = -INFINITY; kmin = 0xffffffffu; kmax = 0u;
+    for (int i = 0; i < kRouteWarps; ++i) {
+        mx = fmaxf(mx, sm.redf[i]);
+        kmin = min(kmin, sm.redk[0][i]);
+        kmax = max(kmax, sm.redk[1][i]);
+    }
+    __syncthreads();
+    if (mx == -INFINITY) return 0;   // no candidates
+
+    const bool keep_all = p >= 1.0f;
+    uint32_t prefix = 0, pmask = 0;
+    unsigned long long take = 0;     // how many of the tie group (key & pmask == prefix) to keep
+    bool all_ties = true;
+    if (!keep_all) {
+        // 2. fixed-point masses and the target
+        unsigned long long tot = 0;
+        for (int i = tid; i < nc; i += kRouteThreads) {
+            const float s = sc[i];
+            if (s != -INFINITY) tot += score_mass(s, mx);
+        }
+        tot = warp_sum_u64(tot);
+        if (lane == 0) sm.redu[w] = tot;
+        __syncthreads();
+        tot = 0;
+        for (int i = 0; i < kRouteWarps; ++i) tot += sm.redu[i];
+        __syncthreads();
+        unsigned long long target =
+            static_cast<unsigned long long>(ceil(static_cast<double>(p) * static_cast<double>(tot)));
+        if (target < 1) target = 1;
+        if (target > tot) target = tot;
+
+        // 3. radix select of the cut key, 8 bits at a time below the highest differing bit
+        unsigned long long above = 0;
+        const int hb = (kmin == kmax) ? -1 : 31 - __clz(kmin ^ kmax);
+        pmask = hb < 0 ? 0xffffffffu : (hb >= 31 ? 0u : ~((2u << hb) - 1u));
+        prefix = kmax & pmask;
+        unsigned long long tie_mass = 0;
+        uint32_t tie_cnt = 0;
+        bool unique = false;
+        for (int top = hb; top >= 0 && !unique; top -= 8) {
+            const int width = top >= 7 ? 8 : top + 1;
+            const int shift = top - width + 1;
+            const uint32_t dmask = (1u << width) - 1u;
+            if (tid < 256) { sm.hist_mass[tid] = 0; sm.hist_cnt[tid] = 0; }
+            __syncthreads();
+            for (int i = tid; i < nc; i += kRouteThreads) {
+                const float s = sc[i];
+                if (s == -INFINITY) continue;
+                const uint32_t k = score_key(s);
+                if ((k & pmask) != prefix) continue;
+                const uint32_t dg = (k >> shift) & dmask;
+                atomicAdd(&sm.hist_cnt[dg], 1u);
+                atomicAdd(&sm.hist_mass[dg], score_mass(s, mx));
+            }
+            __syncthreads();
+            if (w == 0) {
+                // lane j owns digits [8j, 8j+8); find the highest digit where the
+                // cumulative mass from the top first reaches the target.
+                unsigned long long ls = 0;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) ls += sm.hist_mass[lane * 8 + k];
+                unsigned long long suf = ls;   // inclusive suffix sum over lanes >= lane
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const unsigned long long y = __shfl_down_sync(0xffffffffu, suf, o);
+                    if (lane + o < 32) suf += y;
+                }
+                const bool reach = above + suf >= target;
+                const uint32_t bal = __ballot_sync(0xffffffffu, reach);
+                const int J = 31 - __clz(bal);                 // lane 0 always reaches
+                const unsigned long long sufJ1 = __shfl_sync(0xffffffffu, suf - ls, J);
+                if (lane == J) {
+                    unsigned long long run = above + sufJ1;
+                    int dsel = lane * 8;
+                    for (int k = 7; k >= 0; --k) {
+                        const unsigned long long mk = sm.hist_mass[lane * 8 + k];
+                        if (run + mk >= target) { dsel = lane * 8 + k; break; }
+                        run += mk;
+                    }
+                    sm.digit = dsel;
+                    sm.digit_above = run;
+                    sm.digit_cnt = sm.hist_cnt[dsel];
+                    sm.digit_mass = sm.hist_mass[dsel];
+                }
+            }
+            __syncthreads();
+            const uint32_t dsel = static_cast<uint32_t>(sm.digit);
+            above = sm.digit_above;
+            tie_cnt = sm.digit_cnt;
+            tie_mass = sm.digit_mass;
+            prefix |= dsel << shift;
+            pmask |= dmask << shift;
+            unique = tie_cnt == 1;
+            __syncthreads();
+        }
+        if (hb < 0) {   // every candidate has the same key: one tie group
+            unsigned long long c = 0, msum = 0;
+            for (int i = tid; i < nc; i += kRouteThreads)
+                if (sc[i] != -INFINITY) { c += 1; msum += score_mass(sc[i], mx); }
+            c = warp_sum_u64(c);
+            msum = warp_sum_u64(msum);
+            if (lane == 0) { sm.redu[w] = c; sm.hist_mass[w] = msum; }
+            __syncthreads();
+            c = 0; msum = 0;
+            for (int i = 0; i < kRouteWarps; ++i) { c += sm.redu[i]; msum += sm.hist_mass[i]; }
+            __syncthreads();
+            tie_cnt = static_cast<uint32_t>(c);
+            tie_mass = msum;
+        }
+        // all members of the tie group carry the same mass (same key unless unique)
+        const unsigned long long m_tie = tie_mass / tie_cnt;
+        take = (target - above + m_tie - 1) / m_tie;
+        if (take > tie_cnt) take = tie_cnt;
+        all_ties = take == tie_cnt;
+    }
+
+    // 4. compaction in slot order: thread t owns slots [t*per, (t+1)*per)
+    const int per = (nc + kRouteThreads - 1) / kRouteThreads;
+    const int i0 = min(nc, tid * per), i1 = min(nc, i0 + per);
+    int tie_base = 0;
+    if (!keep_all && !all_ties) {
+        int c = 0;
+        for (int i = i0; i < i1; ++i) {
+            const float s = sc[i];
+            if (s != -INFINITY && (score_key(s) & pmask) == prefix) ++c;
+        }
+        int tot;
+        tie_base = block_exclusive_scan<kRouteWarps>(c, sm.scan, &tot);
+    }
+    auto kept = [&](int i, int& tie_rank) -> bool {
+        const float s = sc[i];
+        if (s == -INFINITY) return false;
+        if (keep_all) return true;
+        const uint32_t k = score_key(s) & pmask;
+        if (k > prefix) return true;
+        if (k < prefix) return false;
+        return static_cast<unsigned long long>(tie_rank++) < take;
+    };
+    int c = 0;
+    {
+        int tr = tie_base;
+        for (int i = i0; i < i1; ++i) c += kept(i, tr) ? 1 : 0;
+    }
+    int total;
+    int base = block_exclusive_scan<kRouteWarps>(c, sm.scan, &total);
+    {
+        int tr = tie_base;
+        for (int i = i0; i < i1; ++i)
+            if (kept(i, tr)) out[base++] = node_of(i);
+    }
+    __syncthreads();
+    return total;
+}
+
+// One warp scores the `cnt` (<= b <= NVR) children of one parent: rows of D fp32
+// starting at kh, biases at bh.  NVR dot products are reduced together: after
+// the halving steps lane holds row (lane >> (5 - log2 NVR)) of the block.
+template <int D, int NVR>
+__device__ __forceinline__ void scan_children(const float* __restrict__ kh, const float* __restrict__ bh,
+                                              int cnt, int b, const float* qv, float* __restrict__ out) {
+    constexpr int VF = D / 32;
+    const int lane = threadIdx.x & 31;
+    float v[NVR];
+#pragma unroll
+    for (int r = 0; r < NVR; ++r) {
+        float x[VF];
+        if (r < cnt) {
+            load_n<float, VF>(kh + static_cast<int64_t>(r) * D + lane * VF, x);
+        } else {
+#pragma unroll
+            for (int e = 0; e < VF; ++e) x[e] = 0.f;
+        }
+        float d = 0.f;
+#pragma unroll
+        for (int e = 0; e < VF; ++e) d = fmaf(qv[e], x[e], d);
+        v[r] = d;
+    }
+    constexpr int H = NVR == 32 ? 5 : NVR == 16 ? 4 : NVR == 8 ? 3 : NVR == 4 ? 2 : 1;
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {
+        const int o = 16 >> step;
+        if (step < H) {
+            const int half = NVR >> (step + 1);
+            const bool upper = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < NVR / 2; ++i) {
+                if (i < half) {
+                    const float send = upper ? v[i] : v[i + half];
+                    const float keep = upper ? v[i + half] : v[i];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                }
+            }
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+        }
+    }
+    constexpr int low = 5 - H;
+    if ((lane & ((1 << low) - 1)) == 0) {
+        const int r = (lane >> low) & (NVR - 1);
+        if (r < b) out[r] = r < cnt ? v[0] + bh[r] : -INFINITY;
+    }
+}
+
+// One CTA per (sequence, query head): the whole top-down walk of one decode query.
+// NVR = b rounded up to a power of two (4, 8, 16 or 32).
+template <typename T, int D, int NVR>
+__global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArgs a) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    RouteSmem& sm = *reinterpret_cast<RouteSmem*>(smem_raw);
+    constexpr int VF = D / 32;   // fp32 summary elements per lane
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int cta = blockIdx.x;
+    const int s = cta / a.Hq, hq = cta % a.Hq;
+    const int kv = hq / (a.Hq / a.Hkv);
+    const int64_t slice = static_cast<int64_t>(s) * a.Hkv + kv;
+    const int64_t row = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + hq;
+    const int64_t N = a.N[s];
+    const int64_t Ntree = a.tree.n_tree[s];
+    if (N < 1 || N > a.N_cap || Ntree > N || Ntree < 0) {
+        if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.sel_count[row] = 0; }
+        return;
+    }
+    if (tid < D) sm.q[tid] = to_f32(static_cast<const T*>(a.Q)[row * D + tid]) * a.scale;
+    int64_t n[kMaxLevels];
+    const int L = tree_levels(Ntree, a.B, a.b, a.L_fixed, n);
+    float qv[VF];
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < VF; ++e) qv[e] = sm.q[lane * VF + e];
+
+    const int b = a.b;
+    float* ws_sc = a.ws_scores + static_cast<int64_t>(cta) * a.cand_cap;
+    int32_t* ws_par = a.ws_parents + static_cast<int64_t>(cta) * 2 * a.par_cap;
+    int32_t* bufs[4] = {sm.parents[0], sm.parents[1], ws_par, ws_par + a.par_cap};
+    int cur = 0;   // index into bufs
+
+    // virtual parents of the top level: parent i has children [i*b, i*b+b) of level L
+    int np = static_cast<int>((n[L - 1] + b - 1) / b);
+    if (np > kParentsSmem) cur = 2;
+    for (int i = tid; i < np; i += kRouteThreads) bufs[cur][i] = i;
+    __syncthreads();
+
+    for (int l = L; l >= 1; --l) {
+        const int64_t nl = n[l - 1];
+        const int nc = np * b;
+        float* sc = nc <= kScoresSmem ? sm.scores : ws_sc;
+        const int32_t* par = bufs[cur];
+        const int64_t ncap = a.tree.ncap[l - 1];
+        const float* kh = a.tree.khat[l - 1] + slice * ncap * D;
+        const float* bh = a.tree.bhat[l - 1] + slice * ncap;
+        // ---- scan: one warp per kept parent, its b child rows of D fp32
+        for (int pi = w; pi < np; pi += kRouteWarps) {
+            const int64_t c0 = static_cast<int64_t>(par[pi]) * b;
+            const int cnt = static_cast<int>(min(static_cast<int64_t>(b), nl - c0));
+            scan_children<D, NVR>(kh + c0 * D, bh + c0, cnt, b, qv, sc + static_cast<int64_t>(pi) * b);
+        }
+        __syncthreads();
+        // ---- top-p cut and compaction of the kept node ids
+        const int nxt = nc <= kParentsSmem ? (cur == 0 ? 1 : 0) : (cur == 2 ? 3 : 2);
+        np = top_p_select(sc, nc, a.p[l - 1], bufs[nxt], sm,
+                          [par, b](int i) { return static_cast<int32_t>(par[i / b] * b + i % b); });
+        cur = nxt;
+    }
+    // ---- level-1 selection -> sel
+    const int32_t* fin = bufs[cur];
+    int32_t* out = a.sel + row * a.sel_cap;
+    const int ncopy = min(np, a.sel_cap);
+    for (int i = tid; i < ncopy; i += kRouteThreads) out[i] = fin[i];
+    if (tid == 0) {
+        a.sel_count[row] = np;
+        if (np > a.sel_cap) raise_status(ZHA_ERR_CAPACITY);
+    }
+}
+
+}  // namespace zha

@@ -1,0 +1,186 @@
+/*
+ * zha.h -- C ABI of the tree-indexed sparse attention library for NVIDIA B200
+ * (sm_100a).
+ *
+ * The library computes the data-parallel hot path of Zyphra Hierarchical
+ * Attention (ZHA) as described on two pages, cited below as
+ *   [HTI] "Subquadratic Attention with a Hierarchical Tree-Structured Indexer"
+ *   [EoQ] "Zyphra Hierarchical Attention: The End of Quadratic Attention?"
+ * The path has three steps: build a tree of recursively compressed key
+ * summaries over a KV cache ([HTI] Methodology / Tree Construction), route
+ * each query top-down through it with top-p selection at every level ([HTI]
+ * Methodology / Routing, m_l(q)), and run exact softmax attention over the
+ * selected keys plus the sink token and the current chunk ([HTI] Routing,
+ * I(q) and o(q)).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Pointers named K, V, Q, O, N, tree, ws, sel, sel_count, k_new, v_new,
+ *   Qref are DEVICE pointers owned by the caller.  `cfg` is a HOST pointer.
+ *   The library allocates no device memory: every call works inside the
+ *   buffers it is given, on the caller's `stream`, asynchronously.
+ * - Layouts (row-major, innermost last):
+ *     K, V   [batch][Hkv][N_cap][d]     dtype = cfg->dtype
+ *     Q, O   [batch][n_q][Hq][d]        Q in cfg->dtype, O always fp32
+ *     Qref   [Hkv][levels][R][d] fp32   levels >= zha_levels_cap(cfg)
+ *     N      [batch] int32              keys held in the cache per sequence
+ *     sel    [batch][n_q][Hq][sel_cap] int32, sel_count [batch][n_q][Hq] int32
+ *   Query head h reads KV head h / (Hq/Hkv) (grouped-query attention).
+ * - Every function returns a zha_status.  Host-side checks (bad arguments,
+ *   unsupported shapes, a workspace that is too small) return at once and
+ *   launch nothing.  Errors found on the device (a full cache, a selection
+ *   larger than sel_cap, a bounded wait that ran out) set bits of a sticky
+ *   device status word instead; zha_get_status() reads it.  zha_last_error()
+ *   returns the message of the calling thread's last failed call.
+ * - Device code never traps, asserts or waits without a bound.
+ */
+#ifndef ZHA_H
+#define ZHA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st *zha_stream_t;
+
+#define ZHA_MAX_LEVELS 16
+
+typedef enum {
+    ZHA_OK = 0,
+    ZHA_ERR_INVALID_ARG = 1,  /* null pointer, bad size or inconsistent config       */
+    ZHA_ERR_UNSUPPORTED = 2,  /* valid but not built: d not in {64,128}, R > 1, ...    */
+    ZHA_ERR_CAPACITY = 3,     /* device: cache full (N == N_cap) or sel_cap exceeded   */
+    ZHA_ERR_CUDA = 4,         /* a CUDA runtime call failed (message in last_error)    */
+    ZHA_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up (the call returned)    */
+    ZHA_ERR_WORKSPACE = 6     /* ws_bytes smaller than zha_workspace_bytes()           */
+} zha_status;
+
+typedef enum { ZHA_F32 = 0, ZHA_BF16 = 1 } zha_dtype;
+
+/*
+ * Geometry and precision.  B = leaf block (keys summarised by one level-1
+ * node), b = branching factor (children per node above level 1).  The tree
+ * over N keys has n_1 = floor(N/B) leaf nodes (complete blocks only) and
+ * n_{l+1} = ceil(n_l / b); its depth is the first level with n_L <= b, or
+ * exactly L_fixed levels when L_fixed > 0 (the pages' C4-L6 style).  p[l-1]
+ * is the top-p threshold of level l ([HTI] Routing); p >= 1 keeps every
+ * candidate.  scale = 0 means 1/sqrt(d).
+ */
+typedef struct zha_config {
+    int32_t d;        /* head dim: 64 or 128                                  */
+    int32_t Hq;       /* query heads                                          */
+    int32_t Hkv;      /* KV heads; Hq/Hkv in {1, 2, 4}                        */
+    int32_t B;        /* leaf block, 1..64                                    */
+    int32_t b;        /* branching factor, 2..32                              */
+    int32_t R;        /* reference queries per node (GPU path: 1)             */
+    int32_t dtype;    /* zha_dtype of K, V, Q, k_new, v_new                   */
+    int32_t batch;    /* sequences                                            */
+    int64_t N_cap;    /* rows allocated per (sequence, KV head) in K and V    */
+    int32_t L_fixed;  /* 0 = depth rule, else the fixed number of levels      */
+    float scale;      /* softmax scale; 0 = 1/sqrt(d)                         */
+    float p[ZHA_MAX_LEVELS];
+} zha_config;
+
+/* Levels the tree can reach for any N <= N_cap (Qref must hold this many). */
+int zha_levels_cap(const zha_config *cfg, int32_t *levels);
+
+/* Bytes of the tree buffer for cfg (summaries of every level up to N_cap,
+ * the reference queries, per-sequence counters). */
+int zha_tree_bytes(const zha_config *cfg, size_t *bytes);
+
+/* Where level `level` (1 = leaf blocks) lives inside the tree buffer: byte
+ * offsets of its khat [batch][Hkv][nodes_cap][R][d] fp32 and bhat
+ * [batch][Hkv][nodes_cap][R] fp32 arrays, and nodes_cap.  For inspection. */
+int zha_tree_level(const zha_config *cfg, int32_t level, size_t *khat_offset, size_t *bhat_offset,
+                   int64_t *nodes_cap);
+
+/* Byte offset of the per-sequence count of indexed keys, int32 [batch]. */
+int zha_tree_count_offset(const zha_config *cfg, size_t *offset);
+
+/* Bytes of the workspace that zha_route/zha_attend/zha_decode/zha_dense need
+ * for n_q queries per sequence (decode: n_q = 1).  The workspace must be
+ * zeroed once after allocation (zha_workspace_init); calls leave it reusable. */
+int zha_workspace_bytes(const zha_config *cfg, int32_t n_q, size_t *bytes);
+int zha_workspace_init(const zha_config *cfg, void *ws, size_t ws_bytes, zha_stream_t stream);
+
+/*
+ * zha_build -- build the whole tree over keys [0, N[s]) of every sequence s.
+ * [HTI] Tree Construction: each complete block of B keys gets, for its
+ * reference query qhat, the tangent of F_C(q) = LSE_j(q.k_j * scale) at qhat:
+ * khat = softmax(scale qhat.K) K and bhat = F_C(qhat) - scale qhat.khat.
+ * Upper levels are "constructed recursively from their children's
+ * summaries": each child is a pseudo-key of log-mass scale q.khat_c + bhat_c,
+ * and the node is the tangent of their LSE at the level's reference query.
+ * Qref is copied into the tree.  N is read on the device.
+ */
+int zha_build(const zha_config *cfg, const void *K, const float *Qref, const int32_t *N,
+              void *tree, zha_stream_t stream);
+
+/*
+ * zha_append -- decode-time growth ([EoQ] "the tree is built on the fly as the
+ * context grows").  For every sequence s, writes k_new[s][h], v_new[s][h]
+ * (layout [batch][Hkv][d]) at row N[s] of K and V, increments N[s], and, when
+ * that completes a leaf block, summarises the block and recomputes its
+ * ancestors (adding a level when the top outgrows b).  The result is bitwise
+ * equal to zha_build at the new N.  A full cache (N == N_cap) sets
+ * ZHA_ERR_CAPACITY in the device status and leaves that sequence unchanged.
+ */
+int zha_append(const zha_config *cfg, void *K, void *V, const void *k_new, const void *v_new,
+               int32_t *N, void *tree, zha_stream_t stream);
+
+/*
+ * zha_route -- top-down top-p routing of decode queries (n_q = 1, query at
+ * position t = N[s]-1).  [HTI] Routing: level L's candidates are all its
+ * nodes; each candidate scores s = scale q.khat + bhat; the kept set is the
+ * smallest prefix, in descending score order (ties to the lower node id), whose
+ * normalised mass reaches p_l; the children of kept nodes are the next
+ * level's candidates.  Writes the kept level-1 block ids of every (sequence,
+ * query head), ascending, to sel (capacity sel_cap per row) and their count to
+ * sel_count.  A count above sel_cap sets ZHA_ERR_CAPACITY on the device (the
+ * first sel_cap ids are written).
+ */
+int zha_route(const zha_config *cfg, const void *tree, const void *Q, int32_t n_q, const int32_t *N,
+              int32_t *sel, int32_t *sel_count, int32_t sel_cap, void *ws, size_t ws_bytes,
+              zha_stream_t stream);
+
+/*
+ * zha_attend -- exact softmax attention over I(q) = {0} u (keys of the listed
+ * level-1 blocks) u C_cur(t) ([HTI] Routing, I(q) and o(q) = Attn(q, K_I, V_I);
+ * the first token is the sink, [EoQ]).  C_cur(t) = [min(floor(t/B), n_1)*B, t]
+ * with n_1 the number of leaf blocks in the tree.  n_q = 1 (decode, t =
+ * N[s]-1).  The blocks of the query heads that share a KV head are loaded once.
+ * O is fp32 [batch][n_q][Hq][d].  tree is read only for n_1.
+ */
+int zha_attend(const zha_config *cfg, const void *K, const void *V, const void *tree,
+               const void *Q, int32_t n_q, const int32_t *N, const int32_t *sel,
+               const int32_t *sel_count, int32_t sel_cap, float *O, void *ws, size_t ws_bytes,
+               zha_stream_t stream);
+
+/* zha_decode -- one decode step: zha_append, then zha_route and zha_attend of
+ * the query q [batch][1][Hq][d] at its own position (t = new N - 1).  The
+ * selection goes to the workspace. */
+int zha_decode(const zha_config *cfg, void *K, void *V, void *tree, const void *q,
+               const void *k_new, const void *v_new, int32_t *N, float *O, void *ws,
+               size_t ws_bytes, zha_stream_t stream);
+
+/* zha_dense -- the in-library dense baseline: attention of q [batch][1][Hq][d]
+ * over every key [0, N[s]), with the same loader as zha_attend. */
+int zha_dense(const zha_config *cfg, const void *K, const void *V, const void *Q, int32_t n_q,
+              const int32_t *N, float *O, void *ws, size_t ws_bytes, zha_stream_t stream);
+
+/* Reads (and if clear != 0 resets) the sticky device status of the current
+ * device: bit (1 << code) for each zha_status code raised on the device since
+ * the last clear.  Synchronises `stream`. */
+int zha_get_status(int32_t *status_bits, int32_t clear, zha_stream_t stream);
+
+/* Message of the calling thread's last failed call ("" if none). */
+const char *zha_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ZHA_H */

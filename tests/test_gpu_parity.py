@@ -1,0 +1,304 @@
+"""CUDA path against the fp64 oracle, through the C ABI, on seeded inputs.
+
+Covers the tree build (every level), routing (index sets bit-exact beyond the
+margin), sparse attention (output tolerances), append against rebuild
+(bitwise), the decode step, the dense baseline, and edge cases: empty and
+ragged caches, per-sequence lengths, p = 1 and tiny p, capacity errors.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from hierarchical_tree_indexed_b200 import workloads as W
+from hierarchical_tree_indexed_b200 import zha
+from oracle import oracle as O
+from tests.zha_parity import (Decoder, Report, assert_status_clean, check_queries, compare_tree,
+                              oracle_tree)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    zha.get_status(clear=True)
+    yield
+
+
+def planted_inputs(name, batch, Hq, Hkv, d, N, N_cap, M, n_q, dtype="bf16", seed_base=0):
+    """Planted-cluster K/V/Q on the CPU with the workload generator (the same tensors feed both sides)."""
+    dt = W.torch_dtype(dtype)
+    K = torch.zeros((batch, Hkv, N_cap, d), dtype=dt)
+    V = torch.zeros_like(K)
+    Q = torch.zeros((n_q, batch, Hq, d), dtype=dt)
+    G = Hq // Hkv
+    for s in range(batch):
+        for h in range(Hkv):
+            cl = W.fill_planted_slice(name, s + seed_base, h, N, d, M, K[s, h], V[s, h], run=min(W.RUN, N // 4))
+            Q[:, s, h * G:(h + 1) * G] = W.cluster_queries(name, s + seed_base, h, G, n_q, cl).to(dt)
+    qref = W.reference_queries(name, Hkv, 1, d)
+    return K, V, Q, qref
+
+
+# ---------------------------------------------------------------- tiny fp32 workload
+
+@pytest.mark.parametrize("p", [0.9, 1.0])
+def test_tiny_workload(p):
+    data = W.tiny("cpu")
+    w = data["workload"]
+    cfg = zha.Config(d=w.d, Hq=1, Hkv=1, B=w.B, b=w.b, batch=1, N_cap=w.N, dtype="f32", p=p)
+    dec = Decoder(cfg, data["K"].cuda(), data["V"].cuda(), data["qref"].cuda(), [w.N])
+    dec.build()
+    ot = oracle_tree(data["K"][0, 0], w.N, cfg, data["qref"][0])
+    torch.cuda.synchronize()
+    compare_tree(cfg, dec.tree, ot, 0, 0)
+    rep = Report()
+    sels, cnts, outs = [], [], []
+    for i in range(w.steps):
+        Qi = data["Q"][i:i + 1].reshape(1, 1, 1, w.d).contiguous()
+        dec.route_attend(Qi.cuda())
+        sel, cnt, o = dec.results()
+        sels.append(sel[0, 0, 0].numpy())
+        cnts.append(int(cnt[0, 0, 0]))
+        outs.append(o[0, 0, 0].numpy())
+    check_queries(cfg, ot, data["K"][0, 0], data["V"][0, 0], w.N - 1, data["Q"][:, 0, 0], sels, cnts, outs,
+                  p, rep)
+    rep.check()
+    assert rep.exact_required >= 6, rep
+    if p == 1.0:
+        for i in range(w.steps):
+            assert cnts[i] == w.N // w.B
+            dense = O.dense(data["Q"][i, 0, 0], data["K"][0, 0], data["V"][0, 0], w.N - 1)
+            assert np.max(np.abs(outs[i] - dense)) <= 1e-3
+    assert_status_clean()
+
+
+# ---------------------------------------------------------------- planted clusters, bf16, GQA
+
+@pytest.mark.parametrize("d,G,dtype", [(128, 4, "bf16"), (64, 2, "bf16"), (128, 1, "f32"), (64, 4, "f32")])
+def test_planted_route_attend(d, G, dtype):
+    batch, Hkv = 2, 2
+    Hq = G * Hkv
+    N = [70000 + 37, 51234]                      # ragged tails, different lengths
+    N_cap = 70144
+    K, V, Q, qref = planted_inputs("test", batch, Hq, Hkv, d, max(N), N_cap, 48, 3, dtype)
+    # the second sequence only holds its first N[1] keys
+    K[1, :, N[1]:] = 0
+    V[1, :, N[1]:] = 0
+    cfg = zha.Config(d=d, Hq=Hq, Hkv=Hkv, B=64, b=16, batch=batch, N_cap=N_cap, dtype=dtype, p=0.95)
+    dec = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), N)
+    dec.build()
+    trees = {}
+    for s in range(batch):
+        for h in range(Hkv):
+            trees[(s, h)] = oracle_tree(K[s, h], N[s], cfg, qref[h])
+    torch.cuda.synchronize()
+    for (s, h), ot in trees.items():
+        compare_tree(cfg, dec.tree, ot, s, h)
+    rep = Report()
+    for step in range(Q.shape[0]):
+        Qs = Q[step].reshape(batch, 1, Hq, d).contiguous()
+        dec.route_attend(Qs.cuda())
+        sel, cnt, o = dec.results()
+        for s in range(batch):
+            for hq in range(Hq):
+                h = hq // G
+                check_queries(cfg, trees[(s, h)], K[s, h], V[s, h], N[s] - 1, Qs[s, 0, hq:hq + 1],
+                              [sel[s, 0, hq].numpy()], [int(cnt[s, 0, hq])], [o[s, 0, hq].numpy()], 0.95, rep)
+    rep.check()
+    assert rep.exact_required >= rep.queries // 2, rep
+    assert_status_clean()
+
+
+def test_p_one_and_tiny_p():
+    batch, Hkv, G, d = 1, 1, 4, 128
+    N = 9000
+    K, V, Q, qref = planted_inputs("test", batch, G * Hkv, Hkv, d, N, N, 8, 1)
+    for p, expect in [(1.0, N // 64), (1e-6, None)]:
+        cfg = zha.Config(d=d, Hq=G, Hkv=Hkv, B=64, b=16, batch=batch, N_cap=N, p=p)
+        dec = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), [N])
+        dec.build()
+        dec.route_attend(Q[0].reshape(1, 1, G, d).contiguous().cuda())
+        sel, cnt, o = dec.results()
+        ot = oracle_tree(K[0, 0], N, cfg, qref[0])
+        rep = Report()
+        check_queries(cfg, ot, K[0, 0], V[0, 0], N - 1, Q[0, 0], [sel[0, 0, h].numpy() for h in range(G)],
+                      [int(cnt[0, 0, h]) for h in range(G)], [o[0, 0, h].numpy() for h in range(G)], p, rep)
+        rep.check()
+        if expect is not None:
+            assert all(int(cnt[0, 0, h]) == expect for h in range(G))
+            for h in range(G):
+                dense = O.dense(Q[0, 0, h], K[0, 0], V[0, 0], N - 1)
+                assert np.max(np.abs(o[0, 0, h].numpy() - dense)) <= 2e-2 * np.max(np.abs(dense))
+        else:   # p -> 0 keeps exactly one node per level
+            assert all(int(cnt[0, 0, h]) == 1 for h in range(G))
+    assert_status_clean()
+
+
+@pytest.mark.parametrize("N", [1, 17, 63, 64, 65, 128, 1000, 1024])
+def test_short_caches(N):
+    """No complete block, exactly one, block boundaries: I(q) falls back to the sink and C_cur."""
+    d, G = 128, 4
+    N_cap = 1100
+    K, V, Q, qref = planted_inputs("test", 1, G, 1, d, N, N_cap, 2, 1)
+    cfg = zha.Config(d=d, Hq=G, Hkv=1, B=64, b=16, batch=1, N_cap=N_cap, p=0.9)
+    dec = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), [N])
+    dec.build()
+    dec.route_attend(Q[0].reshape(1, 1, G, d).contiguous().cuda())
+    sel, cnt, o = dec.results()
+    ot = oracle_tree(K[0, 0], N, cfg, qref[0])
+    rep = Report()
+    check_queries(cfg, ot, K[0, 0], V[0, 0], N - 1, Q[0, 0], [sel[0, 0, h].numpy() for h in range(G)],
+                  [int(cnt[0, 0, h]) for h in range(G)], [o[0, 0, h].numpy() for h in range(G)], 0.9, rep)
+    rep.check()
+    assert_status_clean()
+
+
+# ---------------------------------------------------------------- append == rebuild
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_append_matches_rebuild_bitwise(dtype, d):
+    """Appending tokens one by one gives the same tree, bit for bit, as building at the new N,
+    across block completions and a growth of the depth (n_1: 16 -> 17 with b = 4)."""
+    batch, Hkv, G, B, b = 2, 2, 2, 16, 4
+    N0, steps, N_cap = 250, 40, 320
+    K, V, Q, qref = planted_inputs("test", batch, G * Hkv, Hkv, d, N0 + steps, N_cap, 2, 1, dtype)
+    cfg = zha.Config(d=d, Hq=G * Hkv, Hkv=Hkv, B=B, b=b, batch=batch, N_cap=N_cap, dtype=dtype, p=0.9)
+    Kd, Vd = K.clone(), V.clone()
+    Kd[:, :, N0:] = 0
+    Vd[:, :, N0:] = 0
+    dec = Decoder(cfg, Kd.cuda(), Vd.cuda(), qref.cuda(), [N0, N0])
+    dec.build()
+    ref = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), [N0, N0])
+    L0 = len(O.levels(N0, B, b))
+    grew = False
+    for i in range(steps):
+        kn = K[:, :, N0 + i].contiguous().cuda()
+        vn = V[:, :, N0 + i].contiguous().cuda()
+        zha.append(cfg, dec.K, dec.V, kn, vn, dec.N, dec.tree)
+        n_now = N0 + i + 1
+        ref.N.fill_(n_now)
+        ref.tree.zero_()
+        ref.build()
+        torch.cuda.synchronize()
+        assert dec.N.tolist() == [n_now, n_now]
+        assert torch.equal(zha.tree_count_view(cfg, dec.tree).cpu(), torch.tensor([n_now] * batch, dtype=torch.int32))
+        lv = O.levels(n_now, B, b)
+        grew |= len(lv) > L0
+        for l in range(1, len(lv) + 1):
+            ka, ba = zha.tree_level_view(cfg, dec.tree, l)
+            kb, bb = zha.tree_level_view(cfg, ref.tree, l)
+            n = lv[l - 1]
+            assert torch.equal(ka[:, :, :n], kb[:, :, :n]), (i, l)
+            assert torch.equal(ba[:, :, :n], bb[:, :, :n]), (i, l)
+    assert grew
+    assert torch.equal(dec.K.cpu()[:, :, :N0 + steps], K[:, :, :N0 + steps])
+    assert torch.equal(dec.V.cpu()[:, :, :N0 + steps], V[:, :, :N0 + steps])
+    assert_status_clean()
+
+
+# ---------------------------------------------------------------- decode step
+
+def test_decode_steps_against_oracle():
+    """zha_decode (append + route + attend) for several steps, each against the oracle at the new N."""
+    batch, Hkv, G, d = 1, 2, 4, 128
+    N0, steps = 4096 - 3, 6                      # crosses a block boundary at step 3
+    N_cap = N0 + steps
+    K, V, Q, qref = planted_inputs("test", batch, G * Hkv, Hkv, d, N0 + steps, N_cap, 4, steps)
+    cfg = zha.Config(d=d, Hq=G * Hkv, Hkv=Hkv, B=64, b=16, batch=batch, N_cap=N_cap, p=0.95)
+    Kd, Vd = K.clone(), V.clone()
+    Kd[:, :, N0:] = 0
+    Vd[:, :, N0:] = 0
+    dec = Decoder(cfg, Kd.cuda(), Vd.cuda(), qref.cuda(), [N0])
+    dec.build()
+    checked = 0
+    for i in range(steps):
+        q = Q[i].reshape(batch, 1, G * Hkv, d).contiguous()
+        dec.decode(q.cuda(), K[:, :, N0 + i].contiguous().cuda(), V[:, :, N0 + i].contiguous().cuda())
+        _, _, o = dec.results()
+        n_now = N0 + i + 1
+        assert dec.N.item() == n_now
+        for h in range(Hkv):
+            ot = oracle_tree(K[0, h], n_now, cfg, qref[h])
+            for g in range(G):
+                hq = h * G + g
+                rt = O.route(Q[i, 0, hq], ot, 0.95)
+                if rt.min_margin <= 1e-4:
+                    continue        # the set may legitimately differ; not comparable by output
+                idx = O.index_set(rt.sel, n_now - 1, cfg.B, ot.n[0])
+                ref_o = O.attend(Q[i, 0, hq], K[0, h], V[0, h], idx)
+                err = np.max(np.abs(o[0, 0, hq].numpy() - ref_o)) / np.max(np.abs(ref_o))
+                assert err <= 1e-3, (i, hq, err)
+                checked += 1
+    assert checked >= steps * Hkv * G // 2
+    assert_status_clean()
+
+
+def test_dense_baseline():
+    batch, Hkv, G, d = 2, 2, 4, 128
+    N = [5000, 3333]
+    K, V, Q, qref = planted_inputs("test", batch, G * Hkv, Hkv, d, max(N), max(N), 4, 1)
+    cfg = zha.Config(d=d, Hq=G * Hkv, Hkv=Hkv, B=64, b=16, batch=batch, N_cap=max(N))
+    dec = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), N)
+    Qs = Q[0].reshape(batch, 1, G * Hkv, d).contiguous()
+    dec.dense(Qs.cuda())
+    _, _, o = dec.results()
+    for s in range(batch):
+        for hq in range(G * Hkv):
+            ref = O.dense(Qs[s, 0, hq], K[s, hq // G], V[s, hq // G], N[s] - 1)
+            assert np.max(np.abs(o[s, 0, hq].numpy() - ref)) <= 1e-3 * np.max(np.abs(ref))
+    assert_status_clean()
+
+
+# ---------------------------------------------------------------- device status, determinism
+
+def test_capacity_errors_are_reported():
+    d, G = 128, 4
+    N = 3000
+    K, V, Q, qref = planted_inputs("test", 1, G, 1, d, N, N, 2, 1)
+    cfg = zha.Config(d=d, Hq=G, Hkv=1, B=64, b=16, batch=1, N_cap=N, p=1.0)
+    dec = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), [N])
+    dec.build()
+    small = torch.zeros((1, 1, G, 4), dtype=torch.int32, device="cuda")
+    zha.route(cfg, dec.tree, Q[0].reshape(1, 1, G, d).contiguous().cuda(), dec.N, small, dec.cnt, dec.ws)
+    bits = zha.get_status(clear=True)
+    assert bits & (1 << 3), zha.status_names(bits)
+    assert int(dec.cnt[0, 0, 0]) == N // 64
+    # the cache is full: append refuses and leaves N unchanged
+    zha.append(cfg, dec.K, dec.V, K[:, :, 0].contiguous().cuda(), V[:, :, 0].contiguous().cuda(), dec.N, dec.tree)
+    bits = zha.get_status(clear=True)
+    assert bits & (1 << 3)
+    assert dec.N.item() == N
+
+
+def test_invalid_arguments_raise():
+    cfg = zha.Config(d=128, Hq=4, Hkv=1, B=64, b=16, batch=1, N_cap=128)
+    ws = zha.alloc_workspace(cfg)
+    with pytest.raises(zha.ZhaError) as e:
+        zha.route(cfg, torch.zeros(16, device="cuda"), None, torch.zeros(1, dtype=torch.int32, device="cuda"),
+                  torch.zeros((1, 1, 4, 2), dtype=torch.int32, device="cuda"),
+                  torch.zeros((1, 1, 4), dtype=torch.int32, device="cuda"), ws)
+    assert e.value.code == 1
+    with pytest.raises(zha.ZhaError) as e:
+        zha.route(cfg, torch.zeros(16, device="cuda"), torch.zeros(4, device="cuda"),
+                  torch.zeros(1, dtype=torch.int32, device="cuda"),
+                  torch.zeros((1, 1, 4, 2), dtype=torch.int32, device="cuda"),
+                  torch.zeros((1, 1, 4), dtype=torch.int32, device="cuda"), ws[:16])
+    assert e.value.code == 6
+
+
+def test_deterministic():
+    batch, Hkv, G, d = 1, 2, 4, 128
+    N = 20000
+    K, V, Q, qref = planted_inputs("test", batch, G * Hkv, Hkv, d, N, N, 16, 1)
+    cfg = zha.Config(d=d, Hq=G * Hkv, Hkv=Hkv, B=64, b=16, batch=batch, N_cap=N)
+    dec = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), [N])
+    dec.build()
+    Qs = Q[0].reshape(batch, 1, G * Hkv, d).contiguous().cuda()
+    dec.route_attend(Qs)
+    a = [x.clone() for x in dec.results()]
+    dec.route_attend(Qs)
+    b = dec.results()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
