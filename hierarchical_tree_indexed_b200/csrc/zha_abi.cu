@@ -55,6 +55,7 @@ struct TreeLayout {
 struct WsLayout {
     int64_t cand_cap, par_cap, sel_cap, item_cap, words;
     size_t off_scores, off_parents, off_sel, off_count, off_items, off_nitems, off_ml, off_acc, off_counters;
+    size_t off_rows, off_cand;
     size_t total;
 };
 
@@ -141,6 +142,8 @@ int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
     w->off_ml = off;       off = align256(off + sizeof(float2) * groups * kSplitMax * G);
     w->off_acc = off;      off = align256(off + sizeof(float) * groups * kSplitMax * G * c->d);
     w->off_counters = off; off = align256(off + sizeof(uint32_t) * groups);
+    w->off_rows = off;     off = align256(off + sizeof(int32_t) * groups);
+    w->off_cand = off;     off = align256(off + sizeof(int32_t) * ctas);
     w->total = off;
     if (static_cast<size_t>(G) * w->words * 4 > 200 * 1024)
         return fail(ZHA_ERR_UNSUPPORTED, "N_cap too large for the on-chip union bitmap");
@@ -252,6 +255,7 @@ int run_route(const zha_config* c, const TreeLayout& lay, const WsLayout& wl, co
     RouteArgs a{};
     a.tree = tree_view(lay, const_cast<void*>(tree));
     a.Q = Q; a.N = N; a.sel = sel; a.sel_count = cnt;
+    a.cand = at<int32_t>(ws, wl.off_cand);
     a.ws_scores = at<float>(ws, wl.off_scores);
     a.ws_parents = at<int32_t>(ws, wl.off_parents);
     a.cand_cap = wl.cand_cap; a.par_cap = wl.par_cap; a.N_cap = c->N_cap;
@@ -305,6 +309,7 @@ int run_plan(const zha_config* c, const WsLayout& wl, const TreeLayout& lay, con
     a.n_tree = tree_view(lay, const_cast<void*>(tree)).n_tree;
     a.items = at<int2>(ws, wl.off_items);
     a.n_items = at<int32_t>(ws, wl.off_nitems);
+    a.rows = at<int32_t>(ws, wl.off_rows);
     a.item_cap = wl.item_cap; a.N_cap = c->N_cap;
     a.sel_cap = sel_cap; a.Hq = c->Hq; a.Hkv = c->Hkv; a.G = c->Hq / c->Hkv; a.B = c->B; a.n_q = 1;
     a.words = std::max<int64_t>(wl.words, 1);
@@ -382,6 +387,18 @@ int zha_workspace_bytes(const zha_config* cfg, int32_t n_q, size_t* bytes) {
     return ZHA_OK;
 }
 
+int zha_workspace_stats(const zha_config* cfg, int32_t n_q, size_t* rows_offset, size_t* cand_offset) {
+    TreeLayout t;
+    WsLayout w;
+    ZHA_TRY(need(rows_offset, "rows_offset"));
+    ZHA_TRY(need(cand_offset, "cand_offset"));
+    ZHA_TRY(tree_layout(cfg, &t));
+    ZHA_TRY(ws_layout(cfg, n_q, t, &w));
+    *rows_offset = w.off_rows;
+    *cand_offset = w.off_cand;
+    return ZHA_OK;
+}
+
 int zha_workspace_init(const zha_config* cfg, void* ws, size_t ws_bytes, zha_stream_t stream) {
     TreeLayout t;
     WsLayout w;
@@ -431,7 +448,8 @@ int zha_route(const zha_config* cfg, const void* tree, const void* Q, int32_t n_
     ZHA_TRY(need(sel, "sel"));
     ZHA_TRY(need(sel_count, "sel_count"));
     if (sel_cap < 1) return fail(ZHA_ERR_INVALID_ARG, "sel_cap=%d", sel_cap);
-    return ZHA_DISPATCH(cfg, run_route, cfg, t, w, tree, Q, N, sel, sel_count, sel_cap, ws, stream);
+    ZHA_TRY(ZHA_DISPATCH(cfg, run_route, cfg, t, w, tree, Q, N, sel, sel_count, sel_cap, ws, stream));
+    return run_plan(cfg, w, t, tree, N, sel, sel_count, sel_cap, ws, stream);
 }
 
 int zha_attend(const zha_config* cfg, const void* K, const void* V, const void* tree, const void* Q, int32_t n_q,
@@ -447,11 +465,12 @@ int zha_attend(const zha_config* cfg, const void* K, const void* V, const void* 
     ZHA_TRY(need(tree, "tree"));
     ZHA_TRY(need(Q, "Q"));
     ZHA_TRY(need(N, "N"));
-    ZHA_TRY(need(sel, "sel"));
-    ZHA_TRY(need(sel_count, "sel_count"));
     ZHA_TRY(need(O, "O"));
-    if (sel_cap < 1) return fail(ZHA_ERR_INVALID_ARG, "sel_cap=%d", sel_cap);
-    ZHA_TRY(run_plan(cfg, w, t, tree, N, sel, sel_count, sel_cap, ws, stream));
+    if (sel) {   // plan the gather from the given lists; else reuse the plan zha_route left in ws
+        ZHA_TRY(need(sel_count, "sel_count"));
+        if (sel_cap < 1) return fail(ZHA_ERR_INVALID_ARG, "sel_cap=%d", sel_cap);
+        ZHA_TRY(run_plan(cfg, w, t, tree, N, sel, sel_count, sel_cap, ws, stream));
+    }
     return ZHA_DISPATCH(cfg, run_attend, cfg, w, K, V, Q, O, ws, stream);
 }
 
@@ -486,7 +505,8 @@ int zha_dense(const zha_config* cfg, const void* K, const void* V, const void* Q
     ZHA_TRY(need(N, "N"));
     ZHA_TRY(need(O, "O"));
     plan_dense_kernel<<<cfg->batch * cfg->Hkv, 256, 0, stream>>>(N, at<int2>(ws, w.off_items), at<int32_t>(ws, w.off_nitems),
-                                                                w.item_cap, cfg->N_cap, cfg->Hkv, cfg->Hq / cfg->Hkv);
+                                                                at<int32_t>(ws, w.off_rows), w.item_cap, cfg->N_cap,
+                                                                cfg->Hkv, cfg->Hq / cfg->Hkv);
     ZHA_TRY(check_launch("plan_dense"));
     return ZHA_DISPATCH(cfg, run_attend, cfg, w, K, V, Q, O, ws, stream);
 }

@@ -49,6 +49,7 @@ struct PlanArgs {
     const int32_t* n_tree;     // [batch]
     int2* items;               // [groups][item_cap]
     int32_t* n_items;          // [groups]
+    int32_t* rows;             // [groups] keys gathered (accounting)
     int64_t item_cap, N_cap;
     int sel_cap, Hq, Hkv, G, B, n_q;
     int64_t words;             // bitmap words per head: ceil(n1cap / 32)
@@ -64,7 +65,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_decode_kernel(PlanArgs a) {
     const uint32_t all = (1u << G) - 1u;
     const int64_t N = a.N[s], Ntree = a.n_tree[s];
     if (N < 1 || N > a.N_cap || Ntree > N) {
-        if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.n_items[g] = 0; }
+        if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.n_items[g] = 0; a.rows[g] = 0; }
         return;
     }
     const int64_t t = N - 1;
@@ -109,31 +110,37 @@ __global__ void __launch_bounds__(kPlanThreads) plan_decode_kernel(PlanArgs a) {
     }
     if (tid == 0) {
         int n = total;
+        int64_t rows = static_cast<int64_t>(total) * a.B;
         if (n1 >= 1) {   // sink: key 0 for the heads whose block 0 is not in the union
             uint32_t m0 = 0;
             for (int h = 0; h < G; ++h) m0 |= (bits[h * a.words] & 1u) << h;
-            if ((m0 & all) != all) out[n++] = make_item(0, 1, all & ~m0);
+            if ((m0 & all) != all) { out[n++] = make_item(0, 1, all & ~m0); rows += 1; }
         }
         if (cb == n1)   // C_cur past the last leaf block: the keys [n1*B, t], 64 at a time
-            for (int64_t st = cb * a.B; st <= t && n < a.item_cap; st += kAttRows)
-                out[n++] = make_item(st, static_cast<int>((t - st + 1 < kAttRows ? t - st + 1 : kAttRows)), all);
+            for (int64_t st = cb * a.B; st <= t && n < a.item_cap; st += kAttRows) {
+                const int c = static_cast<int>(t - st + 1 < kAttRows ? t - st + 1 : kAttRows);
+                out[n++] = make_item(st, c, all);
+                rows += c;
+            }
         a.n_items[g] = n;
+        a.rows[g] = static_cast<int32_t>(rows);
     }
 }
 
 // Dense baseline plan: items of 64 keys covering [0, N) for every head.
-__global__ void plan_dense_kernel(const int32_t* N, int2* items, int32_t* n_items, int64_t item_cap,
-                                  int64_t N_cap, int Hkv, int G) {
+__global__ void plan_dense_kernel(const int32_t* N, int2* items, int32_t* n_items, int32_t* rows,
+                                  int64_t item_cap, int64_t N_cap, int Hkv, int G) {
     const int g = blockIdx.x, s = g / Hkv;
     const int64_t n = N[s];
     if (n < 1 || n > N_cap) {
-        if (threadIdx.x == 0) { raise_status(ZHA_ERR_INVALID_ARG); n_items[g] = 0; }
+        if (threadIdx.x == 0) { raise_status(ZHA_ERR_INVALID_ARG); n_items[g] = 0; rows[g] = 0; }
         return;
     }
+    if (threadIdx.x == 0) rows[g] = static_cast<int32_t>(n);
     const int64_t cnt = (n + kAttRows - 1) / kAttRows;
     const uint32_t all = (1u << G) - 1u;
     for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x)
-        items[g * item_cap + i] = make_item(i * kAttRows, static_cast<int>((n - i * kAttRows < kAttRows ? n - i * kAttRows : kAttRows)), all);
+        items[g * item_cap + i] = make_item(i * kAttRows, static_cast<int>(n - i * kAttRows < kAttRows ? n - i * kAttRows : kAttRows), all);
     if (threadIdx.x == 0) n_items[g] = static_cast<int32_t>(cnt);
 }
 

@@ -35,6 +35,7 @@ struct RouteArgs {
     const int32_t* N;       // [batch]
     int32_t* sel;           // [batch][n_q][Hq][sel_cap]
     int32_t* sel_count;     // [batch][n_q][Hq]
+    int32_t* cand;          // [batch][n_q][Hq] candidates scored over all levels (accounting)
     float* ws_scores;       // [batch*Hq][cand_cap]
     int32_t* ws_parents;    // [batch*Hq][2][par_cap]
     int64_t cand_cap, par_cap, N_cap;
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
     const int64_t N = a.N[s];
     const int64_t Ntree = a.tree.n_tree[s];
     if (N < 1 || N > a.N_cap || Ntree > N || Ntree < 0) {
-        if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.sel_count[row] = 0; }
+        if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.sel_count[row] = 0; a.cand[row] = 0; }
         return;
     }
     if (tid < D) sm.q[tid] = to_f32(static_cast<const T*>(a.Q)[row * D + tid]) * a.scale;
@@ -331,9 +332,14 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
     for (int i = tid; i < np; i += kRouteThreads) bufs[cur][i] = i;
     __syncthreads();
 
+    int64_t scored = 0;
     for (int l = L; l >= 1; --l) {
         const int64_t nl = n[l - 1];
         const int nc = np * b;
+        if (np > 0) {   // only the last possible parent can have fewer than b children
+            const int64_t last_parent = (nl - 1) / b;
+            scored += nc - (bufs[cur][np - 1] == last_parent ? b - (nl - last_parent * b) : 0);
+        }
         float* sc = nc <= kScoresSmem ? sm.scores : ws_sc;
         const int32_t* par = bufs[cur];
         const int64_t ncap = a.tree.ncap[l - 1];
@@ -359,6 +365,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
     for (int i = tid; i < ncopy; i += kRouteThreads) out[i] = fin[i];
     if (tid == 0) {
         a.sel_count[row] = np;
+        a.cand[row] = static_cast<int32_t>(scored);
         if (np > a.sel_cap) raise_status(ZHA_ERR_CAPACITY);
     }
 }

@@ -214,13 +214,14 @@ def background_tokens(workload: str, seq: int, kv: int, n: int, d: int, device,
 
 
 def planted(w: Workload, device="cpu", N_cap: int | None = None, seqs=None, kv_heads=None,
-            n_queries: int | None = None, run: int = RUN, beta: float = BETA) -> dict:
+            n_queries: int | None = None, run: int = RUN, beta: float = BETA, seq_base: int = 0) -> dict:
     """Generates a planted-cluster workload.
 
     Returns K, V [batch][Hkv][N_cap][d] (w.dtype), the decode queries
     Q [n_queries][batch][Hq][d] (w.dtype), the appended tokens
     k_new/v_new [n_queries][batch][Hkv][d], and the reference queries.
-    `seqs`/`kv_heads` restrict which slices are filled (others stay zero).
+    `seqs`/`kv_heads` restrict which slices are filled (others stay zero);
+    sequence s is drawn from the seeds of sequence seq_base + s.
     """
     N_cap = N_cap or (w.N + (0 if w.prefill else w.steps))
     n_queries = w.steps if n_queries is None else n_queries
@@ -235,13 +236,14 @@ def planted(w: Workload, device="cpu", N_cap: int | None = None, seqs=None, kv_h
     clusters = {}
     for s in seqs:
         for h in kv_heads:
-            cl = fill_planted_slice(w.name, s, h, w.N, w.d, w.n_clusters, K[s, h], V[s, h], run)
+            sg = seq_base + s
+            cl = fill_planted_slice(w.name, sg, h, w.N, w.d, w.n_clusters, K[s, h], V[s, h], run)
             clusters[(s, h)] = cl
             if n_queries:
                 stream = "chunk_queries" if w.prefill else "queries"
-                q = cluster_queries(w.name, s, h, w.G, n_queries, cl, beta, stream)
+                q = cluster_queries(w.name, sg, h, w.G, n_queries, cl, beta, stream)
                 Q[:, s, h * w.G:(h + 1) * w.G] = q.to(dt)
-                kn, vn = background_tokens(w.name, s, h, n_queries, w.d, device,
+                kn, vn = background_tokens(w.name, sg, h, n_queries, w.d, device,
                                            "chunk" if w.prefill else "append")
                 k_new[:, s, h] = kn.to(dt)
                 v_new[:, s, h] = vn.to(dt)

@@ -38,7 +38,7 @@ class ZhaConfig(ctypes.Structure):
                 ("p", ctypes.c_float * MAX_LEVELS)]
 
 
-EXPORTS = ["zha_levels_cap", "zha_tree_bytes", "zha_tree_level", "zha_tree_count_offset", "zha_workspace_bytes", "zha_workspace_init", "zha_build",
+EXPORTS = ["zha_levels_cap", "zha_tree_bytes", "zha_tree_level", "zha_tree_count_offset", "zha_workspace_bytes", "zha_workspace_init", "zha_workspace_stats", "zha_build",
            "zha_append", "zha_route", "zha_attend", "zha_decode", "zha_dense", "zha_get_status",
            "zha_last_error"]
 
@@ -61,6 +61,7 @@ def lib():
         "zha_tree_count_offset": [C, P],
         "zha_workspace_bytes": [C, I32, P],
         "zha_workspace_init": [C, P, SZ, P],
+        "zha_workspace_stats": [C, I32, P, P],
         "zha_build": [C, P, P, P, P, P],
         "zha_append": [C, P, P, P, P, P, P, P],
         "zha_route": [C, P, P, I32, P, P, P, I32, P, SZ, P],
@@ -174,6 +175,14 @@ def workspace_bytes(cfg: Config, n_q: int = 1) -> int:
     return v.value
 
 
+def workspace_stats_view(cfg: Config, ws: torch.Tensor, n_q: int = 1) -> tuple[torch.Tensor, torch.Tensor]:
+    """(rows [batch*Hkv] keys gathered per group, cand [batch*n_q*Hq] nodes scored per query head) int32 views."""
+    ro, co = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().zha_workspace_stats(ctypes.byref(cfg.c()), n_q, ctypes.byref(ro), ctypes.byref(co)))
+    g, c = cfg.batch * cfg.Hkv, cfg.batch * n_q * cfg.Hq
+    return (ws[ro.value:ro.value + 4 * g].view(torch.int32), ws[co.value:co.value + 4 * c].view(torch.int32))
+
+
 def alloc_tree(cfg: Config, device="cuda") -> torch.Tensor:
     return torch.zeros(tree_bytes(cfg), dtype=torch.uint8, device=device)
 
@@ -203,8 +212,10 @@ def route(cfg: Config, tree, Q, N, sel, sel_count, ws, n_q: int = 1, stream=None
 
 
 def attend(cfg: Config, K, V, tree, Q, N, sel, sel_count, O, ws, n_q: int = 1, stream=None):
+    """sel = sel_count = None: use the gather plan the last route() left in ws."""
+    sel_cap = sel.shape[-1] if sel is not None else 0
     _check(lib().zha_attend(ctypes.byref(cfg.c()), _ptr(K), _ptr(V), _ptr(tree), _ptr(Q), n_q, _ptr(N), _ptr(sel),
-                            _ptr(sel_count), sel.shape[-1], _ptr(O), _ptr(ws), ws.numel(), _stream(stream)))
+                            _ptr(sel_count), sel_cap, _ptr(O), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def decode(cfg: Config, K, V, tree, q, k_new, v_new, N, O, ws, stream=None):

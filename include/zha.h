@@ -107,6 +107,13 @@ int zha_tree_count_offset(const zha_config *cfg, size_t *offset);
 int zha_workspace_bytes(const zha_config *cfg, int32_t n_q, size_t *bytes);
 int zha_workspace_init(const zha_config *cfg, void *ws, size_t ws_bytes, zha_stream_t stream);
 
+/* Accounting left in the workspace by the last calls, for measuring the bytes
+ * the path touches: byte offsets of int32 rows[batch*Hkv] (keys gathered per
+ * (sequence, KV head) by the last zha_attend / zha_dense plan) and int32
+ * cand[batch][n_q][Hq] (tree nodes scored over all levels by the last
+ * zha_route). */
+int zha_workspace_stats(const zha_config *cfg, int32_t n_q, size_t *rows_offset, size_t *cand_offset);
+
 /*
  * zha_build -- build the whole tree over keys [0, N[s]) of every sequence s.
  * [HTI] Tree Construction: each complete block of B keys gets, for its
@@ -141,7 +148,8 @@ int zha_append(const zha_config *cfg, void *K, void *V, const void *k_new, const
  * level's candidates.  Writes the kept level-1 block ids of every (sequence,
  * query head), ascending, to sel (capacity sel_cap per row) and their count to
  * sel_count.  A count above sel_cap sets ZHA_ERR_CAPACITY on the device (the
- * first sel_cap ids are written).
+ * first sel_cap ids are written).  It also leaves in ws the gather plan of
+ * zha_attend for these selections (see zha_attend with sel == NULL).
  */
 int zha_route(const zha_config *cfg, const void *tree, const void *Q, int32_t n_q, const int32_t *N,
               int32_t *sel, int32_t *sel_count, int32_t sel_cap, void *ws, size_t ws_bytes,
@@ -153,7 +161,9 @@ int zha_route(const zha_config *cfg, const void *tree, const void *Q, int32_t n_
  * the first token is the sink, [EoQ]).  C_cur(t) = [min(floor(t/B), n_1)*B, t]
  * with n_1 the number of leaf blocks in the tree.  n_q = 1 (decode, t =
  * N[s]-1).  The blocks of the query heads that share a KV head are loaded once.
- * O is fp32 [batch][n_q][Hq][d].  tree is read only for n_1.
+ * O is fp32 [batch][n_q][Hq][d].  tree is read only for n_1.  With sel == NULL
+ * the gather plan that the last zha_route on this workspace left is used
+ * (sel_count and sel_cap are then ignored).
  */
 int zha_attend(const zha_config *cfg, const void *K, const void *V, const void *tree,
                const void *Q, int32_t n_q, const int32_t *N, const int32_t *sel,

@@ -75,6 +75,7 @@ def test_null_pointers_and_small_workspace_are_refused_on_the_host(lib):
     assert lib.zha_route(cc, 1, 1, 1, 1, 1, 1, 16, 256, need - 1, None) == 6
     assert lib.zha_route(cc, 1, 1, 2, 1, 1, 1, 16, 256, need, None) == 2     # n_q > 1: not a decode call
     assert lib.zha_attend(cc, 1, 1, 1, 1, 1, 1, 1, 1, 0, 1, 256, need, None) == 1   # sel_cap 0
+    assert lib.zha_attend(cc, 1, 1, 1, 1, 1, 1, 1, 1, 1, None, 256, need, None) == 1   # O null
     assert lib.zha_decode(cc, None, None, None, None, None, None, None, None, 256, need, None) == 1
     assert lib.zha_dense(cc, 1, 1, 1, 1, 1, 1, None, need, None) == 1
     assert "ws" in lib.zha_last_error().decode()
