@@ -55,7 +55,7 @@ struct TreeLayout {
 struct WsLayout {
     int64_t cand_cap, par_cap, sel_cap, item_cap, words;
     size_t off_scores, off_parents, off_sel, off_count, off_items, off_nitems, off_ml, off_acc, off_counters;
-    size_t off_rows, off_cand;
+    size_t off_rows, off_cand, off_sched;
     size_t total;
 };
 
@@ -144,6 +144,7 @@ int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
     w->off_counters = off; off = align256(off + sizeof(uint32_t) * groups);
     w->off_rows = off;     off = align256(off + sizeof(int32_t) * groups);
     w->off_cand = off;     off = align256(off + sizeof(int32_t) * ctas);
+    w->off_sched = off;    off = align256(off + sizeof(uint32_t) * 2);
     w->total = off;
     if (static_cast<size_t>(G) * w->words * 4 > 200 * 1024)
         return fail(ZHA_ERR_UNSUPPORTED, "N_cap too large for the on-chip union bitmap");
@@ -278,7 +279,11 @@ int run_attend_t(const AttendArgs& a, cudaStream_t st) {
     ZHA_TRY(allow_smem(kern, smem));
     DevInfo di;
     ZHA_TRY(dev_info(&di));
-    kern<<<2 * di.sms, kAttThreads, smem, st>>>(a);
+#ifndef ZHA_ATT_CTAS_PER_SM
+#define ZHA_ATT_CTAS_PER_SM 1
+#endif
+    const int grid = std::min(ZHA_ATT_CTAS_PER_SM * di.sms, kSplitMax);   // a group has at most `grid` partials
+    kern<<<grid, kAttThreads, smem, st>>>(a);
     return check_launch("attend");
 }
 

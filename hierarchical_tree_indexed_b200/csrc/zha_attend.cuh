@@ -14,13 +14,15 @@
 //              the blocks, C_cur (merged into its block when that block is in the
 //              tree, else a partial range) and the sink (key 0 for the heads whose
 //              blocks do not already hold it);
-//   attend  -- persistent split-K kernel: each CTA streams its items' K and V rows
-//              into shared memory with 1-D bulk async copies (3-stage mbarrier
-//              pipeline, 64 rows per stage), and every warp keeps an online
-//              softmax over its 8 rows of each stage for all G heads;
-//              at the end of a split the warps combine, the CTA writes one
-//              (max, sum, acc[d]) partial per head, and the last CTA of a group
-//              (atomic counter, self-resetting) merges the group's partials into O.
+//   attend  -- one CTA per SM; the concatenated item lists of all groups are cut
+//              into equal contiguous pieces, one per CTA (split-K, stream-K style).
+//              A producer warp streams the piece's K and V rows into shared memory
+//              with 1-D bulk async copies (up to 6 stages of 64 rows in flight,
+//              full/empty mbarriers); 8 consumer warps keep an online softmax over
+//              8 rows of each stage for all G heads.  At the end of each group in
+//              its piece the CTA combines its warps into one (max, sum, acc[d])
+//              partial per head; the last CTA of a group (atomic counter,
+//              self-resetting) merges the group's partials into O.
 // Scores are kept in log2 units (q pre-multiplied by scale*log2(e)).
 #pragma once
 
@@ -28,13 +30,24 @@
 
 namespace zha {
 
-constexpr int kAttThreads = 256;
-constexpr int kAttWarps = 8;
-constexpr int kAttRows = 64;          // rows per pipeline stage
-constexpr int kAttStages = 3;
-constexpr int kAttRowsPerWarp = kAttRows / kAttWarps;
-constexpr int kSplitMax = 256;        // partials per group
-constexpr int kItemsPerSplitMin = 4;
+#ifndef ZHA_ATT_STAGE_BUDGET
+#define ZHA_ATT_STAGE_BUDGET (196 * 1024)   // shared memory for the K/V stages of one CTA
+#endif
+#ifndef ZHA_ATT_CHUNK
+#define ZHA_ATT_CHUNK 0
+#endif
+#ifndef ZHA_ATT_ROTATE
+#define ZHA_ATT_ROTATE 1
+#endif
+constexpr int kAttRows = 64;                  // rows per pipeline stage
+// stages in flight per CTA: as many 64-row K+V stages as the budget holds, 2..6
+template <typename T, int D>
+constexpr int att_stages() {
+    constexpr int n = ZHA_ATT_STAGE_BUDGET / (2 * 64 * D * static_cast<int>(sizeof(T)));
+    return n < 2 ? 2 : (n > 6 ? 6 : n);
+}
+constexpr int kAttChunk = ZHA_ATT_CHUNK;      // items per round-robin chunk; 0 = one contiguous piece per CTA
+constexpr int kSplitMax = 512;        // partials per group (>= the attention grid)
 constexpr int kPlanThreads = 512;
 
 // item: x = first key, y = key count | head mask << 16
@@ -153,45 +166,67 @@ struct AttendArgs {
     const int32_t* n_items;
     float2* part_ml;           // [groups][kSplitMax][G]  (max in log2 units, sum)
     float* part_acc;           // [groups][kSplitMax][G][d]
-    uint32_t* counters;        // [groups], zero between calls
+    uint32_t* counters;        // [groups] partials done, zero between calls
     int64_t item_cap, N_cap;
     int groups, Hq, Hkv, n_q;
     float qscale;              // scale * log2(e)
 };
 
+constexpr int kAttConsumers = 8;                       // consumer warps
+constexpr int kAttThreads = 32 * (kAttConsumers + 1);  // + one producer warp
+constexpr int kAttRowsPerWarp = kAttRows / kAttConsumers;
+
 struct StageDesc {
     int n_rows;                // -1: no more work
-    int work;
-    int last;                  // last stage of this split
-    int pad;
+    int group, split;
+    int flags;                 // bit 0: last stage of this CTA's piece of the group; bit 1: first stage
+    uint32_t heads;            // union of the row masks
+    int pad[3];
     uint8_t mask[kAttRows];
 };
 
 template <typename T, int D, int G>
 struct AttSmem {
+    static constexpr int kAttStages = att_stages<T, D>();
     T k[kAttStages][kAttRows][D];
     T v[kAttStages][kAttRows][D];
-    float red[kAttWarps / 2][G][D];
-    float sw[kAttWarps][G][kAttRowsPerWarp];   // scores, per warp
-    float pw[kAttWarps][kAttRowsPerWarp][4];   // probabilities [row][head], per warp
-    float cm[kAttWarps][G], cl[kAttWarps][G];
-    int scan[kAttWarps + 1];
+    T q[kAttStages][G][D];                        // the group's queries, sent with its first stage
+    // combine scratch [kAttConsumers/2][G][D]; the group merge reuses it for 2*kSplitMax*G weights
+    static constexpr int kRed = (kAttConsumers / 2) * G * D > 2 * kSplitMax * G ? (kAttConsumers / 2) * G * D
+                                                                                : 2 * kSplitMax * G;
+    float red[kRed];
+    float sw[kAttConsumers][G][kAttRowsPerWarp];  // scores, per warp
+    float pw[kAttConsumers][kAttRowsPerWarp][4];  // probabilities [row][head], per warp
+    float cm[kAttConsumers][G], cl[kAttConsumers][G];
+    int scan[kAttConsumers + 2];
     StageDesc desc[kAttStages];
-    uint64_t bar[kAttStages];
-    int work_split, last_flag;
-    int prefix[1];                              // [groups + 1], extends past the struct
+    uint64_t full[kAttStages], empty[kAttStages];
+    int last_flag, work_split;
+    int prefix[1];                                 // [groups + 1] first global item of each group
 };
 
-__device__ __forceinline__ void split_shape(int n_items, int& per, int& splits) {
-    per = max(kItemsPerSplitMin, (n_items + kSplitMax - 1) / kSplitMax);
-    splits = n_items > 0 ? (n_items + per - 1) / per : 0;
+__device__ __forceinline__ void consumer_sync() {   // named barrier of the 8 consumer warps
+    asm volatile("bar.sync 1, %0;" ::"n"(kAttConsumers * 32) : "memory");
+}
+
+// Split of the concatenated item lists of all groups into chunks of `ch` items;
+// chunk j belongs to CTA j mod C.  A CTA's chunks inside one group are
+// consecutive in its own order, so it gives at most one partial per group,
+// stored at slot = its index; a group has min(C, chunks it spans) partials.
+__device__ __forceinline__ int64_t chunk_items(int64_t I, int C) {
+    return kAttChunk > 0 ? kAttChunk : (I + C - 1) / C;
+}
+__device__ __forceinline__ int partials_of(int64_t g0, int64_t g1, int64_t ch, int C) {
+    const int64_t j0 = g0 / ch, j1 = (g1 - 1) / ch;
+    return static_cast<int>(min(static_cast<int64_t>(C), j1 - j0 + 1));
 }
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a) {
+__global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     using Smem = AttSmem<T, D, G>;
     Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+    constexpr int kAttStages = Smem::kAttStages;
     constexpr int VEC = Elem<T>::kVec;       // elements per 16-byte row load (QK layout)
     constexpr int LPR = D / VEC;             // lanes per row
     constexpr int RPW = 32 / LPR;            // rows per load
@@ -200,130 +235,174 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a) {
     constexpr int VD = D / 32;               // PV: dims per lane
     static_assert(G * kAttRowsPerWarp <= 32, "one lane per (head, row) in the softmax");
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int sub = lane / LPR, li = lane % LPR;
 
-    // ---- split table: prefix[g] = first work id of group g
+    // ---- prefix[g] = first global item of group g (all warps)
     {
         int* pre = sm.prefix;
         int carry = 0;
         for (int base = 0; base < a.groups; base += kAttThreads) {
             const int g = base + tid;
-            int per, sp = 0;
-            if (g < a.groups) split_shape(a.n_items[g], per, sp);
+            const int n = g < a.groups ? a.n_items[g] : 0;
             int tot;
-            const int x = block_exclusive_scan<kAttWarps>(sp, sm.scan, &tot);
+            const int x = block_exclusive_scan<kAttConsumers + 1>(n, sm.scan, &tot);
             if (g < a.groups) pre[g] = carry + x;
             carry += tot;
         }
-        if (tid == 0) pre[a.groups] = carry;
         if (tid == 0) {
-            for (int i = 0; i < kAttStages; ++i) mbar_init(&sm.bar[i], 1);
+            pre[a.groups] = carry;
+            for (int i = 0; i < kAttStages; ++i) {
+                mbar_init(&sm.full[i], 1);
+                mbar_init(&sm.empty[i], kAttConsumers);
+            }
             fence_mbar_init();
         }
         __syncthreads();
     }
-    const int total_work = sm.prefix[a.groups];
-    auto group_of = [&](int work) {   // last g with prefix[g] <= work
-        int lo = 0, hi = a.groups - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (sm.prefix[mid] <= work) lo = mid; else hi = mid - 1;
-        }
-        return lo;
-    };
+    const int64_t I = sm.prefix[a.groups];
+    const int C = gridDim.x;
+    const int64_t ch = I > 0 ? chunk_items(I, C) : 1;
 
-    // ---- producer (thread 0): fills stages in work order, packing whole items
-    int pw_work = blockIdx.x, p_item = 0, p_end = 0, p_group = 0;
-    auto producer_start = [&]() {
-        if (pw_work < total_work) {
-            p_group = group_of(pw_work);
-            const int split = pw_work - sm.prefix[p_group];
-            int per, sp;
-            split_shape(a.n_items[p_group], per, sp);
-            p_item = split * per;
-            p_end = min(a.n_items[p_group], p_item + per);
-        }
-    };
-    auto fill = [&](int slot) {
-        StageDesc& d = sm.desc[slot];
-        if (pw_work >= total_work) {
-            d.n_rows = -1;
-            mbar_arrive(&sm.bar[slot]);
-            return;
-        }
-        const int2* it = a.items + static_cast<int64_t>(p_group) * a.item_cap;
-        int rows = 0, i = p_item;
-        while (i < p_end) {
-            const int c = it[i].y & 0xffff;
-            if (c < 1 || c > kAttRows) {   // never produced by the plans; skip it
-                raise_status(ZHA_ERR_INVALID_ARG);
-                if (rows == 0) { p_item = ++i; continue; }
-                break;
+    if (w == kAttConsumers) {
+        // ================= producer warp: this CTA's contiguous piece of the item lists, packed
+        // into 64-row stages; K/V rows (and each group's queries) sent by 1-D bulk copies.
+        int fills = 0;
+        bool ok = true;
+        auto acquire_slot = [&](int slot) {   // wait until the consumers released this slot
+            if (fills >= kAttStages && ok) {
+                bool got = true;
+                if (lane == 0) got = mbar_wait_bounded(&sm.empty[slot], ((fills / kAttStages) - 1) & 1);
+                ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+                if (!ok && lane == 0) raise_status(ZHA_ERR_TIMEOUT);
             }
-            if (rows + c > kAttRows) break;
-            const uint32_t m = static_cast<uint32_t>(it[i].y) >> 16;
-            for (int r = 0; r < c; ++r) d.mask[rows + r] = static_cast<uint8_t>(m);
-            rows += c;
-            ++i;
+        };
+        int g = 0;
+        int prev_g = -1;
+        for (int64_t j = blockIdx.x; j * ch < I && ok; j += C) {
+          const int64_t cx_end = min(I, (j + 1) * ch);
+          for (int64_t x = j * ch; x < cx_end && ok;) {
+            while (sm.prefix[g + 1] <= x) ++g;   // the group holding item x (groups with items only)
+            const int64_t g0 = sm.prefix[g], g1 = sm.prefix[g + 1];
+            const int64_t seg_end = min(cx_end, g1);
+            const int split = blockIdx.x;
+            const int i0 = static_cast<int>(x - g0), i1 = static_cast<int>(seg_end - g0);
+            // this CTA's run in group g ends with this chunk when its next chunk starts past the group
+            const bool run_ends = (j + C) * ch >= g1;
+            const bool run_starts = g != prev_g;
+            prev_g = g;
+            const int s = g / a.Hkv, kv = g % a.Hkv;
+            const int64_t kvbase = (static_cast<int64_t>(s) * a.Hkv + kv) * a.N_cap;
+            const T* Kb = static_cast<const T*>(a.K) + kvbase * D;
+            const T* Vb = static_cast<const T*>(a.V) + kvbase * D;
+            const T* Qg = static_cast<const T*>(a.Q) +
+                          ((static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G) * D;
+            const int2* its = a.items + static_cast<int64_t>(g) * a.item_cap;
+            bool first = run_starts;
+            // CTAs start at different points of their segments (the order of the keys does not
+            // matter to the softmax), so concurrent CTAs do not stream the same address pattern
+            const int nseg = i1 - i0;
+            const int rot = ZHA_ATT_ROTATE ? static_cast<int>((static_cast<uint32_t>(blockIdx.x) * 2654435761u) % static_cast<uint32_t>(nseg)) : 0;
+            for (int part = 0; part < 2; ++part) {
+            const int pb0 = part == 0 ? i0 + rot : i0, pb1 = part == 0 ? i1 : i0 + rot;
+            for (int base = pb0; base < pb1 && ok; base += 32) {
+                const int avail = min(32, pb1 - base);
+                int2 it = make_int2(0, 0);
+                if (lane < avail) it = its[base + lane];
+                int c = it.y & 0xffff;
+                if (lane < avail && (c < 1 || c > kAttRows)) { raise_status(ZHA_ERR_INVALID_ARG); c = 0; }
+                const uint32_t m = static_cast<uint32_t>(it.y) >> 16;
+                int pos = 0;
+                while (pos < avail && ok) {
+                    int cc = (lane >= pos && lane < avail) ? c : 0;
+                    int incl = cc;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += y;
+                    }
+                    const bool fit = lane >= pos && lane < avail && incl <= kAttRows;
+                    const int n_fit = __popc(__ballot_sync(0xffffffffu, fit));
+                    const int rows = __shfl_sync(0xffffffffu, incl, pos + n_fit - 1);
+                    const int excl = incl - cc;
+                    const uint32_t heads = warp_or(fit && cc > 0 ? m : 0u);
+                    const bool last = run_ends && pos + n_fit >= avail && base + avail >= pb1 && (part == 1 || rot == 0);
+                    const int slot = fills % kAttStages;
+                    acquire_slot(slot);
+                    if (!ok) break;
+                    StageDesc& d = sm.desc[slot];
+                    {   // every lane writes the masks of rows 2*lane, 2*lane+1: the item holding row r
+                        // is the first fitting lane whose inclusive row count exceeds r
+                        const uint32_t fitm = __ballot_sync(0xffffffffu, fit && cc > 0);
+                        uint32_t pair = 0;
+#pragma unroll
+                        for (int k = 0; k < 2; ++k) {
+                            const int r = 2 * lane + k;
+                            const uint32_t over = __ballot_sync(0xffffffffu, incl > r) & fitm;
+                            const int owner = over ? __ffs(over) - 1 : 0;
+                            const uint32_t mo = __shfl_sync(0xffffffffu, m, owner);
+                            if (over && r < rows) pair |= (mo & 0xffu) << (8 * k);
+                        }
+                        reinterpret_cast<uint16_t*>(d.mask)[lane] = static_cast<uint16_t>(pair);
+                    }
+                    if (lane == 0) {
+                        d.n_rows = rows;
+                        d.group = g;
+                        d.split = split;
+                        d.flags = (last ? 1 : 0) | (first ? 2 : 0);
+                        d.heads = heads;
+                    }
+                    __syncwarp();
+                    __threadfence_block();
+                    const uint32_t bytes = static_cast<uint32_t>(rows * D * sizeof(T) * 2 + (first ? G * D * sizeof(T) : 0));
+                    if (lane == 0) mbar_arrive_expect_tx(&sm.full[slot], bytes);
+                    __syncwarp();
+                    if (fit && cc > 0) {
+                        const int64_t st = it.x;
+                        const uint32_t nb = static_cast<uint32_t>(cc * D * sizeof(T));
+                        bulk_g2s(&sm.k[slot][excl][0], Kb + st * D, nb, &sm.full[slot]);
+                        bulk_g2s(&sm.v[slot][excl][0], Vb + st * D, nb, &sm.full[slot]);
+                    }
+                    if (first && lane == 0)
+                        bulk_g2s(&sm.q[slot][0][0], Qg, static_cast<uint32_t>(G * D * sizeof(T)), &sm.full[slot]);
+                    first = false;
+                    ++fills;
+                    pos += n_fit;
+                }
+            }
+            }
+            x = seg_end;
+          }
         }
-        d.n_rows = rows;
-        d.work = pw_work;
-        d.last = i == p_end;
-        mbar_arrive_expect_tx(&sm.bar[slot], static_cast<uint32_t>(rows * D * sizeof(T) * 2));
-        const int s = p_group / a.Hkv, kv = p_group % a.Hkv;
-        const int64_t kvbase = (static_cast<int64_t>(s) * a.Hkv + kv) * a.N_cap;
-        const T* Kb = static_cast<const T*>(a.K) + kvbase * D;
-        const T* Vb = static_cast<const T*>(a.V) + kvbase * D;
-        int r = 0;
-        for (int j = p_item; j < i; ++j) {
-            const int64_t st = it[j].x;
-            const int c = it[j].y & 0xffff;
-            if (c < 1 || c > kAttRows) continue;
-            const uint32_t bytes = static_cast<uint32_t>(c * D * sizeof(T));
-            bulk_g2s(&sm.k[slot][r][0], Kb + st * D, bytes, &sm.bar[slot]);
-            bulk_g2s(&sm.v[slot][r][0], Vb + st * D, bytes, &sm.bar[slot]);
-            r += c;
+        // sentinel: tells the consumers that no stage follows
+        const int slot = fills % kAttStages;
+        acquire_slot(slot);
+        if (lane == 0) {
+            sm.desc[slot].n_rows = -1;
+            mbar_arrive(&sm.full[slot]);
         }
-        p_item = i;
-        if (i == p_end) {
-            pw_work += gridDim.x;
-            producer_start();
-        }
-    };
-    if (tid == 0) {
-        producer_start();
-        for (int sl = 0; sl < kAttStages; ++sl) fill(sl);
+        return;
     }
 
-    // ---- consumer state (every warp)
+    // ================= consumer warps
     float qv[G][VEC];
     float m_run = -INFINITY, l_run = 0.f;      // for head (lane / 8) of this lane
     float acc[G][VD];
-    int cur_work = -1;
-
-    int it = 0;
-    bool timed_out = false;
-    for (;; ++it) {
+    const int sub = lane / LPR, li = lane % LPR;
+    for (int it = 0;; ++it) {
         const int slot = it % kAttStages;
-        const uint32_t parity = (it / kAttStages) & 1;
-        const bool ok = mbar_wait_bounded(&sm.bar[slot], parity);
-        if (__syncthreads_or(!ok)) {
-            timed_out = true;
+        if (!mbar_wait_bounded(&sm.full[slot], (it / kAttStages) & 1)) {
+            if (lane == 0) raise_status(ZHA_ERR_TIMEOUT);
             break;
         }
-        const int n_rows = sm.desc[slot].n_rows;
+        const StageDesc& d = sm.desc[slot];
+        const int n_rows = d.n_rows;
         if (n_rows < 0) break;
-        const int work = sm.desc[slot].work;
-        if (work != cur_work) {   // a new split: load q of its group, reset the state
-            cur_work = work;
-            const int g = group_of(work);
-            const int s = g / a.Hkv, kv = g % a.Hkv;
-            const T* qp = static_cast<const T*>(a.Q) +
-                          ((static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G) * D;
+        const int g = d.group, split = d.split, flags = d.flags;
+        const uint32_t heads = d.heads;
+        if (flags & 2) {   // first stage of this CTA's piece of a group: its queries, fresh state
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 float x[VEC];
-                Elem<T>::load16(qp + h * D + li * VEC, x);
+                Elem<T>::load16(&sm.q[slot][h][li * VEC], x);
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) qv[h][e] = x[e] * a.qscale;
             }
@@ -350,10 +429,12 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a) {
                 }
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
-                    float d = 0.f;
+                    float dd = 0.f;
+                    if ((heads >> h) & 1u) {
 #pragma unroll
-                    for (int e = 0; e < VEC; ++e) d = fmaf(qv[h][e], x[e], d);
-                    v[h * U + u] = d;
+                        for (int e = 0; e < VEC; ++e) dd = fmaf(qv[h][e], x[e], dd);
+                    }
+                    v[h * U + u] = dd;
                 }
             }
             // transpose-reduce over the LPR lanes of a row group
@@ -397,7 +478,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a) {
             // online softmax: lane -> (head hh = lane / 8, row rr = lane % 8)
             const int hh = lane / kAttRowsPerWarp, rr = lane % kAttRowsPerWarp;
             const int row = r0 + rr;
-            const bool valid = hh < G && row < n_rows && ((sm.desc[slot].mask[row] >> hh) & 1);
+            const bool valid = hh < G && row < n_rows && ((d.mask[row] >> hh) & 1);
             const float sv = valid ? sm.sw[w][hh < G ? hh : 0][rr] : -INFINITY;
             float mx = sv;
 #pragma unroll
@@ -428,101 +509,125 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_kernel(AttendArgs a) {
                     const float pp[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll
                     for (int h = 0; h < G; ++h)
+                        if ((heads >> h) & 1u)
 #pragma unroll
-                        for (int e = 0; e < VD; ++e) acc[h][e] = fmaf(pp[h], vv[e], acc[h][e]);
+                            for (int e = 0; e < VD; ++e) acc[h][e] = fmaf(pp[h], vv[e], acc[h][e]);
                 }
             }
         }
-        if (sm.desc[slot].last) {
-            // ---- combine the warps' states into one partial per head
-            const int g = group_of(work);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[slot]);   // this warp is done with the slot
+
+        if (flags & 1) {
+            // ---- combine the consumer warps' states into one partial per head
             if (lane % kAttRowsPerWarp == 0 && lane / kAttRowsPerWarp < G) {
                 sm.cm[w][lane / kAttRowsPerWarp] = m_run;
                 sm.cl[w][lane / kAttRowsPerWarp] = l_run;
             }
-            __syncthreads();
-            float f[G];
+            consumer_sync();
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 float M = -INFINITY;
-                for (int ww = 0; ww < kAttWarps; ++ww) M = fmaxf(M, sm.cm[ww][h]);
-                f[h] = M == -INFINITY ? 0.f : exp2f(sm.cm[w][h] - M);
+                for (int ww = 0; ww < kAttConsumers; ++ww) M = fmaxf(M, sm.cm[ww][h]);
+                const float f = M == -INFINITY ? 0.f : exp2f(sm.cm[w][h] - M);
 #pragma unroll
-                for (int e = 0; e < VD; ++e) acc[h][e] *= f[h];
+                for (int e = 0; e < VD; ++e) acc[h][e] *= f;
             }
 #pragma unroll
-            for (int half = kAttWarps / 2; half >= 1; half >>= 1) {
+            for (int half = kAttConsumers / 2; half >= 1; half >>= 1) {
                 if (w >= half && w < 2 * half)
 #pragma unroll
                     for (int h = 0; h < G; ++h)
 #pragma unroll
-                        for (int e = 0; e < VD; ++e) sm.red[w - half][h][lane * VD + e] = acc[h][e];
-                __syncthreads();
+                        for (int e = 0; e < VD; ++e) sm.red[((w - half) * G + h) * D + lane * VD + e] = acc[h][e];
+                consumer_sync();
                 if (w < half)
 #pragma unroll
                     for (int h = 0; h < G; ++h)
 #pragma unroll
-                        for (int e = 0; e < VD; ++e) acc[h][e] += sm.red[w][h][lane * VD + e];
-                __syncthreads();
+                        for (int e = 0; e < VD; ++e) acc[h][e] += sm.red[(w * G + h) * D + lane * VD + e];
+                consumer_sync();
             }
-            const int split = work - sm.prefix[g];
             if (w == 0) {
                 const int64_t pbase = (static_cast<int64_t>(g) * kSplitMax + split) * G;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     float M = -INFINITY, Lsum = 0.f;
-                    for (int ww = 0; ww < kAttWarps; ++ww) M = fmaxf(M, sm.cm[ww][h]);
+                    for (int ww = 0; ww < kAttConsumers; ++ww) M = fmaxf(M, sm.cm[ww][h]);
                     if (M != -INFINITY)
-                        for (int ww = 0; ww < kAttWarps; ++ww) Lsum += sm.cl[ww][h] * exp2f(sm.cm[ww][h] - M);
+                        for (int ww = 0; ww < kAttConsumers; ++ww) Lsum += sm.cl[ww][h] * exp2f(sm.cm[ww][h] - M);
                     if (lane == 0) a.part_ml[pbase + h] = make_float2(M, Lsum);
 #pragma unroll
                     for (int e = 0; e < VD; ++e) a.part_acc[(pbase + h) * D + lane * VD + e] = acc[h][e];
                 }
                 __threadfence();
+                __syncwarp();
+                if (lane == 0) {
+                    const int sp = partials_of(sm.prefix[g], sm.prefix[g + 1], ch, C);
+                    const uint32_t done = atomicAdd(&a.counters[g], 1u);
+                    sm.last_flag = done == static_cast<uint32_t>(sp - 1);
+                    sm.work_split = sp;
+                }
             }
-            __syncthreads();
-            if (tid == 0) {
-                int per, sp;
-                split_shape(a.n_items[g], per, sp);
-                const uint32_t done = atomicAdd(&a.counters[g], 1u);
-                sm.last_flag = done == static_cast<uint32_t>(sp - 1);
-                sm.work_split = sp;
-            }
-            __syncthreads();
+            consumer_sync();
             if (sm.last_flag) {
-                // ---- this CTA closes the group: merge its splits into O
+                // ---- this CTA closes the group: merge its partials into O.  Weights
+                // f[k][h] = exp2(m_k - M_h) go to shared memory once; every thread then
+                // sums its (head, dim) outputs over the partials with independent loads.
                 __threadfence();
                 const int sp = sm.work_split;
                 const int s = g / a.Hkv, kv = g % a.Hkv;
-                for (int x = tid; x < G * D; x += kAttThreads) {
-                    const int h = x / D, e = x % D;
-                    const int64_t pb = static_cast<int64_t>(g) * kSplitMax * G;
-                    float M = -INFINITY;
-                    for (int k = 0; k < sp; ++k) M = fmaxf(M, __ldcg(&a.part_ml[pb + k * G + h]).x);
-                    float Ls = 0.f, Os = 0.f;
-                    if (M != -INFINITY) {
-                        for (int k = 0; k < sp; ++k) {
-                            const float2 ml = __ldcg(&a.part_ml[pb + k * G + h]);
-                            const float f2 = exp2f(ml.x - M);
-                            Ls += ml.y * f2;
-                            Os += __ldcg(&a.part_acc[(pb + k * G + h) * D + e]) * f2;
-                        }
-                    }
-                    const int64_t orow = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + h;
-                    a.O[orow * D + e] = Ls > 0.f ? Os / Ls : 0.f;
+                const int ct = tid;   // 0 .. 255
+                const int64_t pb = static_cast<int64_t>(g) * kSplitMax * G;
+                const int slot0 = static_cast<int>((sm.prefix[g] / ch) % C);   // partial k sits at slot (slot0+k) % C
+                float* fw = sm.red;                      // [kSplitMax][G] weights (red is free here)
+                float* fl = fw + kSplitMax * G;          // [kSplitMax][G] partial sums
+                for (int x = ct; x < sp * G; x += kAttConsumers * 32) {
+                    const int k = x / G, h = x % G;
+                    const float2 ml = __ldcg(&a.part_ml[pb + ((slot0 + k) % C) * G + h]);
+                    fw[x] = ml.x;
+                    fl[x] = ml.y;
                 }
-                if (tid == 0) a.counters[g] = 0u;
+                consumer_sync();
+                if (w < G) {   // warp h: M_h, the weights, L_h
+                    float M = -INFINITY;
+                    for (int k = lane; k < sp; k += 32) M = fmaxf(M, fw[k * G + w]);
+                    M = warp_max(M);
+                    float Ls = 0.f;
+                    for (int k = lane; k < sp; k += 32) {
+                        const float f = M == -INFINITY ? 0.f : exp2f(fw[k * G + w] - M);
+                        fw[k * G + w] = f;
+                        Ls += f * fl[k * G + w];
+                    }
+                    Ls = warp_sum(Ls);
+                    if (lane == 0) sm.cl[0][w] = Ls;
+                }
+                consumer_sync();
+                for (int x = ct; x < G * D; x += kAttConsumers * 32) {
+                    const int h = x / D, e = x % D;
+                    const float* src = a.part_acc + (pb + h) * D + e;
+                    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+                    int k = 0;
+                    auto at_k = [&](int kk) { return src + static_cast<int64_t>((slot0 + kk) % C) * G * D; };
+                    for (; k + 4 <= sp; k += 4) {
+                        const float x0 = __ldcg(at_k(k));
+                        const float x1 = __ldcg(at_k(k + 1));
+                        const float x2 = __ldcg(at_k(k + 2));
+                        const float x3 = __ldcg(at_k(k + 3));
+                        o0 = fmaf(fw[k * G + h], x0, o0);
+                        o1 = fmaf(fw[(k + 1) * G + h], x1, o1);
+                        o2 = fmaf(fw[(k + 2) * G + h], x2, o2);
+                        o3 = fmaf(fw[(k + 3) * G + h], x3, o3);
+                    }
+                    for (; k < sp; ++k) o0 = fmaf(fw[k * G + h], __ldcg(at_k(k)), o0);
+                    const float Ls = sm.cl[0][h];
+                    const int64_t orow = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + h;
+                    a.O[orow * D + e] = Ls > 0.f ? ((o0 + o1) + (o2 + o3)) / Ls : 0.f;
+                }
+                if (ct == 0) a.counters[g] = 0u;
+                consumer_sync();   // the weights in red are reused by the next combine
             }
         }
-        __syncthreads();   // every warp is done with this slot
-        if (tid == 0) fill(slot);
-    }
-    // Leaving after a timeout: give the copies still in flight a bounded time to
-    // land before the CTA's shared memory is released.
-    if (timed_out && tid == 0) {
-        raise_status(ZHA_ERR_TIMEOUT);
-        for (int k = 0; k < kAttStages; ++k)
-            mbar_wait_bounded(&sm.bar[(it + k) % kAttStages], ((it + k) / kAttStages) & 1);
     }
 }
 

@@ -44,19 +44,19 @@ struct RouteArgs {
     float p[kMaxLevels];
 };
 
+constexpr int kTieMax = 4096;   // crossing-bin members listed in shared memory (more: found by a scan)
+
 struct RouteSmem {
     float scores[kScoresSmem];
     int32_t parents[2][kParentsSmem];
-    unsigned long long hist_mass[256];
-    uint32_t hist_cnt[256];
+    unsigned long long bin_mass[1024];
+    uint32_t bin_cnt[1024];
+    int32_t tie_slot[kTieMax];
     float q[128];
     int scan[kRouteWarps + 1];
     float redf[kRouteWarps];
-    unsigned long long redu[kRouteWarps];
-    uint32_t redk[2][kRouteWarps];
-    int digit;
-    uint32_t digit_cnt;
-    unsigned long long digit_above, digit_mass;
+    int tie_n, cut_bin;
+    unsigned long long cut_above, cut_target;
 };
 
 // Order-preserving key of a finite float (larger score -> larger key); -0 == +0.
@@ -70,176 +70,132 @@ __device__ __forceinline__ unsigned long long score_mass(float s, float smax) {
 
 // Top-p over sc[0..nc) (invalid slots hold -inf).  Writes the kept node ids,
 // ascending, to out and returns their count.  node_of(i) maps a slot to its id.
+constexpr int kBins = 1024;          // score bins of 1/32 nat below the level's max score
+constexpr float kBinsPerNat = 32.0f;
+
+__device__ __forceinline__ int score_bin(float s, float smax) {
+    const float x = (smax - s) * kBinsPerNat;   // >= 0, weakly decreasing in s
+    return x >= static_cast<float>(kBins - 1) ? kBins - 1 : static_cast<int>(x);
+}
+
+// Top-p cut over sc[0..nc) (invalid slots hold -inf): keeps the smallest prefix,
+// in descending score order with ties to the lower slot (= lower node id), whose
+// fixed-point mass reaches ceil(p * total).  Writes the kept node ids, ascending,
+// to out; returns their count.  node_of(i) maps a slot to its node id.
+//
+// One pass bins the candidates by score (bins are monotone in the score, so the
+// bin order is the sorted order up to the order inside a bin) and sums their
+// masses per bin; one warp finds the bin where the cumulative mass crosses the
+// target; only the candidates of that bin are ranked exactly (by score, then
+// slot) against each other.  Candidate i is kept iff the mass of everything
+// ordered before it is below the target.
 template <typename NodeOf>
 __device__ int top_p_select(const float* sc, int nc, float p, int32_t* out, RouteSmem& sm, NodeOf node_of) {
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    // 1. max score and key range
+    // 1. max score; clear the bins
     float mx = -INFINITY;
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-    for (int i = tid; i < nc; i += kRouteThreads) {
-        const float s = sc[i];
-        if (s != -INFINITY) {
-            mx = fmaxf(mx, s);
-            const uint32_t k = score_key(s);
-            kmin = min(kmin, k);
-            kmax = max(kmax, k);
-        }
-    }
+    for (int i = tid; i < nc; i += kRouteThreads) mx = fmaxf(mx, sc[i]);
     mx = warp_max(mx);
-    kmin = warp_min_u32(kmin);
-    kmax = warp_max_u32(kmax);
-    if (lane == 0) { sm.redf[w] = mx; sm.redk[0][w] = kmin; sm.redk[1][w] = kmax; }
+    if (lane == 0) sm.redf[w] = mx;
+    for (int k = tid; k < kBins; k += kRouteThreads) { sm.bin_mass[k] = 0; sm.bin_cnt[k] = 0; }
+    if (tid == 0) { sm.tie_n = 0; sm.cut_above = 0; sm.cut_target = 0; }
     __syncthreads();
-    mx = -INFINITY; kmin = 0xffffffffu; kmax = 0u;
-    for (int i = 0; i < kRouteWarps; ++i) {
-        mx = fmaxf(mx, sm.redf[i]);
-        kmin = min(kmin, sm.redk[0][i]);
-        kmax = max(kmax, sm.redk[1][i]);
-    }
-    __syncthreads();
-    if (mx == -INFINITY) return 0;   // no candidates
-
+    mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kRouteWarps; ++i) mx = fmaxf(mx, sm.redf[i]);
+    if (mx == -INFINITY) return 0;   // no candidates (uniform: every thread read the same partials)
     const bool keep_all = p >= 1.0f;
-    uint32_t prefix = 0, pmask = 0;
-    unsigned long long take = 0;     // how many of the tie group (key & pmask == prefix) to keep
-    bool all_ties = true;
+    int cbin = kBins;                 // keep_all: every valid candidate is "before the crossing bin"
     if (!keep_all) {
-        // 2. fixed-point masses and the target
-        unsigned long long tot = 0;
+        // 2. mass per bin
         for (int i = tid; i < nc; i += kRouteThreads) {
             const float s = sc[i];
-            if (s != -INFINITY) tot += score_mass(s, mx);
+            if (s == -INFINITY) continue;
+            const int bn = score_bin(s, mx);
+            atomicAdd(&sm.bin_mass[bn], score_mass(s, mx));
+            atomicAdd(&sm.bin_cnt[bn], 1u);
         }
-        tot = warp_sum_u64(tot);
-        if (lane == 0) sm.redu[w] = tot;
         __syncthreads();
-        tot = 0;
-        for (int i = 0; i < kRouteWarps; ++i) tot += sm.redu[i];
+        // 3. one warp: total, target, the crossing bin and the mass of the bins before it
+        if (w == 0) {
+            unsigned long long ls = 0;
+            for (int k = 0; k < kBins / 32; ++k) ls += sm.bin_mass[lane * (kBins / 32) + k];
+            unsigned long long incl = ls;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const unsigned long long tot = __shfl_sync(0xffffffffu, incl, 31);
+            unsigned long long target =
+                static_cast<unsigned long long>(ceil(static_cast<double>(p) * static_cast<double>(tot)));
+            if (target < 1) target = 1;
+            if (target > tot) target = tot;
+            const uint32_t bal = __ballot_sync(0xffffffffu, incl >= target);
+            const int J = __ffs(bal) - 1;            // first lane whose inclusive sum reaches the target
+            if (lane == J) {
+                unsigned long long run = incl - ls;  // mass of the bins of the lanes before J
+                int c = lane * (kBins / 32);
+                for (int k = 0; k < kBins / 32; ++k) {
+                    const unsigned long long mk = sm.bin_mass[lane * (kBins / 32) + k];
+                    if (run + mk >= target) { c = lane * (kBins / 32) + k; break; }
+                    run += mk;
+                }
+                sm.cut_bin = c;
+                sm.cut_above = run;
+                sm.cut_target = target;
+            }
+        }
         __syncthreads();
-        unsigned long long target =
-            static_cast<unsigned long long>(ceil(static_cast<double>(p) * static_cast<double>(tot)));
-        if (target < 1) target = 1;
-        if (target > tot) target = tot;
-
-        // 3. radix select of the cut key, 8 bits at a time below the highest differing bit
-        unsigned long long above = 0;
-        const int hb = (kmin == kmax) ? -1 : 31 - __clz(kmin ^ kmax);
-        pmask = hb < 0 ? 0xffffffffu : (hb >= 31 ? 0u : ~((2u << hb) - 1u));
-        prefix = kmax & pmask;
-        unsigned long long tie_mass = 0;
-        uint32_t tie_cnt = 0;
-        bool unique = false;
-        for (int top = hb; top >= 0 && !unique; top -= 8) {
-            const int width = top >= 7 ? 8 : top + 1;
-            const int shift = top - width + 1;
-            const uint32_t dmask = (1u << width) - 1u;
-            if (tid < 256) { sm.hist_mass[tid] = 0; sm.hist_cnt[tid] = 0; }
-            __syncthreads();
-            for (int i = tid; i < nc; i += kRouteThreads) {
-                const float s = sc[i];
-                if (s == -INFINITY) continue;
-                const uint32_t k = score_key(s);
-                if ((k & pmask) != prefix) continue;
-                const uint32_t dg = (k >> shift) & dmask;
-                atomicAdd(&sm.hist_cnt[dg], 1u);
-                atomicAdd(&sm.hist_mass[dg], score_mass(s, mx));
+        cbin = sm.cut_bin;
+        // 4. gather the crossing bin's candidates
+        for (int i = tid; i < nc; i += kRouteThreads) {
+            const float s = sc[i];
+            if (s != -INFINITY && score_bin(s, mx) == cbin) {
+                const int t = atomicAdd(&sm.tie_n, 1);
+                if (t < kTieMax) sm.tie_slot[t] = i;
             }
-            __syncthreads();
-            if (w == 0) {
-                // lane j owns digits [8j, 8j+8); find the highest digit where the
-                // cumulative mass from the top first reaches the target.
-                unsigned long long ls = 0;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) ls += sm.hist_mass[lane * 8 + k];
-                unsigned long long suf = ls;   // inclusive suffix sum over lanes >= lane
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const unsigned long long y = __shfl_down_sync(0xffffffffu, suf, o);
-                    if (lane + o < 32) suf += y;
-                }
-                const bool reach = above + suf >= target;
-                const uint32_t bal = __ballot_sync(0xffffffffu, reach);
-                const int J = 31 - __clz(bal);                 // lane 0 always reaches
-                const unsigned long long sufJ1 = __shfl_sync(0xffffffffu, suf - ls, J);
-                if (lane == J) {
-                    unsigned long long run = above + sufJ1;
-                    int dsel = lane * 8;
-                    for (int k = 7; k >= 0; --k) {
-                        const unsigned long long mk = sm.hist_mass[lane * 8 + k];
-                        if (run + mk >= target) { dsel = lane * 8 + k; break; }
-                        run += mk;
-                    }
-                    sm.digit = dsel;
-                    sm.digit_above = run;
-                    sm.digit_cnt = sm.hist_cnt[dsel];
-                    sm.digit_mass = sm.hist_mass[dsel];
-                }
-            }
-            __syncthreads();
-            const uint32_t dsel = static_cast<uint32_t>(sm.digit);
-            above = sm.digit_above;
-            tie_cnt = sm.digit_cnt;
-            tie_mass = sm.digit_mass;
-            prefix |= dsel << shift;
-            pmask |= dmask << shift;
-            unique = tie_cnt == 1;
-            __syncthreads();
         }
-        if (hb < 0) {   // every candidate has the same key: one tie group
-            unsigned long long c = 0, msum = 0;
-            for (int i = tid; i < nc; i += kRouteThreads)
-                if (sc[i] != -INFINITY) { c += 1; msum += score_mass(sc[i], mx); }
-            c = warp_sum_u64(c);
-            msum = warp_sum_u64(msum);
-            if (lane == 0) { sm.redu[w] = c; sm.hist_mass[w] = msum; }
-            __syncthreads();
-            c = 0; msum = 0;
-            for (int i = 0; i < kRouteWarps; ++i) { c += sm.redu[i]; msum += sm.hist_mass[i]; }
-            __syncthreads();
-            tie_cnt = static_cast<uint32_t>(c);
-            tie_mass = msum;
-        }
-        // all members of the tie group carry the same mass (same key unless unique)
-        const unsigned long long m_tie = tie_mass / tie_cnt;
-        take = (target - above + m_tie - 1) / m_tie;
-        if (take > tie_cnt) take = tie_cnt;
-        all_ties = take == tie_cnt;
+        __syncthreads();
     }
-
-    // 4. compaction in slot order: thread t owns slots [t*per, (t+1)*per)
+    const unsigned long long above = sm.cut_above, target = sm.cut_target;
+    const int nt = sm.tie_n;
+    // exact order inside the crossing bin: slot i of the bin is kept iff the mass of
+    // the bin's members ordered before it (higher score, or equal score and lower
+    // slot) plus the mass of the earlier bins stays below the target
+    auto before_in_bin = [&](int i, float si) -> unsigned long long {
+        unsigned long long bsum = 0;
+        if (nt <= kTieMax) {
+            for (int u = 0; u < nt; ++u) {
+                const int j = sm.tie_slot[u];
+                const float sj = sc[j];
+                if (sj > si || (sj == si && j < i)) bsum += score_mass(sj, mx);
+            }
+        } else {   // more members than the list holds: scan every slot
+            for (int j = 0; j < nc; ++j) {
+                const float sj = sc[j];
+                if (sj != -INFINITY && score_bin(sj, mx) == cbin && (sj > si || (sj == si && j < i)))
+                    bsum += score_mass(sj, mx);
+            }
+        }
+        return bsum;
+    };
+    // 5. compaction in slot order: thread t owns slots [t*per, (t+1)*per)
     const int per = (nc + kRouteThreads - 1) / kRouteThreads;
     const int i0 = min(nc, tid * per), i1 = min(nc, i0 + per);
-    int tie_base = 0;
-    if (!keep_all && !all_ties) {
-        int c = 0;
-        for (int i = i0; i < i1; ++i) {
-            const float s = sc[i];
-            if (s != -INFINITY && (score_key(s) & pmask) == prefix) ++c;
-        }
-        int tot;
-        tie_base = block_exclusive_scan<kRouteWarps>(c, sm.scan, &tot);
-    }
-    auto kept = [&](int i, int& tie_rank) -> bool {
+    auto kept = [&](int i) -> bool {
         const float s = sc[i];
         if (s == -INFINITY) return false;
         if (keep_all) return true;
-        const uint32_t k = score_key(s) & pmask;
-        if (k > prefix) return true;
-        if (k < prefix) return false;
-        return static_cast<unsigned long long>(tie_rank++) < take;
+        const int bn = score_bin(s, mx);
+        return bn < cbin || (bn == cbin && above + before_in_bin(i, s) < target);
     };
     int c = 0;
-    {
-        int tr = tie_base;
-        for (int i = i0; i < i1; ++i) c += kept(i, tr) ? 1 : 0;
-    }
+    for (int i = i0; i < i1; ++i) c += kept(i) ? 1 : 0;
     int total;
     int base = block_exclusive_scan<kRouteWarps>(c, sm.scan, &total);
-    {
-        int tr = tie_base;
-        for (int i = i0; i < i1; ++i)
-            if (kept(i, tr)) out[base++] = node_of(i);
-    }
+    for (int i = i0; i < i1; ++i)
+        if (kept(i)) out[base++] = node_of(i);
     __syncthreads();
     return total;
 }
@@ -354,8 +310,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
         __syncthreads();
         // ---- top-p cut and compaction of the kept node ids
         const int nxt = nc <= kParentsSmem ? (cur == 0 ? 1 : 0) : (cur == 2 ? 3 : 2);
-        np = top_p_select(sc, nc, a.p[l - 1], bufs[nxt], sm,
-                          [par, b](int i) { return static_cast<int32_t>(par[i / b] * b + i % b); });
+        auto node_of = [par, b](int i) { return static_cast<int32_t>(par[i / b] * b + i % b); };
+        np = top_p_select(sc, nc, a.p[l - 1], bufs[nxt], sm, node_of);
         cur = nxt;
     }
     // ---- level-1 selection -> sel

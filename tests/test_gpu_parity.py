@@ -136,6 +136,50 @@ def test_p_one_and_tiny_p():
     assert_status_clean()
 
 
+@pytest.mark.parametrize("p", [[0.9, 1.0, 1.0, 1.0], [0.97, 0.9, 1.0, 1.0], [0.5, 1.0, 1.0, 1.0]])
+def test_large_candidate_sets(p):
+    """More than 2048 candidates at a level (p = 1 above it): the block-wide cut instead of the warp one."""
+    d, G, Hkv = 128, 4, 1
+    N = 200000                                    # n_1 = 3125 leaf blocks
+    K, V, Q, qref = planted_inputs("test", 1, G, Hkv, d, N, N, 96, 2)
+    cfg = zha.Config(d=d, Hq=G, Hkv=Hkv, B=64, b=16, batch=1, N_cap=N, p=p)
+    dec = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), [N])
+    dec.build()
+    ot = oracle_tree(K[0, 0], N, cfg, qref[0])
+    rep = Report()
+    for step in range(Q.shape[0]):
+        dec.route_attend(Q[step].reshape(1, 1, G, d).contiguous().cuda())
+        sel, cnt, o = dec.results()
+        check_queries(cfg, ot, K[0, 0], V[0, 0], N - 1, Q[step, 0], [sel[0, 0, h].numpy() for h in range(G)],
+                      [int(cnt[0, 0, h]) for h in range(G)], [o[0, 0, h].numpy() for h in range(G)], p, rep)
+    rep.check()
+    assert rep.exact_required >= 4, rep
+    assert_status_clean()
+
+
+def test_thousands_of_exact_ties_keep_the_lowest_ids():
+    """All keys zero: every summary, hence every score, is equal.  p = 0.5 at level 1 (p = 1 above)
+    keeps the lowest half of the 4687 leaf blocks, ties going to the lower id."""
+    d, G = 128, 4
+    N = 4687 * 64
+    K = torch.zeros((1, 1, N, d), dtype=torch.bfloat16)
+    V = torch.randn((1, 1, N, d), generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    qref = W.reference_queries("test", 1, 1, d)
+    Q = torch.randn((1, 1, G, d), generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
+    cfg = zha.Config(d=d, Hq=G, Hkv=1, B=64, b=16, batch=1, N_cap=N, p=[0.5, 1.0, 1.0, 1.0])
+    dec = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), [N])
+    dec.build()
+    dec.route_attend(Q.cuda())
+    sel, cnt, _ = dec.results()
+    ot = oracle_tree(K[0, 0], N, cfg, qref[0])
+    for h in range(G):
+        rt = O.route(Q[0, 0, h], ot, [0.5, 1.0, 1.0, 1.0])
+        assert list(rt.sel) == list(range(2344))
+        assert int(cnt[0, 0, h]) == 2344
+        assert torch.equal(sel[0, 0, h, :2344], torch.arange(2344, dtype=torch.int32))
+    assert_status_clean()
+
+
 @pytest.mark.parametrize("N", [1, 17, 63, 64, 65, 128, 1000, 1024])
 def test_short_caches(N):
     """No complete block, exactly one, block boundaries: I(q) falls back to the sink and C_cur."""
