@@ -341,6 +341,37 @@ int check_ws(const WsLayout& wl, const void* ws, size_t ws_bytes) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- allocation-free attention
+// Scratch of zha_attend_noalloc: one file-scope device array, loaded with the
+// library on every GPU that uses it and kept until the process exits.  All
+// calls on a device share it; a call leaves its contents behind.
+constexpr size_t kNoAllocScratchBytes = size_t{16} << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (the symbol's host-side name is not a device address).
+int noalloc_scratch_ptr(void** out) {
+    static std::mutex mu;
+    static void* ptrs[64] = {};
+    int dev = 0;
+    ZHA_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(ZHA_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> lk(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(ZHA_ERR_CUDA, "cudaGetSymbolAddress(g_noalloc_scratch): %s", cudaGetErrorString(e));
+        ptrs[dev] = p;
+    }
+    *out = ptrs[dev];
+    return ZHA_OK;
+}
+
+}  // namespace
+
 // ======================================================================== C ABI
 extern "C" {
 
@@ -476,6 +507,35 @@ int zha_attend(const zha_config* cfg, const void* K, const void* V, const void* 
         if (sel_cap < 1) return fail(ZHA_ERR_INVALID_ARG, "sel_cap=%d", sel_cap);
         ZHA_TRY(run_plan(cfg, w, t, tree, N, sel, sel_count, sel_cap, ws, stream));
     }
+    return ZHA_DISPATCH(cfg, run_attend, cfg, w, K, V, Q, O, ws, stream);
+}
+
+int zha_attend_noalloc(const zha_config* cfg, const void* K, const void* V, const void* tree, const void* Q,
+                       int32_t n_q, const int32_t* N, const int32_t* sel, const int32_t* sel_count, int32_t sel_cap,
+                       float* O, zha_stream_t stream) {
+    TreeLayout t;
+    WsLayout w;
+    ZHA_TRY(tree_layout(cfg, &t));
+    ZHA_TRY(ws_layout(cfg, n_q, t, &w));
+    if (w.total > kNoAllocScratchBytes)
+        return fail(ZHA_ERR_WORKSPACE,
+                    "zha_attend_noalloc: this configuration needs %zu B of scratch; the library's static scratch "
+                    "holds %zu B (use zha_attend with a workspace)", w.total, kNoAllocScratchBytes);
+    ZHA_TRY(need(K, "K"));
+    ZHA_TRY(need(V, "V"));
+    ZHA_TRY(need(tree, "tree"));
+    ZHA_TRY(need(Q, "Q"));
+    ZHA_TRY(need(N, "N"));
+    ZHA_TRY(need(sel, "sel"));
+    ZHA_TRY(need(sel_count, "sel_count"));
+    ZHA_TRY(need(O, "O"));
+    if (sel_cap < 1) return fail(ZHA_ERR_INVALID_ARG, "sel_cap=%d", sel_cap);
+    void* ws = nullptr;
+    ZHA_TRY(noalloc_scratch_ptr(&ws));
+    // the per-group merge counters must start at zero; everything else is written before it is read
+    ZHA_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + w.off_counters, 0,
+                             sizeof(uint32_t) * static_cast<size_t>(cfg->batch) * cfg->Hkv, stream));
+    ZHA_TRY(run_plan(cfg, w, t, tree, N, sel, sel_count, sel_cap, ws, stream));
     return ZHA_DISPATCH(cfg, run_attend, cfg, w, K, V, Q, O, ws, stream);
 }
 

@@ -39,7 +39,7 @@ class ZhaConfig(ctypes.Structure):
 
 
 EXPORTS = ["zha_levels_cap", "zha_tree_bytes", "zha_tree_level", "zha_tree_count_offset", "zha_workspace_bytes", "zha_workspace_init", "zha_workspace_stats", "zha_build",
-           "zha_append", "zha_route", "zha_attend", "zha_decode", "zha_dense", "zha_get_status",
+           "zha_append", "zha_route", "zha_attend", "zha_attend_noalloc", "zha_decode", "zha_dense", "zha_get_status",
            "zha_last_error"]
 
 
@@ -66,6 +66,7 @@ def lib():
         "zha_append": [C, P, P, P, P, P, P, P],
         "zha_route": [C, P, P, I32, P, P, P, I32, P, SZ, P],
         "zha_attend": [C, P, P, P, P, I32, P, P, P, I32, P, P, SZ, P],
+        "zha_attend_noalloc": [C, P, P, P, P, I32, P, P, P, I32, P, P],
         "zha_decode": [C, P, P, P, P, P, P, P, P, P, SZ, P],
         "zha_dense": [C, P, P, P, I32, P, P, P, SZ, P],
         "zha_get_status": [P, I32, P],
@@ -216,6 +217,12 @@ def attend(cfg: Config, K, V, tree, Q, N, sel, sel_count, O, ws, n_q: int = 1, s
     sel_cap = sel.shape[-1] if sel is not None else 0
     _check(lib().zha_attend(ctypes.byref(cfg.c()), _ptr(K), _ptr(V), _ptr(tree), _ptr(Q), n_q, _ptr(N), _ptr(sel),
                             _ptr(sel_count), sel_cap, _ptr(O), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def attend_noalloc(cfg: Config, K, V, tree, Q, N, sel, sel_count, O, n_q: int = 1, stream=None):
+    """zha_attend without a workspace: the library's static device scratch (see include/zha.h)."""
+    _check(lib().zha_attend_noalloc(ctypes.byref(cfg.c()), _ptr(K), _ptr(V), _ptr(tree), _ptr(Q), n_q, _ptr(N),
+                                    _ptr(sel), _ptr(sel_count), sel.shape[-1], _ptr(O), _stream(stream)))
 
 
 def decode(cfg: Config, K, V, tree, q, k_new, v_new, N, O, ws, stream=None):

@@ -170,6 +170,30 @@ int zha_attend(const zha_config *cfg, const void *K, const void *V, const void *
                const int32_t *sel_count, int32_t sel_cap, float *O, void *ws, size_t ws_bytes,
                zha_stream_t stream);
 
+/*
+ * zha_attend_noalloc -- zha_attend for callers that cannot allocate device
+ * memory and so cannot hand in a workspace: code embedded in a host framework
+ * that owns every device allocation and exposes no allocator to it, or a
+ * serving path that is not allowed to call cudaMalloc (it can synchronise the
+ * device and fragment a pre-reserved pool).  The pages describe no counterpart;
+ * it is a convenience of this library.
+ *
+ * Arguments, layouts and results are those of zha_attend (sel must not be
+ * NULL); the caller still owns K, V, tree, Q, N, sel, sel_count and O.  The
+ * scratch is one static device array of 16 MiB inside the library, present on
+ * every GPU that loads the library until the process exits.  A configuration
+ * whose scratch (zha_workspace_bytes) exceeds 16 MiB is refused with
+ * ZHA_ERR_WORKSPACE before anything runs.  The call allocates nothing.
+ * - The first call on a device looks the array's device address up with
+ *   cudaGetSymbolAddress; make that first call before any stream capture.
+ * - All calls on a device share the array and it keeps the last call's
+ *   contents: calls that may overlap on the GPU (two streams, or two host
+ *   threads) race on it and must be serialised by the caller.
+ */
+int zha_attend_noalloc(const zha_config *cfg, const void *K, const void *V, const void *tree,
+                       const void *Q, int32_t n_q, const int32_t *N, const int32_t *sel,
+                       const int32_t *sel_count, int32_t sel_cap, float *O, zha_stream_t stream);
+
 /* zha_decode -- one decode step: zha_append, then zha_route and zha_attend of
  * the query q [batch][1][Hq][d] at its own position (t = new N - 1).  The
  * selection goes to the workspace. */
