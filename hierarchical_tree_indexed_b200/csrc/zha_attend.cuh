@@ -195,8 +195,8 @@ struct AttSmem {
     static constexpr int kRed = (kAttConsumers / 2) * G * D > 2 * kSplitMax * G ? (kAttConsumers / 2) * G * D
                                                                                 : 2 * kSplitMax * G;
     float red[kRed];
-    float sw[kAttConsumers][G][kAttRowsPerWarp];  // scores, per warp
-    float pw[kAttConsumers][kAttRowsPerWarp][4];  // probabilities [row][head], per warp
+    float sw[kAttConsumers][2][G][kAttRowsPerWarp];  // scores, per warp and stage of a pair
+    float pw[kAttConsumers][2][kAttRowsPerWarp][4];  // probabilities [row][head], per warp and stage
     float cm[kAttConsumers][G], cl[kAttConsumers][G];
     int scan[kAttConsumers + 2];
     StageDesc desc[kAttStages];
@@ -383,26 +383,49 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
     }
 
     // ================= consumer warps
+    // A warp takes two stages of the same run at a time when it can (the run's last stage
+    // may come alone), so every phase below has two independent streams of work.
     float qv[G][VEC];
     float m_run = -INFINITY, l_run = 0.f;      // for head (lane / 8) of this lane
     float acc[G][VD];
     const int sub = lane / LPR, li = lane % LPR;
-    for (int it = 0;; ++it) {
-        const int slot = it % kAttStages;
-        if (!mbar_wait_bounded(&sm.full[slot], (it / kAttStages) & 1)) {
+    const int r0 = w * kAttRowsPerWarp;
+    int it = 0;
+    bool stop = false;
+    while (!stop) {
+        const int slotA = it % kAttStages;
+        if (!mbar_wait_bounded(&sm.full[slotA], (it / kAttStages) & 1)) {
             if (lane == 0) raise_status(ZHA_ERR_TIMEOUT);
             break;
         }
-        const StageDesc& d = sm.desc[slot];
-        const int n_rows = d.n_rows;
-        if (n_rows < 0) break;
-        const int g = d.group, split = d.split, flags = d.flags;
-        const uint32_t heads = d.heads;
+        const StageDesc& dA = sm.desc[slotA];
+        const int nA = dA.n_rows;
+        if (nA < 0) break;
+        const int g = dA.group, split = dA.split;
+        int flags = dA.flags;
+        uint32_t heads = dA.heads;
+        int slotB = slotA, nB = 0, nst = 1;
+        if (!(flags & 1)) {   // not the run's last stage: the next stage belongs to the same run
+            slotB = (it + 1) % kAttStages;
+            if (!mbar_wait_bounded(&sm.full[slotB], ((it + 1) / kAttStages) & 1)) {
+                if (lane == 0) raise_status(ZHA_ERR_TIMEOUT);
+                break;
+            }
+            nB = sm.desc[slotB].n_rows;
+            if (nB < 0) {        // only after a producer timeout: no second stage
+                nB = 0;
+                stop = true;
+            } else {
+                nst = 2;
+                flags |= sm.desc[slotB].flags & 1;
+                heads |= sm.desc[slotB].heads;
+            }
+        }
         if (flags & 2) {   // first stage of this CTA's piece of a group: its queries, fresh state
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 float x[VEC];
-                Elem<T>::load16(&sm.q[slot][h][li * VEC], x);
+                Elem<T>::load16(&sm.q[slotA][h][li * VEC], x);
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) qv[h][e] = x[e] * a.qscale;
             }
@@ -413,31 +436,35 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
 #pragma unroll
                 for (int e = 0; e < VD; ++e) acc[h][e] = 0.f;
         }
-        const int r0 = w * kAttRowsPerWarp;
-        if (r0 < n_rows) {
+        const int slot_s[2] = {slotA, slotB};
+        const int n_s[2] = {nA, nB};
+        if (r0 < nA || r0 < nB) {
             // QK: lane (sub, li) covers rows r0 + u*RPW + sub, dims [li*VEC, li*VEC+VEC)
-            float v[NV];
+            float v[2][NV];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int r = r0 + u * RPW + sub;
-                float x[VEC];
-                if (r < n_rows) {
-                    Elem<T>::load16(&sm.k[slot][r][li * VEC], x);
-                } else {
+            for (int st = 0; st < 2; ++st) {
 #pragma unroll
-                    for (int e = 0; e < VEC; ++e) x[e] = 0.f;
-                }
+                for (int u = 0; u < U; ++u) {
+                    const int r = r0 + u * RPW + sub;
+                    float x[VEC];
+                    if (r < n_s[st]) {
+                        Elem<T>::load16(&sm.k[slot_s[st]][r][li * VEC], x);
+                    } else {
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    float dd = 0.f;
-                    if ((heads >> h) & 1u) {
-#pragma unroll
-                        for (int e = 0; e < VEC; ++e) dd = fmaf(qv[h][e], x[e], dd);
+                        for (int e = 0; e < VEC; ++e) x[e] = 0.f;
                     }
-                    v[h * U + u] = dd;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        float dd = 0.f;
+                        if ((heads >> h) & 1u) {
+#pragma unroll
+                            for (int e = 0; e < VEC; ++e) dd = fmaf(qv[h][e], x[e], dd);
+                        }
+                        v[st][h * U + u] = dd;
+                    }
                 }
             }
-            // transpose-reduce over the LPR lanes of a row group
+            // transpose-reduce over the LPR lanes of a row group (both stages interleaved)
             constexpr int LOG_LPR = LPR == 32 ? 5 : LPR == 16 ? 4 : LPR == 8 ? 3 : 2;
             constexpr int LOG_NV = NV >= 32 ? 5 : NV == 16 ? 4 : NV == 8 ? 3 : NV == 4 ? 2 : NV == 2 ? 1 : 0;
             constexpr int H = LOG_NV < LOG_LPR ? LOG_NV : LOG_LPR;   // halving steps
@@ -450,13 +477,17 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
 #pragma unroll
                     for (int i = 0; i < NV / 2; ++i) {
                         if (i < half) {
-                            const float send = upper ? v[i] : v[i + half];
-                            const float keep = upper ? v[i + half] : v[i];
-                            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+#pragma unroll
+                            for (int st = 0; st < 2; ++st) {
+                                const float send = upper ? v[st][i] : v[st][i + half];
+                                const float keep = upper ? v[st][i + half] : v[st][i];
+                                v[st][i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                            }
                         }
                     }
                 } else {
-                    v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+#pragma unroll
+                    for (int st = 0; st < 2; ++st) v[st][0] += __shfl_xor_sync(0xffffffffu, v[st][0], o);
                 }
             }
             // the halving steps fix the top H bits of the value index from li's top
@@ -470,28 +501,35 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
                     for (int k = 0; k < NV / NVH; ++k) {
                         const int vi = vi0 * (NV / NVH) + k;   // = h * U + u
                         const int h = vi / U, u = vi % U;
-                        sm.sw[w][h][u * RPW + sub] = v[k];
+#pragma unroll
+                        for (int st = 0; st < 2; ++st) sm.sw[w][st][h][u * RPW + sub] = v[st][k];
                     }
                 }
             }
             __syncwarp();
-            // online softmax: lane -> (head hh = lane / 8, row rr = lane % 8)
+            // online softmax over both stages' rows: lane -> (head hh = lane / 8, row rr = lane % 8)
             const int hh = lane / kAttRowsPerWarp, rr = lane % kAttRowsPerWarp;
             const int row = r0 + rr;
-            const bool valid = hh < G && row < n_rows && ((d.mask[row] >> hh) & 1);
-            const float sv = valid ? sm.sw[w][hh < G ? hh : 0][rr] : -INFINITY;
-            float mx = sv;
+            const bool va = hh < G && row < nA && ((dA.mask[row] >> hh) & 1);
+            const bool vb = hh < G && row < nB && ((sm.desc[slotB].mask[row] >> hh) & 1);
+            const float sa = va ? sm.sw[w][0][hh < G ? hh : 0][rr] : -INFINITY;
+            const float sb = vb ? sm.sw[w][1][hh < G ? hh : 0][rr] : -INFINITY;
+            float mx = fmaxf(sa, sb);
 #pragma unroll
             for (int o = 1; o < kAttRowsPerWarp; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             const float mn = fmaxf(m_run, mx);
             const float alpha = mn == -INFINITY ? 1.f : exp2f(m_run - mn);
-            const float pr = valid ? exp2f(sv - mn) : 0.f;
-            float ps = pr;
+            const float pa = va ? exp2f(sa - mn) : 0.f;
+            const float pb = vb ? exp2f(sb - mn) : 0.f;
+            float ps = pa + pb;
 #pragma unroll
             for (int o = 1; o < kAttRowsPerWarp; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
             l_run = l_run * alpha + ps;
             m_run = mn;
-            if (hh < G) sm.pw[w][rr][hh] = pr;
+            if (hh < G) {
+                sm.pw[w][0][rr][hh] = pa;
+                sm.pw[w][1][rr][hh] = pb;
+            }
             __syncwarp();
             // PV: lane owns dims [lane*VD, lane*VD+VD) of every head
 #pragma unroll
@@ -502,21 +540,28 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
             }
 #pragma unroll
             for (int r = 0; r < kAttRowsPerWarp; ++r) {
-                if (r0 + r < n_rows) {
-                    float vv[VD];
-                    load_n<T, VD>(&sm.v[slot][r0 + r][lane * VD], vv);
-                    const float4 p4 = *reinterpret_cast<const float4*>(&sm.pw[w][r][0]);
-                    const float pp[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll
-                    for (int h = 0; h < G; ++h)
-                        if ((heads >> h) & 1u)
+                for (int st = 0; st < 2; ++st) {
+                    if (r0 + r < n_s[st]) {
+                        float vv[VD];
+                        load_n<T, VD>(&sm.v[slot_s[st]][r0 + r][lane * VD], vv);
+                        const float4 p4 = *reinterpret_cast<const float4*>(&sm.pw[w][st][r][0]);
+                        const float pp[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll
-                            for (int e = 0; e < VD; ++e) acc[h][e] = fmaf(pp[h], vv[e], acc[h][e]);
+                        for (int h = 0; h < G; ++h)
+                            if ((heads >> h) & 1u)
+#pragma unroll
+                                for (int e = 0; e < VD; ++e) acc[h][e] = fmaf(pp[h], vv[e], acc[h][e]);
+                    }
                 }
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.empty[slot]);   // this warp is done with the slot
+        if (lane == 0) {   // this warp is done with the slot(s)
+            mbar_arrive(&sm.empty[slotA]);
+            if (nst == 2) mbar_arrive(&sm.empty[slotB]);
+        }
+        it += nst;
 
         if (flags & 1) {
             // ---- combine the consumer warps' states into one partial per head
