@@ -15,6 +15,7 @@
 #include "zha.h"
 #include "zha_common.cuh"
 #include "zha_build.cuh"
+#include "zha_plan.cuh"
 #include "zha_route.cuh"
 #include "zha_attend.cuh"
 
@@ -53,9 +54,9 @@ struct TreeLayout {
 };
 
 struct WsLayout {
-    int64_t cand_cap, par_cap, sel_cap, item_cap, words;
+    int64_t cand_cap, par_cap, kb_cap, sel_cap, item_cap, words;
     size_t off_scores, off_parents, off_sel, off_count, off_items, off_nitems, off_ml, off_acc, off_counters;
-    size_t off_rows, off_cand, off_sched;
+    size_t off_rows, off_cand, off_sched, off_ballot, off_grp;
     size_t total;
 };
 
@@ -129,6 +130,7 @@ int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
     const int G = c->Hq / c->Hkv;
     w->cand_cap = t.ncap[0] + c->b;
     w->par_cap = std::max<int64_t>(t.ncap[0], 1);
+    w->kb_cap = (w->cand_cap + 31) / 32;
     w->sel_cap = std::max<int64_t>(t.ncap[0], 1);
     w->item_cap = t.ncap[0] + 2 + (c->N_cap + kAttRows - 1) / kAttRows;
     w->words = (t.ncap[0] + 31) / 32;
@@ -145,6 +147,8 @@ int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
     w->off_rows = off;     off = align256(off + sizeof(int32_t) * groups);
     w->off_cand = off;     off = align256(off + sizeof(int32_t) * ctas);
     w->off_sched = off;    off = align256(off + sizeof(uint32_t) * 2);
+    w->off_ballot = off;   off = align256(off + sizeof(uint32_t) * ctas * 2 * w->kb_cap);
+    w->off_grp = off;      off = align256(off + sizeof(uint32_t) * groups);
     w->total = off;
     if (static_cast<size_t>(G) * w->words * 4 > 200 * 1024)
         return fail(ZHA_ERR_UNSUPPORTED, "N_cap too large for the on-chip union bitmap");
@@ -242,6 +246,10 @@ int run_append(const zha_config* c, const TreeLayout& lay, void* K, void* V, con
 }
 
 // ---------------------------------------------------------------- route
+PlanArgs plan_args(const zha_config* c, const WsLayout& wl, const TreeLayout& lay, const void* tree,
+                   const int32_t* N, const int32_t* sel, const int32_t* cnt, int32_t sel_cap, void* ws);
+bool plan_fits_route(const zha_config* c, const WsLayout& wl);
+
 template <typename T, int D, int NVR>
 int run_route_t(const RouteArgs& a, int ctas, cudaStream_t st) {
     auto kern = route_decode_kernel<T, D, NVR>;
@@ -252,18 +260,22 @@ int run_route_t(const RouteArgs& a, int ctas, cudaStream_t st) {
 
 template <typename T, int D>
 int run_route(const zha_config* c, const TreeLayout& lay, const WsLayout& wl, const void* tree, const void* Q,
-              const int32_t* N, int32_t* sel, int32_t* cnt, int32_t sel_cap, void* ws, cudaStream_t st) {
+              const int32_t* N, int32_t* sel, int32_t* cnt, int32_t sel_cap, void* ws, bool fuse, cudaStream_t st) {
     RouteArgs a{};
     a.tree = tree_view(lay, const_cast<void*>(tree));
     a.Q = Q; a.N = N; a.sel = sel; a.sel_count = cnt;
     a.cand = at<int32_t>(ws, wl.off_cand);
     a.ws_scores = at<float>(ws, wl.off_scores);
     a.ws_parents = at<int32_t>(ws, wl.off_parents);
-    a.cand_cap = wl.cand_cap; a.par_cap = wl.par_cap; a.N_cap = c->N_cap;
+    a.ws_ballot = at<uint32_t>(ws, wl.off_ballot);
+    a.cand_cap = wl.cand_cap; a.par_cap = wl.par_cap; a.kb_cap = wl.kb_cap; a.N_cap = c->N_cap;
     a.sel_cap = sel_cap; a.batch = c->batch; a.Hq = c->Hq; a.Hkv = c->Hkv; a.B = c->B; a.b = c->b;
     a.L_fixed = c->L_fixed; a.n_q = 1;
     a.scale = scale_of(c);
     for (int l = 0; l < kMaxLevels; ++l) a.p[l] = c->p[l];
+    a.plan = plan_args(c, wl, lay, tree, N, sel, cnt, sel_cap, ws);
+    a.grp_done = at<uint32_t>(ws, wl.off_grp);
+    a.fuse_plan = fuse ? 1 : 0;
     const int ctas = c->batch * c->Hq;
     if (c->b <= 4) return run_route_t<T, D, 4>(a, ctas, st);
     if (c->b <= 8) return run_route_t<T, D, 8>(a, ctas, st);
@@ -307,8 +319,8 @@ int run_attend(const zha_config* c, const WsLayout& wl, const void* K, const voi
     }
 }
 
-int run_plan(const zha_config* c, const WsLayout& wl, const TreeLayout& lay, const void* tree, const int32_t* N,
-             const int32_t* sel, const int32_t* cnt, int32_t sel_cap, void* ws, cudaStream_t st) {
+PlanArgs plan_args(const zha_config* c, const WsLayout& wl, const TreeLayout& lay, const void* tree,
+                   const int32_t* N, const int32_t* sel, const int32_t* cnt, int32_t sel_cap, void* ws) {
     PlanArgs a{};
     a.sel = sel; a.sel_count = cnt; a.N = N;
     a.n_tree = tree_view(lay, const_cast<void*>(tree)).n_tree;
@@ -318,6 +330,17 @@ int run_plan(const zha_config* c, const WsLayout& wl, const TreeLayout& lay, con
     a.item_cap = wl.item_cap; a.N_cap = c->N_cap;
     a.sel_cap = sel_cap; a.Hq = c->Hq; a.Hkv = c->Hkv; a.G = c->Hq / c->Hkv; a.B = c->B; a.n_q = 1;
     a.words = std::max<int64_t>(wl.words, 1);
+    return a;
+}
+
+// The route kernel builds the plan itself when the group's bitmap fits its score buffer.
+bool plan_fits_route(const zha_config* c, const WsLayout& wl) {
+    return static_cast<int64_t>(c->Hq / c->Hkv) * std::max<int64_t>(wl.words, 1) <= kScoresSmem;
+}
+
+int run_plan(const zha_config* c, const WsLayout& wl, const TreeLayout& lay, const void* tree, const int32_t* N,
+             const int32_t* sel, const int32_t* cnt, int32_t sel_cap, void* ws, cudaStream_t st) {
+    const PlanArgs a = plan_args(c, wl, lay, tree, N, sel, cnt, sel_cap, ws);
     const size_t smem = sizeof(uint32_t) * a.G * a.words;
     ZHA_TRY(allow_smem(plan_decode_kernel, smem));
     plan_decode_kernel<<<c->batch * c->Hkv, kPlanThreads, smem, st>>>(a);
@@ -484,8 +507,9 @@ int zha_route(const zha_config* cfg, const void* tree, const void* Q, int32_t n_
     ZHA_TRY(need(sel, "sel"));
     ZHA_TRY(need(sel_count, "sel_count"));
     if (sel_cap < 1) return fail(ZHA_ERR_INVALID_ARG, "sel_cap=%d", sel_cap);
-    ZHA_TRY(ZHA_DISPATCH(cfg, run_route, cfg, t, w, tree, Q, N, sel, sel_count, sel_cap, ws, stream));
-    return run_plan(cfg, w, t, tree, N, sel, sel_count, sel_cap, ws, stream);
+    const bool fuse = plan_fits_route(cfg, w);
+    ZHA_TRY(ZHA_DISPATCH(cfg, run_route, cfg, t, w, tree, Q, N, sel, sel_count, sel_cap, ws, fuse, stream));
+    return fuse ? ZHA_OK : run_plan(cfg, w, t, tree, N, sel, sel_count, sel_cap, ws, stream);
 }
 
 int zha_attend(const zha_config* cfg, const void* K, const void* V, const void* tree, const void* Q, int32_t n_q,
@@ -552,8 +576,9 @@ int zha_decode(const zha_config* cfg, void* K, void* V, void* tree, const void* 
     int32_t* sel = at<int32_t>(ws, w.off_sel);
     int32_t* cnt = at<int32_t>(ws, w.off_count);
     const int32_t sel_cap = static_cast<int32_t>(w.sel_cap);
-    ZHA_TRY(ZHA_DISPATCH(cfg, run_route, cfg, t, w, tree, q, N, sel, cnt, sel_cap, ws, stream));
-    ZHA_TRY(run_plan(cfg, w, t, tree, N, sel, cnt, sel_cap, ws, stream));
+    const bool fuse = plan_fits_route(cfg, w);
+    ZHA_TRY(ZHA_DISPATCH(cfg, run_route, cfg, t, w, tree, q, N, sel, cnt, sel_cap, ws, fuse, stream));
+    if (!fuse) ZHA_TRY(run_plan(cfg, w, t, tree, N, sel, cnt, sel_cap, ws, stream));
     return ZHA_DISPATCH(cfg, run_attend, cfg, w, K, V, q, O, ws, stream);
 }
 

@@ -27,6 +27,7 @@
 #pragma once
 
 #include "zha_common.cuh"
+#include "zha_plan.cuh"
 
 namespace zha {
 
@@ -39,7 +40,7 @@ namespace zha {
 #ifndef ZHA_ATT_ROTATE
 #define ZHA_ATT_ROTATE 1
 #endif
-constexpr int kAttRows = 64;                  // rows per pipeline stage
+constexpr int kAttRows = kItemRowsMax;        // rows per pipeline stage
 // stages in flight per CTA: as many 64-row K+V stages as the budget holds, 2..6
 template <typename T, int D>
 constexpr int att_stages() {
@@ -48,114 +49,6 @@ constexpr int att_stages() {
 }
 constexpr int kAttChunk = ZHA_ATT_CHUNK;      // items per round-robin chunk; 0 = one contiguous piece per CTA
 constexpr int kSplitMax = 512;        // partials per group (>= the attention grid)
-constexpr int kPlanThreads = 512;
-
-// item: x = first key, y = key count | head mask << 16
-__device__ __forceinline__ int2 make_item(int64_t start, int count, uint32_t mask) {
-    return make_int2(static_cast<int>(start), count | static_cast<int>(mask << 16));
-}
-
-struct PlanArgs {
-    const int32_t* sel;        // [batch][n_q][Hq][sel_cap]
-    const int32_t* sel_count;  // [batch][n_q][Hq]
-    const int32_t* N;          // [batch]
-    const int32_t* n_tree;     // [batch]
-    int2* items;               // [groups][item_cap]
-    int32_t* n_items;          // [groups]
-    int32_t* rows;             // [groups] keys gathered (accounting)
-    int64_t item_cap, N_cap;
-    int sel_cap, Hq, Hkv, G, B, n_q;
-    int64_t words;             // bitmap words per head: ceil(n1cap / 32)
-};
-
-// One CTA per (sequence, KV head).
-__global__ void __launch_bounds__(kPlanThreads) plan_decode_kernel(PlanArgs a) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    uint32_t* bits = reinterpret_cast<uint32_t*>(smem_raw);   // [G][words]
-    __shared__ int scan[kPlanThreads / 32 + 1];
-    const int g = blockIdx.x, s = g / a.Hkv, kv = g % a.Hkv, tid = threadIdx.x;
-    const int G = a.G;
-    const uint32_t all = (1u << G) - 1u;
-    const int64_t N = a.N[s], Ntree = a.n_tree[s];
-    if (N < 1 || N > a.N_cap || Ntree > N) {
-        if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.n_items[g] = 0; a.rows[g] = 0; }
-        return;
-    }
-    const int64_t t = N - 1;
-    const int64_t n1 = Ntree / a.B;
-    const int64_t words = (n1 + 31) / 32;
-    for (int64_t i = tid; i < G * words; i += kPlanThreads) bits[(i / words) * a.words + i % words] = 0u;
-    __syncthreads();
-    for (int h = 0; h < G; ++h) {
-        const int64_t row = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + h;
-        const int cnt = min(a.sel_count[row], a.sel_cap);
-        const int32_t* sl = a.sel + row * a.sel_cap;
-        for (int i = tid; i < cnt; i += kPlanThreads) {
-            const int32_t blk = sl[i];
-            if (blk >= 0 && blk < n1) atomicOr(&bits[h * a.words + (blk >> 5)], 1u << (blk & 31));
-        }
-    }
-    const int64_t cb = min(t / a.B, n1);   // C_cur = [cb*B, t]
-    if (tid < G && cb < n1) atomicOr(&bits[tid * a.words + (cb >> 5)], 1u << (cb & 31));
-    __syncthreads();
-    // compaction of the union, ascending: thread owns words [w0, w1)
-    const int64_t per = (words + kPlanThreads - 1) / kPlanThreads;
-    const int64_t w0 = min(words, tid * per), w1 = min(words, w0 + per);
-    int c = 0;
-    for (int64_t wd = w0; wd < w1; ++wd) {
-        uint32_t o = 0;
-        for (int h = 0; h < G; ++h) o |= bits[h * a.words + wd];
-        c += __popc(o);
-    }
-    int total;
-    int pos = block_exclusive_scan<kPlanThreads / 32>(c, scan, &total);
-    int2* out = a.items + static_cast<int64_t>(g) * a.item_cap;
-    for (int64_t wd = w0; wd < w1; ++wd) {
-        uint32_t o = 0;
-        for (int h = 0; h < G; ++h) o |= bits[h * a.words + wd];
-        while (o) {
-            const int bit = __ffs(o) - 1;
-            o &= o - 1;
-            uint32_t m = 0;
-            for (int h = 0; h < G; ++h) m |= ((bits[h * a.words + wd] >> bit) & 1u) << h;
-            out[pos++] = make_item((wd * 32 + bit) * a.B, a.B, m);
-        }
-    }
-    if (tid == 0) {
-        int n = total;
-        int64_t rows = static_cast<int64_t>(total) * a.B;
-        if (n1 >= 1) {   // sink: key 0 for the heads whose block 0 is not in the union
-            uint32_t m0 = 0;
-            for (int h = 0; h < G; ++h) m0 |= (bits[h * a.words] & 1u) << h;
-            if ((m0 & all) != all) { out[n++] = make_item(0, 1, all & ~m0); rows += 1; }
-        }
-        if (cb == n1)   // C_cur past the last leaf block: the keys [n1*B, t], 64 at a time
-            for (int64_t st = cb * a.B; st <= t && n < a.item_cap; st += kAttRows) {
-                const int c = static_cast<int>(t - st + 1 < kAttRows ? t - st + 1 : kAttRows);
-                out[n++] = make_item(st, c, all);
-                rows += c;
-            }
-        a.n_items[g] = n;
-        a.rows[g] = static_cast<int32_t>(rows);
-    }
-}
-
-// Dense baseline plan: items of 64 keys covering [0, N) for every head.
-__global__ void plan_dense_kernel(const int32_t* N, int2* items, int32_t* n_items, int32_t* rows,
-                                  int64_t item_cap, int64_t N_cap, int Hkv, int G) {
-    const int g = blockIdx.x, s = g / Hkv;
-    const int64_t n = N[s];
-    if (n < 1 || n > N_cap) {
-        if (threadIdx.x == 0) { raise_status(ZHA_ERR_INVALID_ARG); n_items[g] = 0; rows[g] = 0; }
-        return;
-    }
-    if (threadIdx.x == 0) rows[g] = static_cast<int32_t>(n);
-    const int64_t cnt = (n + kAttRows - 1) / kAttRows;
-    const uint32_t all = (1u << G) - 1u;
-    for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x)
-        items[g * item_cap + i] = make_item(i * kAttRows, static_cast<int>(n - i * kAttRows < kAttRows ? n - i * kAttRows : kAttRows), all);
-    if (threadIdx.x == 0) n_items[g] = static_cast<int32_t>(cnt);
-}
 
 struct AttendArgs {
     const void* K;
@@ -403,7 +296,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
         if (nA < 0) break;
         const int g = dA.group, split = dA.split;
         int flags = dA.flags;
-        uint32_t heads = dA.heads;
+        uint32_t heads_s[2] = {dA.heads, 0u};
         int slotB = slotA, nB = 0, nst = 1;
         if (!(flags & 1)) {   // not the run's last stage: the next stage belongs to the same run
             slotB = (it + 1) % kAttStages;
@@ -418,7 +311,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
             } else {
                 nst = 2;
                 flags |= sm.desc[slotB].flags & 1;
-                heads |= sm.desc[slotB].heads;
+                heads_s[1] = sm.desc[slotB].heads;
             }
         }
         if (flags & 2) {   // first stage of this CTA's piece of a group: its queries, fresh state
@@ -436,8 +329,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
 #pragma unroll
                 for (int e = 0; e < VD; ++e) acc[h][e] = 0.f;
         }
-        const int slot_s[2] = {slotA, slotB};
         const int n_s[2] = {nA, nB};
+        // this warp's rows of both stages, and the heads each stage needs
+        const T* krow_s[2] = {&sm.k[slotA][r0][0], &sm.k[slotB][r0][0]};
+        const T* vrow_s[2] = {&sm.v[slotA][r0][0], &sm.v[slotB][r0][0]};
+        const uint8_t* mrow_s[2] = {&dA.mask[r0], &sm.desc[slotB].mask[r0]};
         if (r0 < nA || r0 < nB) {
             // QK: lane (sub, li) covers rows r0 + u*RPW + sub, dims [li*VEC, li*VEC+VEC)
             float v[2][NV];
@@ -445,10 +341,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
             for (int st = 0; st < 2; ++st) {
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    const int r = r0 + u * RPW + sub;
+                    const int rl = u * RPW + sub;           // row within the warp's 8
                     float x[VEC];
-                    if (r < n_s[st]) {
-                        Elem<T>::load16(&sm.k[slot_s[st]][r][li * VEC], x);
+                    if (r0 + rl < n_s[st]) {
+                        Elem<T>::load16(krow_s[st] + rl * D + li * VEC, x);
                     } else {
 #pragma unroll
                         for (int e = 0; e < VEC; ++e) x[e] = 0.f;
@@ -456,7 +352,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
                         float dd = 0.f;
-                        if ((heads >> h) & 1u) {
+                        if ((heads_s[st] >> h) & 1u) {
 #pragma unroll
                             for (int e = 0; e < VEC; ++e) dd = fmaf(qv[h][e], x[e], dd);
                         }
@@ -510,8 +406,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
             // online softmax over both stages' rows: lane -> (head hh = lane / 8, row rr = lane % 8)
             const int hh = lane / kAttRowsPerWarp, rr = lane % kAttRowsPerWarp;
             const int row = r0 + rr;
-            const bool va = hh < G && row < nA && ((dA.mask[row] >> hh) & 1);
-            const bool vb = hh < G && row < nB && ((sm.desc[slotB].mask[row] >> hh) & 1);
+            const bool va = hh < G && row < nA && ((mrow_s[0][rr] >> hh) & 1);
+            const bool vb = hh < G && row < nB && ((mrow_s[1][rr] >> hh) & 1);
             const float sa = va ? sm.sw[w][0][hh < G ? hh : 0][rr] : -INFINITY;
             const float sb = vb ? sm.sw[w][1][hh < G ? hh : 0][rr] : -INFINITY;
             float mx = fmaxf(sa, sb);
@@ -544,12 +440,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
                 for (int st = 0; st < 2; ++st) {
                     if (r0 + r < n_s[st]) {
                         float vv[VD];
-                        load_n<T, VD>(&sm.v[slot_s[st]][r0 + r][lane * VD], vv);
+                        load_n<T, VD>(vrow_s[st] + r * D + lane * VD, vv);
                         const float4 p4 = *reinterpret_cast<const float4*>(&sm.pw[w][st][r][0]);
                         const float pp[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll
                         for (int h = 0; h < G; ++h)
-                            if ((heads >> h) & 1u)
+                            if ((heads_s[st] >> h) & 1u)
 #pragma unroll
                                 for (int e = 0; e < VD; ++e) acc[h][e] = fmaf(pp[h], vv[e], acc[h][e]);
                     }

@@ -21,6 +21,7 @@
 #pragma once
 
 #include "zha_common.cuh"
+#include "zha_plan.cuh"
 
 namespace zha {
 
@@ -38,7 +39,11 @@ struct RouteArgs {
     int32_t* cand;          // [batch][n_q][Hq] candidates scored over all levels (accounting)
     float* ws_scores;       // [batch*Hq][cand_cap]
     int32_t* ws_parents;    // [batch*Hq][2][par_cap]
-    int64_t cand_cap, par_cap, N_cap;
+    uint32_t* ws_ballot;    // [batch*Hq][2][kb_cap]
+    int64_t cand_cap, par_cap, kb_cap, N_cap;
+    PlanArgs plan;          // the gather plan, built here by the group's last CTA when fuse_plan
+    uint32_t* grp_done;     // [batch*Hkv] query heads routed, zero between calls
+    int fuse_plan;
     int sel_cap, batch, Hq, Hkv, B, b, L_fixed, n_q;
     float scale;
     float p[kMaxLevels];
@@ -50,11 +55,14 @@ struct RouteSmem {
     float scores[kScoresSmem];
     int32_t parents[2][kParentsSmem];
     unsigned long long bin_mass[1024];
-    uint32_t bin_cnt[1024];
+    uint32_t keep_ballot[kScoresSmem / 32];
+    int32_t keep_prefix[kScoresSmem / 32];
     int32_t tie_slot[kTieMax];
     float q[128];
     int scan[kRouteWarps + 1];
     float redf[kRouteWarps];
+    int redi[kRouteWarps];
+    int plan_last;
     int tie_n, cut_bin;
     unsigned long long cut_above, cut_target;
 };
@@ -89,15 +97,87 @@ __device__ __forceinline__ int score_bin(float s, float smax) {
 // target; only the candidates of that bin are ranked exactly (by score, then
 // slot) against each other.  Candidate i is kept iff the mass of everything
 // ordered before it is below the target.
+// The same cut for nc <= 64, by warp 0 alone: the (score, slot) pairs are sorted by a
+// bitonic network (descending score, ascending slot; two elements per lane), the
+// fixed-point masses are prefix-summed in that order, and candidate e is kept iff the
+// mass before it is below ceil(p * total).  The kept slots, ascending, go to out.
+__device__ __forceinline__ float key_score(uint32_t k) {   // inverse of score_key
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 template <typename NodeOf>
-__device__ int top_p_select(const float* sc, int nc, float p, int32_t* out, RouteSmem& sm, NodeOf node_of) {
+__device__ int top_p_small(const float* sc, int nc, float p, int32_t* out, NodeOf node_of) {
+    const int lane = threadIdx.x & 31;
+    auto make = [&](int i) -> unsigned long long {
+        const float s = i < nc ? sc[i] : -INFINITY;
+        return s == -INFINITY ? 0ull
+                              : (static_cast<unsigned long long>(score_key(s)) << 32) | (0xffffffffu - static_cast<uint32_t>(i));
+    };
+    unsigned long long a = make(lane), b = make(lane + 32);   // elements lane and lane + 32
+    for (int size = 2; size <= 64; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride == 32) {
+                if (a < b) { const unsigned long long t = a; a = b; b = t; }   // size 64: descending
+            } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    unsigned long long& x = h == 0 ? a : b;
+                    const int e = lane + 32 * h;
+                    const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, stride);
+                    const bool desc = (e & size) == 0;
+                    const bool lower = (e & stride) == 0;
+                    x = (lower == desc) ? (x > y ? x : y) : (x < y ? x : y);
+                }
+            }
+        }
+    }
+    // sorted: element lane = a, element lane + 32 = b (descending); masses in that order
+    const float smax = key_score(static_cast<uint32_t>(__shfl_sync(0xffffffffu, a, 0) >> 32));
+    if (__shfl_sync(0xffffffffu, a, 0) == 0ull) return 0;   // no valid candidate
+    const unsigned long long ma = a ? score_mass(key_score(static_cast<uint32_t>(a >> 32)), smax) : 0ull;
+    const unsigned long long mb = b ? score_mass(key_score(static_cast<uint32_t>(b >> 32)), smax) : 0ull;
+    unsigned long long ca = ma, cb = mb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long ya = __shfl_up_sync(0xffffffffu, ca, o);
+        const unsigned long long yb = __shfl_up_sync(0xffffffffu, cb, o);
+        if (lane >= o) { ca += ya; cb += yb; }
+    }
+    const unsigned long long half = __shfl_sync(0xffffffffu, ca, 31);
+    cb += half;
+    const unsigned long long tot = __shfl_sync(0xffffffffu, cb, 31);
+    bool ka, kb;
+    if (p >= 1.0f) {
+        ka = a != 0ull;
+        kb = b != 0ull;
+    } else {
+        unsigned long long target =
+            static_cast<unsigned long long>(ceil(static_cast<double>(p) * static_cast<double>(tot)));
+        if (target < 1) target = 1;
+        if (target > tot) target = tot;
+        ka = a != 0ull && ca - ma < target;
+        kb = b != 0ull && cb - mb < target;
+    }
+    // kept slots as a 64-bit set, then written in ascending slot order
+    unsigned long long set = (ka ? 1ull << (0xffffffffu - static_cast<uint32_t>(a)) : 0ull) |
+                             (kb ? 1ull << (0xffffffffu - static_cast<uint32_t>(b)) : 0ull);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) set |= __shfl_xor_sync(0xffffffffu, set, o);
+    if ((set >> lane) & 1ull) out[__popcll(set & ((1ull << lane) - 1ull))] = node_of(lane);
+    if ((set >> (lane + 32)) & 1ull) out[__popcll(set & ((1ull << (lane + 32)) - 1ull))] = node_of(lane + 32);
+    return __popcll(set);
+}
+
+// kball/kpre: ceil(nc/32) words each (shared memory, or the workspace for large nc).
+template <typename NodeOf>
+__device__ int top_p_select(const float* sc, int nc, float p, int32_t* out, RouteSmem& sm, uint32_t* kball,
+                            int32_t* kpre, NodeOf node_of) {
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     // 1. max score; clear the bins
     float mx = -INFINITY;
     for (int i = tid; i < nc; i += kRouteThreads) mx = fmaxf(mx, sc[i]);
     mx = warp_max(mx);
     if (lane == 0) sm.redf[w] = mx;
-    for (int k = tid; k < kBins; k += kRouteThreads) { sm.bin_mass[k] = 0; sm.bin_cnt[k] = 0; }
+    for (int k = tid; k < kBins; k += kRouteThreads) sm.bin_mass[k] = 0;
     if (tid == 0) { sm.tie_n = 0; sm.cut_above = 0; sm.cut_target = 0; }
     __syncthreads();
     mx = -INFINITY;
@@ -111,15 +191,21 @@ __device__ int top_p_select(const float* sc, int nc, float p, int32_t* out, Rout
         for (int i = tid; i < nc; i += kRouteThreads) {
             const float s = sc[i];
             if (s == -INFINITY) continue;
-            const int bn = score_bin(s, mx);
-            atomicAdd(&sm.bin_mass[bn], score_mass(s, mx));
-            atomicAdd(&sm.bin_cnt[bn], 1u);
+            atomicAdd(&sm.bin_mass[score_bin(s, mx)], score_mass(s, mx));
         }
         __syncthreads();
-        // 3. one warp: total, target, the crossing bin and the mass of the bins before it
+        // 3. one warp: total, target, the crossing bin and the mass of the bins before it.
+        //    Lane j first sums bins [32j, 32j+32) (independent partial sums), then the
+        //    crossing lane's 32 bins are scanned one per lane.
         if (w == 0) {
-            unsigned long long ls = 0;
-            for (int k = 0; k < kBins / 32; ++k) ls += sm.bin_mass[lane * (kBins / 32) + k];
+            const ulonglong2* bm = reinterpret_cast<const ulonglong2*>(sm.bin_mass + lane * 32);
+            unsigned long long p0 = 0, p1 = 0, p2 = 0, p3 = 0;
+#pragma unroll
+            for (int k = 0; k < 16; k += 2) {
+                const ulonglong2 x = bm[k], y = bm[k + 1];
+                p0 += x.x; p1 += x.y; p2 += y.x; p3 += y.y;
+            }
+            const unsigned long long ls = (p0 + p1) + (p2 + p3);
             unsigned long long incl = ls;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -131,18 +217,19 @@ __device__ int top_p_select(const float* sc, int nc, float p, int32_t* out, Rout
                 static_cast<unsigned long long>(ceil(static_cast<double>(p) * static_cast<double>(tot)));
             if (target < 1) target = 1;
             if (target > tot) target = tot;
-            const uint32_t bal = __ballot_sync(0xffffffffu, incl >= target);
-            const int J = __ffs(bal) - 1;            // first lane whose inclusive sum reaches the target
-            if (lane == J) {
-                unsigned long long run = incl - ls;  // mass of the bins of the lanes before J
-                int c = lane * (kBins / 32);
-                for (int k = 0; k < kBins / 32; ++k) {
-                    const unsigned long long mk = sm.bin_mass[lane * (kBins / 32) + k];
-                    if (run + mk >= target) { c = lane * (kBins / 32) + k; break; }
-                    run += mk;
-                }
-                sm.cut_bin = c;
-                sm.cut_above = run;
+            const int J = __ffs(__ballot_sync(0xffffffffu, incl >= target)) - 1;
+            const unsigned long long base = __shfl_sync(0xffffffffu, incl - ls, J);   // bins before lane J's
+            const unsigned long long mb = sm.bin_mass[J * 32 + lane];
+            unsigned long long run = mb;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long y = __shfl_up_sync(0xffffffffu, run, o);
+                if (lane >= o) run += y;
+            }
+            const int k = __ffs(__ballot_sync(0xffffffffu, base + run >= target)) - 1;
+            if (lane == k) {
+                sm.cut_bin = J * 32 + k;
+                sm.cut_above = base + run - mb;
                 sm.cut_target = target;
             }
         }
@@ -180,9 +267,6 @@ __device__ int top_p_select(const float* sc, int nc, float p, int32_t* out, Rout
         }
         return bsum;
     };
-    // 5. compaction in slot order: thread t owns slots [t*per, (t+1)*per)
-    const int per = (nc + kRouteThreads - 1) / kRouteThreads;
-    const int i0 = min(nc, tid * per), i1 = min(nc, i0 + per);
     auto kept = [&](int i) -> bool {
         const float s = sc[i];
         if (s == -INFINITY) return false;
@@ -190,12 +274,38 @@ __device__ int top_p_select(const float* sc, int nc, float p, int32_t* out, Rout
         const int bn = score_bin(s, mx);
         return bn < cbin || (bn == cbin && above + before_in_bin(i, s) < target);
     };
-    int c = 0;
-    for (int i = i0; i < i1; ++i) c += kept(i) ? 1 : 0;
-    int total;
-    int base = block_exclusive_scan<kRouteWarps>(c, sm.scan, &total);
-    for (int i = i0; i < i1; ++i)
-        if (kept(i)) out[base++] = node_of(i);
+    // 5. compaction in slot order: one ballot per 32-slot group (warp w takes groups
+    //    w, w + 16, ...), an in-order prefix of the groups' counts by one warp, then writes
+    const int ngrp = (nc + 31) / 32;
+    for (int gi = w; gi < ngrp; gi += kRouteWarps) {
+        const int i = gi * 32 + lane;
+        const uint32_t bal = __ballot_sync(0xffffffffu, i < nc && kept(i));
+        if (lane == 0) kball[gi] = bal;
+    }
+    __syncthreads();
+    if (w == 0) {
+        int run = 0;
+        for (int gi = 0; gi < ngrp; gi += 32) {
+            const int g2 = gi + lane;
+            const int c = g2 < ngrp ? __popc(kball[g2]) : 0;
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (g2 < ngrp) kpre[g2] = run + incl - c;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) sm.redi[0] = run;
+    }
+    __syncthreads();
+    const int total = sm.redi[0];
+    for (int gi = w; gi < ngrp; gi += kRouteWarps) {
+        const uint32_t bal = kball[gi];
+        const int i = gi * 32 + lane;
+        if ((bal >> lane) & 1u) out[kpre[gi] + __popc(bal & ((1u << lane) - 1u))] = node_of(i);
+    }
     __syncthreads();
     return total;
 }
@@ -249,25 +359,77 @@ __device__ __forceinline__ void scan_children(const float* __restrict__ kh, cons
     }
 }
 
-// One CTA per (sequence, query head): the whole top-down walk of one decode query.
-// NVR = b rounded up to a power of two (4, 8, 16 or 32).
+// scan_children for two parents at once: both blocks' loads are issued before either
+// reduction, so a warp keeps twice the bytes in flight.
+template <int D, int NVR>
+__device__ __forceinline__ void scan_children2(const float* __restrict__ kh0, const float* __restrict__ bh0, int cnt0,
+                                               const float* __restrict__ kh1, const float* __restrict__ bh1, int cnt1,
+                                               int b, const float* qv, float* __restrict__ out0,
+                                               float* __restrict__ out1) {
+    constexpr int VF = D / 32;
+    const int lane = threadIdx.x & 31;
+    float x0[NVR][VF], x1[NVR][VF];
+#pragma unroll
+    for (int r = 0; r < NVR; ++r) {
+        if (r < cnt0) load_n<float, VF>(kh0 + static_cast<int64_t>(r) * D + lane * VF, x0[r]);
+        else
+#pragma unroll
+            for (int e = 0; e < VF; ++e) x0[r][e] = 0.f;
+        if (r < cnt1) load_n<float, VF>(kh1 + static_cast<int64_t>(r) * D + lane * VF, x1[r]);
+        else
+#pragma unroll
+            for (int e = 0; e < VF; ++e) x1[r][e] = 0.f;
+    }
+    float v0[NVR], v1[NVR];
+#pragma unroll
+    for (int r = 0; r < NVR; ++r) {
+        float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < VF; ++e) {
+            d0 = fmaf(qv[e], x0[r][e], d0);
+            d1 = fmaf(qv[e], x1[r][e], d1);
+        }
+        v0[r] = d0;
+        v1[r] = d1;
+    }
+    constexpr int H = NVR == 32 ? 5 : NVR == 16 ? 4 : NVR == 8 ? 3 : NVR == 4 ? 2 : 1;
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {
+        const int o = 16 >> step;
+        if (step < H) {
+            const int half = NVR >> (step + 1);
+            const bool upper = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < NVR / 2; ++i) {
+                if (i < half) {
+                    const float s0 = upper ? v0[i] : v0[i + half], k0 = upper ? v0[i + half] : v0[i];
+                    const float s1 = upper ? v1[i] : v1[i + half], k1 = upper ? v1[i + half] : v1[i];
+                    v0[i] = k0 + __shfl_xor_sync(0xffffffffu, s0, o);
+                    v1[i] = k1 + __shfl_xor_sync(0xffffffffu, s1, o);
+                }
+            }
+        } else {
+            v0[0] += __shfl_xor_sync(0xffffffffu, v0[0], o);
+            v1[0] += __shfl_xor_sync(0xffffffffu, v1[0], o);
+        }
+    }
+    constexpr int low = 5 - H;
+    if ((lane & ((1 << low) - 1)) == 0) {
+        const int r = (lane >> low) & (NVR - 1);
+        if (r < b) {
+            out0[r] = r < cnt0 ? v0[0] + bh0[r] : -INFINITY;
+            out1[r] = r < cnt1 ? v1[0] + bh1[r] : -INFINITY;
+        }
+    }
+}
+
+// The top-down walk of one decode query (the body of route_decode_kernel).
 template <typename T, int D, int NVR>
-__global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArgs a) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    RouteSmem& sm = *reinterpret_cast<RouteSmem*>(smem_raw);
+__device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, int cta, int64_t row, int64_t slice,
+                                           int64_t N, int64_t Ntree) {
     constexpr int VF = D / 32;   // fp32 summary elements per lane
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    const int cta = blockIdx.x;
-    const int s = cta / a.Hq, hq = cta % a.Hq;
-    const int kv = hq / (a.Hq / a.Hkv);
-    const int64_t slice = static_cast<int64_t>(s) * a.Hkv + kv;
-    const int64_t row = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + hq;
-    const int64_t N = a.N[s];
-    const int64_t Ntree = a.tree.n_tree[s];
-    if (N < 1 || N > a.N_cap || Ntree > N || Ntree < 0) {
-        if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.sel_count[row] = 0; a.cand[row] = 0; }
-        return;
-    }
+    (void)N;
     if (tid < D) sm.q[tid] = to_f32(static_cast<const T*>(a.Q)[row * D + tid]) * a.scale;
     int64_t n[kMaxLevels];
     const int L = tree_levels(Ntree, a.B, a.b, a.L_fixed, n);
@@ -279,6 +441,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
     const int b = a.b;
     float* ws_sc = a.ws_scores + static_cast<int64_t>(cta) * a.cand_cap;
     int32_t* ws_par = a.ws_parents + static_cast<int64_t>(cta) * 2 * a.par_cap;
+    uint32_t* ws_kb = a.ws_ballot + static_cast<int64_t>(cta) * 2 * a.kb_cap;
     int32_t* bufs[4] = {sm.parents[0], sm.parents[1], ws_par, ws_par + a.par_cap};
     int cur = 0;   // index into bufs
 
@@ -302,16 +465,35 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
         const float* kh = a.tree.khat[l - 1] + slice * ncap * D;
         const float* bh = a.tree.bhat[l - 1] + slice * ncap;
         // ---- scan: one warp per kept parent, its b child rows of D fp32
-        for (int pi = w; pi < np; pi += kRouteWarps) {
+        for (int pi = w; pi < np; pi += 2 * kRouteWarps) {
+            const int pj = pi + kRouteWarps;   // a second parent in the same round, if any
             const int64_t c0 = static_cast<int64_t>(par[pi]) * b;
-            const int cnt = static_cast<int>(min(static_cast<int64_t>(b), nl - c0));
-            scan_children<D, NVR>(kh + c0 * D, bh + c0, cnt, b, qv, sc + static_cast<int64_t>(pi) * b);
+            const int cnt0 = static_cast<int>(min(static_cast<int64_t>(b), nl - c0));
+            if (pj < np) {
+                const int64_t c1 = static_cast<int64_t>(par[pj]) * b;
+                const int cnt1 = static_cast<int>(min(static_cast<int64_t>(b), nl - c1));
+                scan_children2<D, NVR>(kh + c0 * D, bh + c0, cnt0, kh + c1 * D, bh + c1, cnt1, b, qv,
+                                       sc + static_cast<int64_t>(pi) * b, sc + static_cast<int64_t>(pj) * b);
+            } else {
+                scan_children<D, NVR>(kh + c0 * D, bh + c0, cnt0, b, qv, sc + static_cast<int64_t>(pi) * b);
+            }
         }
         __syncthreads();
         // ---- top-p cut and compaction of the kept node ids
         const int nxt = nc <= kParentsSmem ? (cur == 0 ? 1 : 0) : (cur == 2 ? 3 : 2);
         auto node_of = [par, b](int i) { return static_cast<int32_t>(par[i / b] * b + i % b); };
-        np = top_p_select(sc, nc, a.p[l - 1], bufs[nxt], sm, node_of);
+        if (nc <= 64) {
+            if (w == 0) {
+                const int c = top_p_small(sc, nc, a.p[l - 1], bufs[nxt], node_of);
+                if (lane == 0) sm.redi[0] = c;
+            }
+            __syncthreads();
+            np = sm.redi[0];
+        } else {
+            const bool big = (nc + 31) / 32 > kScoresSmem / 32;
+            np = top_p_select(sc, nc, a.p[l - 1], bufs[nxt], sm, big ? ws_kb : sm.keep_ballot,
+                              big ? reinterpret_cast<int32_t*>(ws_kb) + a.kb_cap : sm.keep_prefix, node_of);
+        }
         cur = nxt;
     }
     // ---- level-1 selection -> sel
@@ -323,6 +505,41 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
         a.sel_count[row] = np;
         a.cand[row] = static_cast<int32_t>(scored);
         if (np > a.sel_cap) raise_status(ZHA_ERR_CAPACITY);
+    }
+}
+
+
+// One CTA per (sequence, query head): the whole top-down walk of one decode query.
+// NVR = b rounded up to a power of two (4, 8, 16 or 32).
+template <typename T, int D, int NVR>
+__global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArgs a) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    RouteSmem& sm = *reinterpret_cast<RouteSmem*>(smem_raw);
+    const int tid = threadIdx.x;
+    const int cta = blockIdx.x;
+    const int s = cta / a.Hq, hq = cta % a.Hq;
+    const int kv = hq / (a.Hq / a.Hkv);
+    const int64_t slice = static_cast<int64_t>(s) * a.Hkv + kv;
+    const int64_t row = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + hq;
+    const int64_t N = a.N[s];
+    const int64_t Ntree = a.tree.n_tree[s];
+    const bool valid = !(N < 1 || N > a.N_cap || Ntree > N || Ntree < 0);
+    if (!valid) {
+        if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.sel_count[row] = 0; a.cand[row] = 0; }
+    } else {
+        route_walk<T, D, NVR>(a, sm, cta, row, slice, N, Ntree);
+    }
+    if (a.fuse_plan) {
+        // the last of the group's G query-head CTAs builds the group's gather plan
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) sm.plan_last = atomicAdd(&a.grp_done[slice], 1u) == static_cast<uint32_t>(a.Hq / a.Hkv - 1);
+        __syncthreads();
+        if (sm.plan_last) {
+            __threadfence();
+            plan_group(a.plan, static_cast<int>(slice), reinterpret_cast<uint32_t*>(sm.scores), sm.scan);
+            if (tid == 0) a.grp_done[slice] = 0u;
+        }
     }
 }
 
