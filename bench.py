@@ -52,6 +52,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling cases)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's N (profiling cases)")
+    ap.add_argument("--sweep", default="", help="comma-separated context lengths: tree path vs dense baseline")
     return ap.parse_args()
 
 
@@ -72,7 +73,7 @@ def config_dict(w, world: int) -> dict:
                         f"bf16 K/V, N={w.N}, leaf block {w.B}, branching {w.b}, p={w.p}",
             "global_batch": w.batch * world, "seq_len": w.N, "parallelism": f"dp{world}",
             "kv_dtype": w.dtype, "l2": "flushed (256 MiB write) before every timed step; KV 16 GiB > L2",
-            "step": "append + route + attend, each phase one CUDA graph"}
+            "step": "append + route (plan fused) + attend, each phase one CUDA graph"}
 
 
 def measured_peaks() -> tuple[float, str]:
@@ -200,16 +201,186 @@ def reference_arm(args, rank):
 
 # ------------------------------------------------------------------ GPU arm
 
+class DecodeRun:
+    """Device buffers of one decode workload and its three captured phases."""
+
+    def __init__(self, w, dev, N_cap, rank):
+        import torch
+
+        from hierarchical_tree_indexed_b200 import workloads as W
+        from hierarchical_tree_indexed_b200 import zha
+        self.w, self.dev, self.zha = w, dev, zha
+        # weak scaling: every rank owns a batch of w.batch sequences of its own
+        data = W.planted(w, device=dev, N_cap=N_cap, n_queries=POOL, seq_base=rank.rank * w.batch)
+        self.K, self.V, self.Qp, self.knp, self.vnp = data["K"], data["V"], data["Q"], data["k_new"], data["v_new"]
+        self.cfg = zha.Config(d=w.d, Hq=w.Hq, Hkv=w.Hkv, B=w.B, b=w.b, batch=w.batch, N_cap=N_cap,
+                              dtype=w.dtype, p=w.p)
+        cfg = self.cfg
+        self.N = torch.full((w.batch,), w.N, dtype=torch.int32, device=dev)
+        self.tree = zha.alloc_tree(cfg, dev)
+        self.ws = zha.alloc_workspace(cfg, device=dev)
+        self.sel = torch.zeros((w.batch, 1, w.Hq, max(N_cap // w.B, 1)), dtype=torch.int32, device=dev)
+        self.cnt = torch.zeros((w.batch, 1, w.Hq), dtype=torch.int32, device=dev)
+        self.O = torch.zeros((w.batch, 1, w.Hq, w.d), dtype=torch.float32, device=dev)
+        self.q_in = torch.empty((w.batch, 1, w.Hq, w.d), dtype=self.K.dtype, device=dev)
+        self.k_in = torch.empty((w.batch, w.Hkv, w.d), dtype=self.K.dtype, device=dev)
+        self.v_in = torch.empty_like(self.k_in)
+        self.rows_v, self.cand_v = zha.workspace_stats_view(cfg, self.ws)
+        zha.get_status(clear=True)
+        self.qref_dev = zha.build(cfg, self.K, data["qref"], self.N, self.tree)
+        del data
+        torch.cuda.synchronize()
+        self.load(0)
+        self.append(); self.route(); self.attend()
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        self.graphs = []
+        for fn in (self.append, self.route, self.attend):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                fn()
+            self.graphs.append(g)
+        self.dense()
+        torch.cuda.synchronize()
+        self.g_dense = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_dense, stream=s):
+            self.dense()
+        torch.cuda.synchronize()
+        self.step = 1
+
+    def load(self, i):
+        j = i % POOL
+        w = self.w
+        self.q_in.copy_(self.Qp[j].reshape(w.batch, 1, w.Hq, w.d))
+        self.k_in.copy_(self.knp[j])
+        self.v_in.copy_(self.vnp[j])
+
+    def append(self):
+        self.zha.append(self.cfg, self.K, self.V, self.k_in, self.v_in, self.N, self.tree)
+
+    def route(self):
+        self.zha.route(self.cfg, self.tree, self.q_in, self.N, self.sel, self.cnt, self.ws)
+
+    def attend(self):
+        self.zha.attend(self.cfg, self.K, self.V, self.tree, self.q_in, self.N, None, None, self.O, self.ws)
+
+    def dense(self):
+        self.zha.dense(self.cfg, self.K, self.V, self.q_in, self.N, self.O, self.ws)
+
+    def check_status(self, what):
+        bits = self.zha.get_status(clear=True)
+        if bits:
+            raise RuntimeError(f"device status after {what}: {self.zha.status_names(bits)}")
+
+    def timed_steps(self, steps, flush, clocks=None):
+        """Device times of `steps` decode steps (append, route, attend), L2 flushed before each."""
+        import torch
+        stream = torch.cuda.current_stream()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        rows_acc = torch.zeros((), dtype=torch.float64, device=self.dev)
+        cand_acc = torch.zeros((), dtype=torch.float64, device=self.dev)
+        g_app, g_route, g_att = self.graphs
+        for k in range(steps):
+            self.load(self.step)
+            self.step += 1
+            flush.zero_()
+            e = ev[k]
+            e[0].record(stream)
+            g_app.replay()
+            e[1].record(stream)
+            g_route.replay()
+            e[2].record(stream)
+            g_att.replay()
+            e[3].record(stream)
+            rows_acc += self.rows_v.sum()
+            cand_acc += self.cand_v.sum()
+        torch.cuda.synchronize()
+        self.check_status("the timed steps")
+        t = [sum(e[i].elapsed_time(e[i + 1]) for e in ev) / 1e3 for i in range(3)]
+        return dict(t_app=t[0], t_route=t[1], t_att=t[2], t_step=sum(t),
+                    rows=rows_acc.item() / steps, cand=cand_acc.item() / steps)
+
+    def dense_time(self, reps, flush):
+        import torch
+        stream = torch.cuda.current_stream()
+        evs = []
+        for _ in range(reps + 2):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream); self.g_dense.replay(); b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        self.check_status("the dense baseline")
+        return sum(a.elapsed_time(b) for a, b in evs[2:]) / reps / 1e3
+
+    def bytes_per_step(self, rows, cand):
+        w = self.w
+        es = 2 if w.dtype == "bf16" else 4
+        attend = rows * w.d * es * 2 + w.batch * w.Hq * w.d * (es + 4)
+        route = cand * (4 * w.d + 4) + w.batch * w.Hq * w.d * es
+        append = w.batch * w.Hkv * (2 * w.d * es + (w.B * w.d * es + (w.d + 1) * 4 * 4) / w.B)
+        return attend, route, append
+
+
+def sweep(args, rank):
+    """Tree path vs the in-library dense baseline across context lengths (batch from --batch, 1 by
+    default): per N, decode steps (append + route + attend) and dense steps, L2 flushed before each."""
+    import dataclasses
+
+    import torch
+
+    from hierarchical_tree_indexed_b200 import dist as D
+    from hierarchical_tree_indexed_b200 import workloads as W
+    dev = torch.device("cuda", rank.local)
+    torch.cuda.set_device(dev)
+    base = W.WORKLOADS["decode1m"]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    points = []
+    for n in [int(x) for x in args.sweep.split(",")]:
+        w = dataclasses.replace(base, N=n, n_clusters=max(1, n // 2048), batch=args.batch or 1)
+        run = DecodeRun(w, dev, n + args.warmup + args.steps + 8, rank)
+        for _ in range(args.warmup):
+            run.load(run.step); run.step += 1
+            for g in run.graphs:
+                g.replay()
+        r = run.timed_steps(args.steps, flush)
+        td = run.dense_time(5, flush)
+        ms = r["t_step"] / args.steps * 1e3
+        points.append({"N": n, "tree_ms": ms, "dense_ms": td * 1e3, "speedup": td * 1e3 / ms,
+                       "read_fraction": r["rows"] / (w.batch * w.Hkv * n),
+                       "route_ms": r["t_route"] / args.steps * 1e3, "attend_ms": r["t_att"] / args.steps * 1e3})
+        del run
+        torch.cuda.empty_cache()
+    cross = None
+    for a_, b_ in zip(points, points[1:]):
+        if a_["speedup"] < 1.0 <= b_["speedup"]:
+            # log-linear interpolation of the crossover in N
+            import math
+            fa, fb = math.log(a_["speedup"]), math.log(b_["speedup"])
+            x = math.log(a_["N"]) + (0 - fa) * (math.log(b_["N"]) - math.log(a_["N"])) / (fb - fa)
+            cross = round(math.exp(x))
+    if points and points[0]["speedup"] >= 1.0:
+        cross = f"<= {points[0]['N']}"
+    if rank.leader:
+        print(json.dumps({"metric": "decode step time, tree path vs in-library dense baseline", "unit": "ms",
+                          "batch": args.batch or 1, "steps": args.steps, "points": points,
+                          "crossover_N": cross}), flush=True)
+    D.finish(rank)
+    return 0
+
+
 def main():
     args = parse()
     from hierarchical_tree_indexed_b200 import dist as D
     rank = D.from_env()
     if args.impl == "reference":
         return reference_arm(args, rank)
+    if args.sweep:
+        return sweep(args, rank)
 
     import torch
 
-    from hierarchical_tree_indexed_b200 import workloads as W
     from hierarchical_tree_indexed_b200 import zha
 
     dev = torch.device("cuda", rank.local)
@@ -219,142 +390,49 @@ def main():
     K_steps, W_steps = args.steps, args.warmup
     e2e_steps = 0 if args.no_e2e else min(K_steps, 500)
     N_cap = w.N + W_steps + K_steps + e2e_steps + 8
-    # weak scaling: every rank owns a batch of w.batch sequences of its own
-    data = W.planted(w, device=dev, N_cap=N_cap, n_queries=POOL, seq_base=rank.rank * w.batch)
-    K, V, Qp, knp, vnp = data["K"], data["V"], data["Q"], data["k_new"], data["v_new"]
-    cfg = zha.Config(d=w.d, Hq=w.Hq, Hkv=w.Hkv, B=w.B, b=w.b, batch=w.batch, N_cap=N_cap, dtype=w.dtype, p=w.p)
-    N = torch.full((w.batch,), w.N, dtype=torch.int32, device=dev)
-    tree = zha.alloc_tree(cfg, dev)
-    ws = zha.alloc_workspace(cfg, device=dev)
-    sel = torch.zeros((w.batch, 1, w.Hq, max(N_cap // w.B, 1)), dtype=torch.int32, device=dev)
-    cnt = torch.zeros((w.batch, 1, w.Hq), dtype=torch.int32, device=dev)
-    O = torch.zeros((w.batch, 1, w.Hq, w.d), dtype=torch.float32, device=dev)
-    q_in = torch.empty((w.batch, 1, w.Hq, w.d), dtype=K.dtype, device=dev)
-    k_in = torch.empty((w.batch, w.Hkv, w.d), dtype=K.dtype, device=dev)
-    v_in = torch.empty_like(k_in)
+    run = DecodeRun(w, dev, N_cap, rank)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    rows_v, cand_v = zha.workspace_stats_view(cfg, ws)
-    zha.get_status(clear=True)
-
-    qref_dev = zha.build(cfg, K, data["qref"], N, tree)
+    for _ in range(W_steps):
+        run.load(run.step)
+        run.step += 1
+        for g in run.graphs:
+            g.replay()
     torch.cuda.synchronize()
+    run.check_status("warm-up")
 
-    def load_inputs(i):
-        j = i % POOL
-        q_in.copy_(Qp[j].reshape(w.batch, 1, w.Hq, w.d))
-        k_in.copy_(knp[j])
-        v_in.copy_(vnp[j])
-
-    def do_append():
-        zha.append(cfg, K, V, k_in, v_in, N, tree)
-
-    def do_route():
-        zha.route(cfg, tree, q_in, N, sel, cnt, ws)
-
-    def do_attend():
-        zha.attend(cfg, K, V, tree, q_in, N, None, None, O, ws)
-
-    # one untimed pass outside capture (kernel attributes), then capture each phase in a graph
-    load_inputs(0)
-    do_append(); do_route(); do_attend()
-    torch.cuda.synchronize()
-    graphs = []
-    s = torch.cuda.Stream(device=dev)
-    s.wait_stream(torch.cuda.current_stream())
-    for fn in (do_append, do_route, do_attend):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=s):
-            fn()
-        graphs.append(g)
-    torch.cuda.synchronize()
-    g_app, g_route, g_att = graphs
-
-    stream = torch.cuda.current_stream()
-    for i in range(W_steps):
-        load_inputs(i + 1)
-        g_app.replay(); g_route.replay(); g_att.replay()
-    torch.cuda.synchronize()
-    bits = zha.get_status(clear=True)
-    if bits:
-        raise RuntimeError(f"device status after warm-up: {zha.status_names(bits)}")
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_steps)]
-    rows_acc = torch.zeros((), dtype=torch.float64, device=dev)
-    cand_acc = torch.zeros((), dtype=torch.float64, device=dev)
     D.barrier(rank, dev)
     torch.cuda.synchronize()
     clocks = Clocks(rank.local) if rank.leader else None
     time.sleep(0.25)
-    for k in range(K_steps):
-        load_inputs(W_steps + 1 + k)
-        flush.zero_()
-        e = ev[k]
-        e[0].record(stream)
-        g_app.replay()
-        e[1].record(stream)
-        g_route.replay()
-        e[2].record(stream)
-        g_att.replay()
-        e[3].record(stream)
-        rows_acc += rows_v.sum()
-        cand_acc += cand_v.sum()
-    torch.cuda.synchronize()
+    r = run.timed_steps(K_steps, flush)
     clk = clocks.stop() if clocks else None
     D.barrier(rank, dev)
-    bits = zha.get_status(clear=True)
-    if bits:
-        raise RuntimeError(f"device status after the timed steps: {zha.status_names(bits)}")
-
-    t_app = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
-    t_route = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
-    t_att = sum(e[2].elapsed_time(e[3]) for e in ev) / 1e3
-    t_step = sum(e[0].elapsed_time(e[3]) for e in ev) / 1e3
-    t_max = D.max_over_ranks(t_step, rank, dev)
+    t_max = D.max_over_ranks(r["t_step"], rank, dev)
     queries = w.batch * K_steps * rank.world
     value = queries / t_max
 
-    # ---- algorithmic bytes (bf16 K/V, fp32 summaries)
-    es = 2 if w.dtype == "bf16" else 4
-    rows_mean = rows_acc.item() / K_steps                    # keys gathered per step, all groups
-    cand_mean = cand_acc.item() / K_steps                    # tree nodes scored per step, all heads
-    attend_bytes = rows_mean * w.d * es * 2 + w.batch * w.Hq * w.d * (es + 4)
-    route_bytes = cand_mean * (4 * w.d + 4) + w.batch * w.Hq * w.d * es
-    append_bytes = w.batch * w.Hkv * (2 * w.d * es + (w.B * w.d * es + (w.d + 1) * 4 * 4) / w.B)
+    attend_bytes, route_bytes, append_bytes = run.bytes_per_step(r["rows"], r["cand"])
     step_bytes = attend_bytes + route_bytes + append_bytes
     peak, peak_src = measured_peaks()
-    att_gbs = attend_bytes / (t_att / K_steps) / 1e9
-    step_gbs = step_bytes / (t_step / K_steps) / 1e9
-    read_fraction = rows_mean / (w.batch * w.Hkv * w.N)
+    att_gbs = attend_bytes / (r["t_att"] / K_steps) / 1e9
+    step_gbs = step_bytes / (r["t_step"] / K_steps) / 1e9
+    read_fraction = r["rows"] / (w.batch * w.Hkv * w.N)
     khash = source_hash(ATTEND_SOURCES)
     tr = profiled_traffic(khash)
-    traffic = (tr[0] * rows_mean + tr[1]) if tr else None
+    traffic = (tr[0] * r["rows"] + tr[1]) if tr else None
 
-    # ---- dense baseline at the same N (in-library, same loader)
-    def do_dense():
-        zha.dense(cfg, K, V, q_in, N, O, ws)
-    do_dense()
-    torch.cuda.synchronize()
-    gd = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gd, stream=s):
-        do_dense()
-    dense_ev = []
-    for k in range(10):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream); gd.replay(); b.record(stream)
-        dense_ev.append((a, b))
-    torch.cuda.synchronize()
-    t_dense = sum(a.elapsed_time(b) for a, b in dense_ev[2:]) / len(dense_ev[2:]) / 1e3
-    dense_rows = w.batch * w.Hkv * int(N[0].item())
-    dense_gbs = (dense_rows * w.d * es * 2) / t_dense / 1e9
+    t_dense = run.dense_time(8, flush)
+    es = 2 if w.dtype == "bf16" else 4
+    dense_gbs = (w.batch * w.Hkv * int(run.N[0].item()) * w.d * es * 2) / t_dense / 1e9
 
     # ---- end to end through the public C-ABI call with host buffers
     e2e = None
     if e2e_steps:
-        qh = torch.empty((POOL, w.batch, 1, w.Hq, w.d), dtype=K.dtype).pin_memory()
-        qh.copy_(Qp.reshape(POOL, w.batch, 1, w.Hq, w.d).cpu())
-        kh = knp.cpu().pin_memory()
-        vh = vnp.cpu().pin_memory()
+        stream = torch.cuda.current_stream()
+        qh = torch.empty((POOL, w.batch, 1, w.Hq, w.d), dtype=run.K.dtype).pin_memory()
+        qh.copy_(run.Qp.reshape(POOL, w.batch, 1, w.Hq, w.d).cpu())
+        kh = run.knp.cpu().pin_memory()
+        vh = run.vnp.cpu().pin_memory()
         oh = torch.empty((e2e_steps, w.batch, 1, w.Hq, w.d), dtype=torch.float32).pin_memory()
         torch.cuda.synchronize()
         D.barrier(rank, dev)
@@ -362,21 +440,19 @@ def main():
         a.record(stream)
         for k in range(e2e_steps):
             j = k % POOL
-            q_in.copy_(qh[j], non_blocking=True)
-            k_in.copy_(kh[j], non_blocking=True)
-            v_in.copy_(vh[j], non_blocking=True)
-            zha.decode(cfg, K, V, tree, q_in, k_in, v_in, N, O, ws)
-            oh[k].copy_(O, non_blocking=True)
+            run.q_in.copy_(qh[j], non_blocking=True)
+            run.k_in.copy_(kh[j], non_blocking=True)
+            run.v_in.copy_(vh[j], non_blocking=True)
+            zha.decode(run.cfg, run.K, run.V, run.tree, run.q_in, run.k_in, run.v_in, run.N, run.O, run.ws)
+            oh[k].copy_(run.O, non_blocking=True)
         b.record(stream)
         torch.cuda.synchronize()
         t_e2e = D.max_over_ranks(a.elapsed_time(b) / 1e3, rank, dev)
         e2e = {"value": w.batch * e2e_steps * rank.world / t_e2e, "unit": UNIT,
-               "h2d_bytes_per_step": (q_in.numel() + k_in.numel() + v_in.numel()) * es,
-               "d2h_bytes_per_step": O.numel() * 4, "steps": e2e_steps,
+               "h2d_bytes_per_step": (run.q_in.numel() + run.k_in.numel() + run.v_in.numel()) * es,
+               "d2h_bytes_per_step": run.O.numel() * 4, "steps": e2e_steps,
                "note": "zha_decode per step (not graphed), pinned host inputs/outputs, L2 not flushed"}
-        bits = zha.get_status(clear=True)
-        if bits:
-            raise RuntimeError(f"device status after the e2e steps: {zha.status_names(bits)}")
+        run.check_status("the e2e steps")
 
     cpu = None
     if rank.leader and rank.world == 1 and not args.no_cpu_baseline:
@@ -397,19 +473,19 @@ def main():
                          "unit": "GB/s", "frac": att_gbs / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} copy bandwidth", "algorithmic_bytes_per_launch": attend_bytes,
                          "kernel_source_sha256_16": khash},
-            "phases_ms": {"append": t_app / K_steps * 1e3, "route": t_route / K_steps * 1e3,
-                          "attend": t_att / K_steps * 1e3},
+            "phases_ms": {"append": r["t_app"] / K_steps * 1e3, "route": r["t_route"] / K_steps * 1e3,
+                          "attend": r["t_att"] / K_steps * 1e3},
             "bytes_per_step": {"attend": attend_bytes, "route": route_bytes, "append": append_bytes},
             "read_fraction": read_fraction,
             "dense_baseline": {"ms_per_step": t_dense * 1e3, "hbm_gbs": dense_gbs,
                                "queries_per_s": w.batch / t_dense, "speedup_of_tree": t_dense / (t_max / K_steps)},
-            "gpu_launches": 4 * K_steps,
+            "gpu_launches": 3 * K_steps,
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    del qref_dev
+    del run
     D.finish(rank)
     return 0
 
