@@ -310,7 +310,7 @@ def test_index_set_golden():
         got = O.index_set(sel, int(t), int(B), int(n1))
         assert list(got) == _ranges(rhs), line
         n += 1
-    assert n >= 7
+    assert n >= 9
 
 
 def test_attention_matches_numpy_softmax():
@@ -340,6 +340,25 @@ def test_p_one_routes_every_key_and_equals_dense_attention():
     assert list(idx) == list(range(N))
     w = softmax(tree.scale * K.astype(np.float64) @ x)
     assert np.max(np.abs(o - w @ V.astype(np.float64))) < 1e-13
+
+
+def test_prefill_query_with_p_one_is_causal_dense_attention():
+    """Chunked prefill reading: a tree over the first N_p keys only, a chunk query at
+    t > N_p.  With p = 1 every tree block is kept and the causal tail [n_1 B, t]
+    completes the set, so I(q) = [0, t] and o is causal dense attention up to t."""
+    d, B, b, Np, n_chunk = 16, 4, 3, 4 * 3 * 3 * 2 + 2, 9
+    r = rng(610)
+    K = r.standard_normal((Np + n_chunk, d)).astype(np.float32)
+    V = r.standard_normal((Np + n_chunk, d)).astype(np.float32)
+    tree, _ = _tree(K, Np, B, b)
+    assert tree.n[0] * B < Np          # an incomplete prefix block stays out of the tree
+    for i in (0, 4, n_chunk - 1):
+        t = Np + i
+        x = r.standard_normal(d) * 3
+        rt, idx, o = O.decode_query(x, tree, K, V, t, 1.0)
+        assert list(idx) == list(range(t + 1))
+        w = softmax(tree.scale * K[:t + 1].astype(np.float64) @ x)
+        assert np.max(np.abs(o - w @ V[:t + 1].astype(np.float64))) < 1e-13
 
 
 @pytest.mark.parametrize("which", ["flat_top_p", "routed"])
