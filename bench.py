@@ -33,6 +33,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "ZHA decode queries/s at 1M ctx + achieved HBM GB/s vs B200 peak"
+PREFILL_METRIC = "ZHA chunked prefill queries/s at 256K ctx (4096-query chunk, tensor-core attention)"
+FALLBACK_BF16_TFLOPS = 1590.0
 UNIT = "queries/s"
 FALLBACK_HBM_GBS = 6650.0
 POOL = 64                 # distinct (q, k_new, v_new) sets cycled through by the steps
@@ -76,13 +78,13 @@ def config_dict(w, world: int) -> dict:
             "step": "append + route (plan fused) + attend, each phase one CUDA graph"}
 
 
-def measured_peaks() -> tuple[float, str]:
+def measured_peaks(key: str = "hbm_gbs") -> tuple[float, str]:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(p) as f:
-            return float(json.load(f)["hbm_gbs"]), "measured"
+            return float(json.load(f)[key]), "measured"
     except (OSError, KeyError, ValueError):
-        return FALLBACK_HBM_GBS, "fallback"
+        return (FALLBACK_HBM_GBS if key == "hbm_gbs" else FALLBACK_BF16_TFLOPS), "fallback"
 
 
 def source_hash(paths) -> str:
@@ -149,31 +151,36 @@ class Clocks:
 
 def oracle_sample(w, seconds: float, warmup: int = 1, steps: int | None = None):
     """Times the oracle's route + attend of single query heads on one (sequence, KV head)
-    slice of the workload (tree built once, not timed).  Returns (seconds per head-query,
-    head-queries timed, setup seconds)."""
+    slice of the workload (tree built once, not timed).  Decode: the query of the token
+    appended at N.  Chunked prefill: queries of the chunk at t = N + i over a tree on the
+    first N keys.  Returns (seconds per head-query, head-queries timed, setup seconds)."""
     import torch
 
     from hierarchical_tree_indexed_b200 import workloads as W
     from oracle import oracle as O
 
     t0 = time.perf_counter()
-    K = torch.zeros((w.N + 1, w.d), dtype=torch.bfloat16)
+    extra = w.steps if w.prefill else 1
+    K = torch.zeros((w.N + extra, w.d), dtype=torch.bfloat16)
     V = torch.zeros_like(K)
     cl = W.fill_planted_slice(w.name, 0, 0, w.N, w.d, w.n_clusters, K, V)
-    kn, vn = W.background_tokens(w.name, 0, 0, 1, w.d, "cpu")
-    K[w.N], V[w.N] = kn[0].to(torch.bfloat16), vn[0].to(torch.bfloat16)
+    kn, vn = W.background_tokens(w.name, 0, 0, extra, w.d, "cpu", "chunk" if w.prefill else "append")
+    K[w.N:], V[w.N:] = kn.to(torch.bfloat16), vn.to(torch.bfloat16)
     qref = W.reference_queries(w.name, w.Hkv, 1, w.d)[0]
-    tree = O.build_tree(K, w.N + 1, w.B, w.b, qref)
-    qs = W.cluster_queries(w.name, 0, 0, w.G, 64, cl).to(torch.bfloat16).float().reshape(-1, w.d)
+    tree = O.build_tree(K, w.N if w.prefill else w.N + 1, w.B, w.b, qref)
+    nq = 64
+    qs = W.cluster_queries(w.name, 0, 0, w.G, nq, cl, stream="chunk_queries" if w.prefill else "queries")
+    qs = qs.to(torch.bfloat16).float().reshape(-1, w.d)
+    pos = [w.N + ((k // w.G) * 61) % extra if w.prefill else w.N for k in range(len(qs))]
     setup = time.perf_counter() - t0
     done, spent, i = 0, 0.0, 0
     for _ in range(warmup):
-        O.decode_query(qs[0], tree, K, V, w.N, w.p)
+        O.decode_query(qs[0], tree, K, V, pos[0], w.p)
     while (steps is None and spent < seconds) or (steps is not None and done < steps):
-        q = qs[i % len(qs)]
+        k = i % len(qs)
         i += 1
         t = time.perf_counter()
-        O.decode_query(q, tree, K, V, w.N, w.p)
+        O.decode_query(qs[k], tree, K, V, pos[k], w.p)
         spent += time.perf_counter() - t
         done += 1
     return spent / done, done, setup
@@ -186,9 +193,10 @@ def reference_arm(args, rank):
     per_head, done, setup = oracle_sample(w, 0.0, warmup=args.warmup, steps=args.steps)
     value = 1.0 / (per_head * w.Hq)
     sample = (f"{done} single-head route+attend calls of the fp64 C oracle on one (sequence, KV head) "
-              f"slice of {w.name} (N={w.N}, tree built once in {setup:.1f}s untimed), scaled to decode "
-              f"queries of all {w.Hq} heads")
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+              f"slice of {w.name} (N={w.N}, tree built once in {setup:.1f}s untimed), scaled to "
+              f"{'chunk' if w.prefill else 'decode'} queries of all {w.Hq} heads")
+    line = {"metric": PREFILL_METRIC if w.prefill else METRIC, "value": value, "unit": UNIT, "impl": "reference",
+            "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_head * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
@@ -370,6 +378,178 @@ def sweep(args, rank):
     return 0
 
 
+def prefill_main(args, rank, w):
+    """One step = one chunk of w.steps queries per sequence over a tree on the first N keys:
+    zha_route + zha_attend with n_q = w.steps (each one CUDA graph), L2 flushed before each."""
+    import torch
+
+    from hierarchical_tree_indexed_b200 import dist as D
+    from hierarchical_tree_indexed_b200 import workloads as W
+    from hierarchical_tree_indexed_b200 import zha
+
+    dev = torch.device("cuda", rank.local)
+    torch.cuda.set_device(dev)
+    D.init(rank, "nccl")
+    n_q, Np = w.steps, w.N
+    N_cap = Np + n_q
+    data = W.planted(w, device=dev, N_cap=N_cap, n_queries=n_q, seq_base=rank.rank * w.batch)
+    K, V = data["K"], data["V"]
+    K[:, :, Np:] = data["k_new"].permute(1, 2, 0, 3)
+    V[:, :, Np:] = data["v_new"].permute(1, 2, 0, 3)
+    Q = data["Q"].permute(1, 0, 2, 3).contiguous()
+    qref = data["qref"]
+    del data
+    cfg = zha.Config(d=w.d, Hq=w.Hq, Hkv=w.Hkv, B=w.B, b=w.b, batch=w.batch, N_cap=N_cap, dtype=w.dtype, p=w.p)
+    N = torch.full((w.batch,), N_cap, dtype=torch.int32, device=dev)
+    tree = zha.alloc_tree(cfg, dev)
+    ws = zha.alloc_workspace(cfg, n_q, device=dev)
+    sel_cap = Np // w.B
+    sel = torch.zeros((w.batch, n_q, w.Hq, sel_cap), dtype=torch.int32, device=dev)
+    cnt = torch.zeros((w.batch, n_q, w.Hq), dtype=torch.int32, device=dev)
+    O = torch.zeros((w.batch, n_q, w.Hq, w.d), dtype=torch.float32, device=dev)
+    Od = torch.zeros_like(O)
+    steps_v, cand_v = zha.workspace_stats_view(cfg, ws, n_q)
+    zha.get_status(clear=True)
+    zha.build(cfg, K, qref, torch.full((w.batch,), Np, dtype=torch.int32, device=dev), tree)
+
+    def do_route():
+        zha.route(cfg, tree, Q, N, sel, cnt, ws, n_q=n_q)
+
+    def do_attend():
+        zha.attend(cfg, K, V, tree, Q, N, sel, cnt, O, ws, n_q=n_q)
+
+    def do_dense():
+        zha.dense(cfg, K, V, Q, N, Od, ws, n_q=n_q)
+
+    for fn in (do_route, do_attend, do_dense):
+        fn()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    graphs = []
+    for fn in (do_route, do_attend, do_dense):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            fn()
+        graphs.append(g)
+    torch.cuda.synchronize()
+    g_route, g_att, g_dense = graphs
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        g_route.replay(); g_att.replay()
+    torch.cuda.synchronize()
+    bits = zha.get_status(clear=True)
+    if bits:
+        raise RuntimeError(f"device status after warm-up: {zha.status_names(bits)}")
+    stream = torch.cuda.current_stream()
+    K_steps = args.steps
+    D.barrier(rank, dev)
+    torch.cuda.synchronize()
+    clocks = Clocks(rank.local) if rank.leader else None
+    time.sleep(0.25)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_steps)]
+    for k in range(K_steps):
+        flush.zero_()
+        e = ev[k]
+        e[0].record(stream); g_route.replay(); e[1].record(stream); g_att.replay(); e[2].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else None
+    bits = zha.get_status(clear=True)
+    if bits:
+        raise RuntimeError(f"device status after the timed steps: {zha.status_names(bits)}")
+    t_route = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_att = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_step = t_route + t_att
+    D.barrier(rank, dev)
+    t_max = D.max_over_ranks(t_step, rank, dev)
+    queries = w.batch * n_q * K_steps * rank.world
+    value = queries / t_max
+    # work of the method: every (query, head) row attends over |I(q)| keys (QK and PV,
+    # 2 flops per multiply-add each); the tensor cores load `steps` 64-key blocks for 128 rows
+    blocks = cnt.to(torch.int64).sum().item()
+    tail = sum((Np - (Np // w.B) * w.B) + i + 1 for i in range(n_q)) * w.batch * w.Hq
+    # rows whose block 0 was not selected still read key 0 (the sink)
+    sink = ((cnt == 0) | (sel[..., 0] != 0)).sum().item() if Np >= w.B else 0
+    keys = blocks * w.B + tail + sink
+    useful_flops = keys * w.d * 4
+    issued_flops = steps_v.to(torch.int64).sum().item() * 128 * 64 * w.d * 4
+    peak, peak_src = measured_peaks("bf16_tflops_sustained")
+    att_tflops = useful_flops / (t_att / K_steps) / 1e12
+    issued_tflops = issued_flops / (t_att / K_steps) / 1e12
+    # dense causal prefill, same kernel without the selection
+    dense_ev = []
+    for _ in range(5):
+        flush.zero_()
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream); g_dense.replay(); b_.record(stream)
+        dense_ev.append((a_, b_))
+    torch.cuda.synchronize()
+    t_dense = sum(a_.elapsed_time(b_) for a_, b_ in dense_ev[1:]) / 4 / 1e3
+    dense_flops = sum(Np + i + 1 for i in range(n_q)) * w.batch * w.Hq * w.d * 4
+    # end to end: host Q and chunk K/V in, O out, through the public calls
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = max(1, min(K_steps, 10))
+        qh = Q.cpu().pin_memory()
+        kh = K[:, :, Np:].cpu().pin_memory()
+        vh = V[:, :, Np:].cpu().pin_memory()
+        oh = torch.empty_like(O, device="cpu").pin_memory()
+        torch.cuda.synchronize()
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        for _ in range(e2e_steps):
+            Q.copy_(qh, non_blocking=True)
+            K[:, :, Np:].copy_(kh, non_blocking=True)
+            V[:, :, Np:].copy_(vh, non_blocking=True)
+            do_route()
+            do_attend()
+            oh.copy_(O, non_blocking=True)
+        b_.record(stream)
+        torch.cuda.synchronize()
+        t_e2e = D.max_over_ranks(a_.elapsed_time(b_) / 1e3, rank, dev)
+        e2e = {"value": w.batch * n_q * e2e_steps * rank.world / t_e2e, "unit": UNIT,
+               "h2d_bytes_per_step": qh.numel() * 2 + kh.numel() * 2 + vh.numel() * 2,
+               "d2h_bytes_per_step": oh.numel() * 4, "steps": e2e_steps,
+               "note": "zha_route + zha_attend per chunk (not graphed), pinned host Q, chunk K/V and O"}
+    cpu = None
+    if rank.leader and rank.world == 1 and not args.no_cpu_baseline:
+        per_head, done, setup = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": 1.0 / (per_head * w.Hq), "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{done} single-head route+attend calls of the fp64 C oracle for chunk queries of one "
+                         f"(sequence, KV head) slice of {w.name} (tree built once, {setup:.1f}s untimed), scaled "
+                         f"to chunk queries of all {w.Hq} heads"}
+    if rank.leader:
+        line = {
+            "metric": PREFILL_METRIC, "value": value, "unit": UNIT, "n_gpus": rank.world, "steps": K_steps,
+            "warmup": args.warmup, "ms_per_step": t_max / K_steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: batch {w.batch} per GPU, {w.Hq} query / {w.Hkv} KV heads, d {w.d}, "
+                                   f"bf16, prefix N={Np} in the tree, chunk of {n_q} causal queries, leaf block "
+                                   f"{w.B}, branching {w.b}, p={w.p}",
+                       "global_batch": w.batch * rank.world, "seq_len": N_cap, "parallelism": f"dp{rank.world}",
+                       "l2": "flushed (256 MiB write) before every timed step",
+                       "step": "zha_route + zha_attend of one chunk, each one CUDA graph"},
+            "roofline": {"bound": "tensor", "kernel": "attend phase (plan + attend_prefill_kernel + merge)",
+                         "achieved": att_tflops, "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak,
+                         "traffic": None, "peak_source": f"{peak_src} bf16 dense (sustained)",
+                         "algorithmic_flops_per_launch": useful_flops, "issued_mma_flops_per_launch": issued_flops,
+                         "issued_tflops": issued_tflops},
+            "phases_ms": {"route": t_route / K_steps * 1e3, "attend": t_att / K_steps * 1e3},
+            "keys_per_row": keys / (w.batch * n_q * w.Hq),
+            "dense_baseline": {"ms_per_step": t_dense * 1e3, "tflops": dense_flops / t_dense / 1e12,
+                               "queries_per_s": w.batch * n_q / t_dense,
+                               "speedup_of_tree": t_dense / (t_max / K_steps)},
+            "gpu_launches": 8 * K_steps,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    del graphs, g_route, g_att, g_dense
+    D.finish(rank)
+    return 0
+
+
 def main():
     args = parse()
     from hierarchical_tree_indexed_b200 import dist as D
@@ -378,6 +558,8 @@ def main():
         return reference_arm(args, rank)
     if args.sweep:
         return sweep(args, rank)
+    if workload(args).prefill:
+        return prefill_main(args, rank, workload(args))
 
     import torch
 

@@ -1,6 +1,8 @@
 // zha_abi.cu -- the C ABI (include/zha.h): argument checks, buffer layouts and
 // kernel launches.  Every step of the path runs in the kernels included below;
 // this file only validates, lays out the caller's buffers and launches.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -18,6 +20,7 @@
 #include "zha_plan.cuh"
 #include "zha_route.cuh"
 #include "zha_attend.cuh"
+#include "zha_prefill.cuh"
 
 using namespace zha;
 
@@ -347,6 +350,211 @@ int run_plan(const zha_config* c, const WsLayout& wl, const TreeLayout& lay, con
     return check_launch("plan");
 }
 
+// ---------------------------------------------------------------- chunked prefill (n_q > 1)
+// Workspace of the prefill calls: route spill areas, the superblock plan, the
+// partials of every row and the accounting counters.
+struct PfLayout {
+    int64_t slices, R, rows, cand_cap, par_cap, nJ_cap, item_cap, n1_cap, pair_cap;
+    size_t off_spill_sc, off_spill_par, off_cand, off_totals, off_hdr, off_ctr, off_row_cnt, off_row_pairs, off_row_off;
+    size_t off_jcount, off_jcur, off_pairs, off_items, off_tail_ml, off_tail_o, off_sel_ml, off_sel_o, off_steps;
+    size_t total;
+};
+
+int pf_layout(const zha_config* c, int n_q, const TreeLayout& t, PfLayout* p) {
+    if (n_q < 2) return fail(ZHA_ERR_INVALID_ARG, "n_q=%d", n_q);
+    if (c->dtype != ZHA_BF16) return fail(ZHA_ERR_UNSUPPORTED, "n_q=%d: chunked prefill takes bf16 K, V and Q", n_q);
+    if (c->B != 64) return fail(ZHA_ERR_UNSUPPORTED, "n_q=%d: chunked prefill needs leaf blocks of B = 64 keys", n_q);
+    const int G = c->Hq / c->Hkv;
+    p->n1_cap = std::max<int64_t>(t.ncap[0], 1);
+    if (p->n1_cap > (int64_t{kBitmapWords} * 32) * kPairsPerRow)
+        return fail(ZHA_ERR_UNSUPPORTED, "chunked prefill: N_cap=%lld gives more than %d leaf blocks",
+                    (long long)c->N_cap, kBitmapWords * 32 * kPairsPerRow);
+    p->slices = static_cast<int64_t>(c->batch) * c->Hkv;
+    p->R = static_cast<int64_t>(n_q) * G;
+    p->rows = p->slices * p->R;
+    if (p->rows * kPairsPerRow > (int64_t{1} << 31) - 1)
+        return fail(ZHA_ERR_UNSUPPORTED, "chunked prefill: batch * n_q * Hq = %lld rows is too many", (long long)p->rows);
+    p->cand_cap = t.ncap[0] + c->b;
+    p->par_cap = std::max<int64_t>(t.ncap[0], 1);
+    p->nJ_cap = (p->n1_cap + 3) / 4 + 1;
+    p->pair_cap = p->rows * kPairsPerRow;
+    p->item_cap = p->slices * ((p->R * kPairsPerRow + kTileRows - 1) / kTileRows + p->nJ_cap);
+    const size_t D = static_cast<size_t>(c->d);
+    size_t off = 0;
+    p->off_spill_sc = off;  off = align256(off + sizeof(float) * kPRSpillWarps * p->cand_cap);
+    p->off_spill_par = off; off = align256(off + sizeof(int32_t) * kPRSpillWarps * 2 * p->par_cap);
+    p->off_cand = off;      off = align256(off + sizeof(int32_t) * p->rows);
+    p->off_totals = off;    off = align256(off + sizeof(unsigned long long) * p->slices * kSBOpts);
+    p->off_hdr = off;       off = align256(off + sizeof(int32_t) * 8);
+    p->off_ctr = off;       off = align256(off + sizeof(int32_t) * 2);
+    p->off_row_cnt = off;   off = align256(off + sizeof(int32_t) * p->rows);
+    p->off_row_pairs = off; off = align256(off + sizeof(int32_t) * p->rows);
+    p->off_row_off = off;   off = align256(off + sizeof(int32_t) * p->rows);
+    p->off_jcount = off;    off = align256(off + sizeof(int32_t) * p->slices * p->nJ_cap);
+    p->off_jcur = off;      off = align256(off + sizeof(int32_t) * p->slices * p->nJ_cap);
+    p->off_pairs = off;     off = align256(off + sizeof(int4) * p->pair_cap);
+    p->off_items = off;     off = align256(off + sizeof(int4) * p->item_cap);
+    p->off_tail_ml = off;   off = align256(off + sizeof(float2) * p->rows);
+    p->off_tail_o = off;    off = align256(off + sizeof(float) * p->rows * D);
+    p->off_sel_ml = off;    off = align256(off + sizeof(float2) * p->pair_cap);
+    p->off_sel_o = off;     off = align256(off + sizeof(float) * p->pair_cap * D);
+    p->off_steps = off;     off = align256(off + sizeof(int32_t) * p->slices);
+    p->total = off;
+    return ZHA_OK;
+}
+
+// Tiled TMA map over K or V viewed as [batch*Hkv][N_cap][d] bf16, boxes of 64 keys x 64
+// columns with the 128-byte swizzle the tensor-core operands expect.
+int make_kv_map(const zha_config* c, const void* base, CUtensorMap* map) {
+    static std::mutex mu;
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            ZHA_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+            if (q != cudaDriverEntryPointSuccess || !fn) return fail(ZHA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+            encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+    }
+    if (reinterpret_cast<uintptr_t>(base) % 16) return fail(ZHA_ERR_INVALID_ARG, "K/V must be 16-byte aligned");
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(c->d), static_cast<cuuint64_t>(c->N_cap),
+                                static_cast<cuuint64_t>(c->batch) * c->Hkv};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(c->d) * 2, static_cast<cuuint64_t>(c->N_cap) * c->d * 2};
+    const cuuint32_t box[3] = {64, 64, 1};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                              estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ZHA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return ZHA_OK;
+}
+
+template <int D, int NVR>
+int run_proute_t(const PRouteArgs& a, int64_t rows, cudaStream_t st) {
+    auto kern = route_prefill_kernel<uint16_t, D, NVR>;
+    ZHA_TRY(allow_smem(kern, sizeof(PRouteSmem)));
+    DevInfo di;
+    ZHA_TRY(dev_info(&di));
+    const int64_t want = (rows + kPRWarps - 1) / kPRWarps;
+    const int grid = static_cast<int>(std::min<int64_t>({want, 2 * di.sms, kPRSpillWarps / kPRWarps}));
+    kern<<<grid, kPRThreads, sizeof(PRouteSmem), st>>>(a);
+    return check_launch("route_prefill");
+}
+
+template <int D>
+int run_proute(const zha_config* c, const TreeLayout& lay, const PfLayout& pl, const void* tree, const void* Q,
+               int n_q, const int32_t* N, int32_t* sel, int32_t* cnt, int32_t sel_cap, void* ws, cudaStream_t st) {
+    PRouteArgs a{};
+    a.tree = tree_view(lay, const_cast<void*>(tree));
+    a.Q = Q; a.N = N; a.sel = sel; a.sel_count = cnt;
+    a.cand = at<int32_t>(ws, pl.off_cand);
+    a.spill_sc = at<float>(ws, pl.off_spill_sc);
+    a.spill_par = at<int32_t>(ws, pl.off_spill_par);
+    a.cand_cap = pl.cand_cap; a.par_cap = pl.par_cap; a.N_cap = c->N_cap;
+    a.sel_cap = sel_cap; a.batch = c->batch; a.Hq = c->Hq; a.Hkv = c->Hkv; a.B = c->B; a.b = c->b;
+    a.L_fixed = c->L_fixed; a.n_q = n_q;
+    a.scale = scale_of(c);
+    for (int l = 0; l < kMaxLevels; ++l) a.p[l] = c->p[l];
+    const int64_t rows = static_cast<int64_t>(c->batch) * n_q * c->Hq;
+    if (c->b <= 4) return run_proute_t<D, 4>(a, rows, st);
+    if (c->b <= 8) return run_proute_t<D, 8>(a, rows, st);
+    if (c->b <= 16) return run_proute_t<D, 16>(a, rows, st);
+    return run_proute_t<D, 32>(a, rows, st);
+}
+
+PAttnArgs pattn_args(const zha_config* c, const PfLayout& pl, const TreeLayout& lay, const void* tree, const void* Q,
+                     int n_q, const int32_t* N, const int32_t* sel, const int32_t* cnt, int32_t sel_cap, float* O,
+                     void* ws, int dense) {
+    PAttnArgs a{};
+    a.Q = Q; a.O = O; a.N = N;
+    a.n_tree = tree ? tree_view(lay, const_cast<void*>(tree)).n_tree : nullptr;
+    a.sel = sel; a.sel_cap = sel_cap;
+    a.row_cnt = at<int32_t>(ws, pl.off_row_cnt);
+    a.pairs = at<int4>(ws, pl.off_pairs);
+    a.items = at<int4>(ws, pl.off_items);
+    a.hdr = at<int32_t>(ws, pl.off_hdr);
+    a.ctr = at<int32_t>(ws, pl.off_ctr);
+    a.tail_ml = at<float2>(ws, pl.off_tail_ml);
+    a.tail_o = at<float>(ws, pl.off_tail_o);
+    a.sel_ml = at<float2>(ws, pl.off_sel_ml);
+    a.sel_o = at<float>(ws, pl.off_sel_o);
+    a.steps = at<int32_t>(ws, pl.off_steps);
+    a.N_cap = c->N_cap; a.item_cap = pl.item_cap;
+    a.n_q = n_q; a.Hq = c->Hq; a.Hkv = c->Hkv; a.G = c->Hq / c->Hkv; a.B = c->B;
+    a.R = static_cast<int>(pl.R); a.slices = static_cast<int>(pl.slices);
+    a.tiles = static_cast<int>((pl.R + kTileRows - 1) / kTileRows);
+    a.dense = dense;
+    a.qscale = scale_of(c) * 1.4426950408889634f;
+    return a;
+}
+
+template <int D>
+int run_pattn_t(const zha_config* c, const PAttnArgs& a, const void* K, const void* V, cudaStream_t st) {
+    CUtensorMap mk, mv;
+    ZHA_TRY(make_kv_map(c, K, &mk));
+    ZHA_TRY(make_kv_map(c, V, &mv));
+    auto kern = attend_prefill_kernel<D>;
+    ZHA_TRY(allow_smem(kern, PAttnLayout<D>::kSmem));
+    DevInfo di;
+    ZHA_TRY(dev_info(&di));
+    kern<<<2 * di.sms, 128, PAttnLayout<D>::kSmem, st>>>(mk, mv, a);
+    return check_launch("attend_prefill");
+}
+
+int run_pattn(const zha_config* c, const PAttnArgs& a, const void* K, const void* V, cudaStream_t st) {
+    return c->d == 128 ? run_pattn_t<128>(c, a, K, V, st) : run_pattn_t<64>(c, a, K, V, st);
+}
+
+// Plan + tensor-core attention + merge of a prefill chunk.
+int run_prefill_attend(const zha_config* c, const TreeLayout& lay, const PfLayout& pl, const void* K, const void* V,
+                       const void* tree, const void* Q, int n_q, const int32_t* N, const int32_t* sel,
+                       const int32_t* cnt, int32_t sel_cap, float* O, void* ws, cudaStream_t st) {
+    PPlanArgs p{};
+    p.sel = sel; p.sel_count = cnt;
+    p.n_tree = tree_view(lay, const_cast<void*>(tree)).n_tree;
+    p.totals = at<unsigned long long>(ws, pl.off_totals);
+    p.hdr = at<int32_t>(ws, pl.off_hdr);
+    p.row_cnt = at<int32_t>(ws, pl.off_row_cnt);
+    p.row_pairs = at<int32_t>(ws, pl.off_row_pairs);
+    p.row_off = at<int32_t>(ws, pl.off_row_off);
+    p.jcount = at<int32_t>(ws, pl.off_jcount);
+    p.jcur = at<int32_t>(ws, pl.off_jcur);
+    p.pairs = at<int4>(ws, pl.off_pairs);
+    p.items = at<int4>(ws, pl.off_items);
+    p.nJ_cap = pl.nJ_cap; p.item_cap = pl.item_cap; p.n1_cap = pl.n1_cap;
+    p.sel_cap = sel_cap; p.n_q = n_q; p.Hq = c->Hq; p.Hkv = c->Hkv; p.G = c->Hq / c->Hkv; p.B = c->B;
+    p.R = static_cast<int>(pl.R); p.slices = static_cast<int>(pl.slices);
+    const int chunks = static_cast<int>(pl.slices) * kPlanChunks;
+    ZHA_CUDA(cudaMemsetAsync(at<int32_t>(ws, pl.off_steps), 0, sizeof(int32_t) * pl.slices, st));
+    prefill_count_kernel<<<chunks, 256, 0, st>>>(p);
+    prefill_choose_kernel<<<1, 1024, 0, st>>>(p);
+    prefill_pairs_kernel<<<chunks, 256, 0, st>>>(p);
+    prefill_scan_kernel<<<static_cast<int>(pl.slices), 1024, 0, st>>>(p);
+    prefill_scatter_kernel<<<chunks, 256, 0, st>>>(p);
+    ZHA_TRY(check_launch("prefill plan"));
+    const PAttnArgs a = pattn_args(c, pl, lay, tree, Q, n_q, N, sel, cnt, sel_cap, O, ws, 0);
+    ZHA_TRY(run_pattn(c, a, K, V, st));
+    PMergeArgs m{};
+    m.O = O;
+    m.tail_ml = a.tail_ml; m.tail_o = a.tail_o; m.sel_ml = a.sel_ml; m.sel_o = a.sel_o;
+    m.row_pairs = p.row_pairs; m.row_off = p.row_off;
+    m.n_q = n_q; m.Hq = c->Hq; m.Hkv = c->Hkv; m.G = a.G; m.R = a.R; m.rows = pl.rows;
+    const unsigned grid = static_cast<unsigned>((pl.rows * 32 + 255) / 256);
+    if (c->d == 128) merge_prefill_kernel<128><<<grid, 256, 0, st>>>(m);
+    else merge_prefill_kernel<64><<<grid, 256, 0, st>>>(m);
+    return check_launch("merge_prefill");
+}
+
+int pf_setup(const zha_config* cfg, int n_q, TreeLayout* t, PfLayout* p, const void* ws, size_t ws_bytes) {
+    ZHA_TRY(tree_layout(cfg, t));
+    ZHA_TRY(pf_layout(cfg, n_q, *t, p));
+    if (!ws) return fail(ZHA_ERR_INVALID_ARG, "ws is null");
+    if (ws_bytes < p->total) return fail(ZHA_ERR_WORKSPACE, "workspace of %zu B < %zu B needed", ws_bytes, p->total);
+    return ZHA_OK;
+}
+
 // Dispatch on (dtype, d).
 #define ZHA_DISPATCH(c, FN, ...)                                                          \
     ((c)->dtype == ZHA_BF16 ? ((c)->d == 128 ? FN<uint16_t, 128>(__VA_ARGS__) : FN<uint16_t, 64>(__VA_ARGS__)) \
@@ -441,6 +649,12 @@ int zha_workspace_bytes(const zha_config* cfg, int32_t n_q, size_t* bytes) {
     WsLayout w;
     ZHA_TRY(need(bytes, "bytes"));
     ZHA_TRY(tree_layout(cfg, &t));
+    if (n_q > 1) {
+        PfLayout p;
+        ZHA_TRY(pf_layout(cfg, n_q, t, &p));
+        *bytes = p.total;
+        return ZHA_OK;
+    }
     ZHA_TRY(ws_layout(cfg, n_q, t, &w));
     *bytes = w.total;
     return ZHA_OK;
@@ -452,6 +666,13 @@ int zha_workspace_stats(const zha_config* cfg, int32_t n_q, size_t* rows_offset,
     ZHA_TRY(need(rows_offset, "rows_offset"));
     ZHA_TRY(need(cand_offset, "cand_offset"));
     ZHA_TRY(tree_layout(cfg, &t));
+    if (n_q > 1) {
+        PfLayout p;
+        ZHA_TRY(pf_layout(cfg, n_q, t, &p));
+        *rows_offset = p.off_steps;
+        *cand_offset = p.off_cand;
+        return ZHA_OK;
+    }
     ZHA_TRY(ws_layout(cfg, n_q, t, &w));
     *rows_offset = w.off_rows;
     *cand_offset = w.off_cand;
@@ -464,7 +685,7 @@ int zha_workspace_init(const zha_config* cfg, void* ws, size_t ws_bytes, zha_str
     ZHA_TRY(tree_layout(cfg, &t));
     ZHA_TRY(ws_layout(cfg, 1, t, &w));
     ZHA_TRY(check_ws(w, ws, ws_bytes));
-    ZHA_CUDA(cudaMemsetAsync(ws, 0, w.total, stream));
+    ZHA_CUDA(cudaMemsetAsync(ws, 0, ws_bytes, stream));
     return ZHA_OK;
 }
 
@@ -498,6 +719,18 @@ int zha_route(const zha_config* cfg, const void* tree, const void* Q, int32_t n_
               int32_t* sel_count, int32_t sel_cap, void* ws, size_t ws_bytes, zha_stream_t stream) {
     TreeLayout t;
     WsLayout w;
+    if (n_q > 1) {
+        PfLayout p;
+        ZHA_TRY(pf_setup(cfg, n_q, &t, &p, ws, ws_bytes));
+        ZHA_TRY(need(tree, "tree"));
+        ZHA_TRY(need(Q, "Q"));
+        ZHA_TRY(need(N, "N"));
+        ZHA_TRY(need(sel, "sel"));
+        ZHA_TRY(need(sel_count, "sel_count"));
+        if (sel_cap < 1) return fail(ZHA_ERR_INVALID_ARG, "sel_cap=%d", sel_cap);
+        return cfg->d == 128 ? run_proute<128>(cfg, t, p, tree, Q, n_q, N, sel, sel_count, sel_cap, ws, stream)
+                             : run_proute<64>(cfg, t, p, tree, Q, n_q, N, sel, sel_count, sel_cap, ws, stream);
+    }
     ZHA_TRY(tree_layout(cfg, &t));
     ZHA_TRY(ws_layout(cfg, n_q, t, &w));
     ZHA_TRY(check_ws(w, ws, ws_bytes));
@@ -517,6 +750,20 @@ int zha_attend(const zha_config* cfg, const void* K, const void* V, const void* 
                size_t ws_bytes, zha_stream_t stream) {
     TreeLayout t;
     WsLayout w;
+    if (n_q > 1) {
+        PfLayout p;
+        ZHA_TRY(pf_setup(cfg, n_q, &t, &p, ws, ws_bytes));
+        ZHA_TRY(need(K, "K"));
+        ZHA_TRY(need(V, "V"));
+        ZHA_TRY(need(tree, "tree"));
+        ZHA_TRY(need(Q, "Q"));
+        ZHA_TRY(need(N, "N"));
+        ZHA_TRY(need(O, "O"));
+        ZHA_TRY(need(sel, "sel (n_q > 1 takes the selection lists)"));
+        ZHA_TRY(need(sel_count, "sel_count"));
+        if (sel_cap < 1) return fail(ZHA_ERR_INVALID_ARG, "sel_cap=%d", sel_cap);
+        return run_prefill_attend(cfg, t, p, K, V, tree, Q, n_q, N, sel, sel_count, sel_cap, O, ws, stream);
+    }
     ZHA_TRY(tree_layout(cfg, &t));
     ZHA_TRY(ws_layout(cfg, n_q, t, &w));
     ZHA_TRY(check_ws(w, ws, ws_bytes));
@@ -586,6 +833,18 @@ int zha_dense(const zha_config* cfg, const void* K, const void* V, const void* Q
               float* O, void* ws, size_t ws_bytes, zha_stream_t stream) {
     TreeLayout t;
     WsLayout w;
+    if (n_q > 1) {
+        PfLayout p;
+        ZHA_TRY(pf_setup(cfg, n_q, &t, &p, ws, ws_bytes));
+        ZHA_TRY(need(K, "K"));
+        ZHA_TRY(need(V, "V"));
+        ZHA_TRY(need(Q, "Q"));
+        ZHA_TRY(need(N, "N"));
+        ZHA_TRY(need(O, "O"));
+        ZHA_CUDA(cudaMemsetAsync(at<int32_t>(ws, p.off_steps), 0, sizeof(int32_t) * p.slices, stream));
+        const PAttnArgs a = pattn_args(cfg, p, t, nullptr, Q, n_q, N, nullptr, nullptr, 0, O, ws, 1);
+        return run_pattn(cfg, a, K, V, stream);
+    }
     ZHA_TRY(tree_layout(cfg, &t));
     ZHA_TRY(ws_layout(cfg, n_q, t, &w));
     ZHA_TRY(check_ws(w, ws, ws_bytes));

@@ -102,16 +102,19 @@ int zha_tree_level(const zha_config *cfg, int32_t level, size_t *khat_offset, si
 int zha_tree_count_offset(const zha_config *cfg, size_t *offset);
 
 /* Bytes of the workspace that zha_route/zha_attend/zha_decode/zha_dense need
- * for n_q queries per sequence (decode: n_q = 1).  The workspace must be
- * zeroed once after allocation (zha_workspace_init); calls leave it reusable. */
+ * for n_q queries per sequence (decode: n_q = 1; a chunked prefill: n_q > 1,
+ * which takes bf16 K/V/Q, leaf blocks of B = 64 and at most 262144 leaf blocks,
+ * else ZHA_ERR_UNSUPPORTED).  The workspace must be zeroed once after allocation
+ * (zha_workspace_init); calls leave it reusable. */
 int zha_workspace_bytes(const zha_config *cfg, int32_t n_q, size_t *bytes);
 int zha_workspace_init(const zha_config *cfg, void *ws, size_t ws_bytes, zha_stream_t stream);
 
 /* Accounting left in the workspace by the last calls, for measuring the bytes
  * the path touches: byte offsets of int32 rows[batch*Hkv] (keys gathered per
- * (sequence, KV head) by the last zha_attend / zha_dense plan) and int32
- * cand[batch][n_q][Hq] (tree nodes scored over all levels by the last
- * zha_route). */
+ * (sequence, KV head) by the last zha_attend / zha_dense plan; with n_q > 1 the
+ * number of 64-key blocks the tensor-core attention loaded, each for up to 128
+ * query rows) and int32 cand[batch][n_q][Hq] (tree nodes scored over all levels
+ * by the last zha_route). */
 int zha_workspace_stats(const zha_config *cfg, int32_t n_q, size_t *rows_offset, size_t *cand_offset);
 
 /*
@@ -151,6 +154,14 @@ int zha_append(const zha_config *cfg, void *K, void *V, const void *k_new, const
  * first sel_cap ids are written).  It also leaves in ws the gather plan of
  * zha_attend for these selections (see zha_attend with sel == NULL).
  */
+/*
+ * zha_route with n_q > 1 -- a chunked prefill.  N[s] counts the keys in the
+ * cache including the chunk's n_q keys, which the caller has written at rows
+ * [N[s] - n_q, N[s]) of K and V; the tree must index exactly the N[s] - n_q keys
+ * before the chunk (else ZHA_ERR_INVALID_ARG on the device and empty
+ * selections).  Query i of the chunk sits at t = N[s] - n_q + i.  Each (query,
+ * query head) is routed as above, independently.  No gather plan is left in ws.
+ */
 int zha_route(const zha_config *cfg, const void *tree, const void *Q, int32_t n_q, const int32_t *N,
               int32_t *sel, int32_t *sel_count, int32_t sel_cap, void *ws, size_t ws_bytes,
               zha_stream_t stream);
@@ -164,6 +175,17 @@ int zha_route(const zha_config *cfg, const void *tree, const void *Q, int32_t n_
  * O is fp32 [batch][n_q][Hq][d].  tree is read only for n_1.  With sel == NULL
  * the gather plan that the last zha_route on this workspace left is used
  * (sel_count and sel_cap are then ignored).
+ */
+/*
+ * zha_attend with n_q > 1 -- the chunked prefill's attention, on the tensor
+ * cores.  Same index set with C_cur(t) = [n_1*B, t], the causal tail (n_1 = the
+ * tree's leaf blocks, the tree indexing the N[s] - n_q keys before the chunk).
+ * sel and sel_count are required; each row's list must be ascending and below
+ * n_1 (else ZHA_ERR_INVALID_ARG on the device, and the valid prefix is used).
+ * The softmax weights are rounded to bf16 for the P V product (their sum is
+ * taken over the rounded values), so an output moves by at most 2^-8 max|v|
+ * against exact attention over the same set.  Deterministic: the same inputs
+ * give bitwise the same outputs.
  */
 int zha_attend(const zha_config *cfg, const void *K, const void *V, const void *tree,
                const void *Q, int32_t n_q, const int32_t *N, const int32_t *sel,
@@ -202,7 +224,9 @@ int zha_decode(const zha_config *cfg, void *K, void *V, void *tree, const void *
                size_t ws_bytes, zha_stream_t stream);
 
 /* zha_dense -- the in-library dense baseline: attention of q [batch][1][Hq][d]
- * over every key [0, N[s]), with the same loader as zha_attend. */
+ * over every key [0, N[s]), with the same loader as zha_attend.  With n_q > 1,
+ * causal dense attention of the chunk's queries (query i over [0, N[s] - n_q +
+ * i]) on the tensor-core kernel of zha_attend's prefill; tree is not needed. */
 int zha_dense(const zha_config *cfg, const void *K, const void *V, const void *Q, int32_t n_q,
               const int32_t *N, float *O, void *ws, size_t ws_bytes, zha_stream_t stream);
 

@@ -73,7 +73,11 @@ def test_null_pointers_and_small_workspace_are_refused_on_the_host(lib):
     assert lib.zha_append(cc, None, None, None, None, None, None, None) == 1
     need = zha.workspace_bytes(c)
     assert lib.zha_route(cc, 1, 1, 1, 1, 1, 1, 16, 256, need - 1, None) == 6
-    assert lib.zha_route(cc, 1, 1, 2, 1, 1, 1, 16, 256, need, None) == 2     # n_q > 1: not a decode call
+    pneed = zha.workspace_bytes(c, 64)                                      # chunked prefill of 64 queries
+    assert lib.zha_route(cc, 1, 1, 64, 1, 1, 1, 16, 256, pneed - 1, None) == 6
+    assert lib.zha_attend(cc, 1, 1, 1, 1, 64, 1, None, 1, 16, 1, 1, pneed, None) == 1   # prefill needs sel
+    cf = cfg(batch=1, N_cap=4096, dtype="f32")
+    assert lib.zha_route(ctypes.byref(cf.c()), 1, 1, 64, 1, 1, 1, 16, 256, pneed, None) == 2   # bf16 only
     assert lib.zha_attend(cc, 1, 1, 1, 1, 1, 1, 1, 1, 0, 1, 256, need, None) == 1   # sel_cap 0
     assert lib.zha_attend(cc, 1, 1, 1, 1, 1, 1, 1, 1, 1, None, 256, need, None) == 1   # O null
     assert lib.zha_decode(cc, None, None, None, None, None, None, None, None, 256, need, None) == 1
