@@ -460,14 +460,19 @@ struct PAttnArgs {
 };
 
 struct PAttnCtl {
-    uint64_t kv_full[2];
-    uint64_t s_done, o_done;
+    uint64_t kv_full[2];      // TMA -> MMA: K and V of a block landed in buffer i
+    uint64_t s_full[2];       // MMA -> softmax: S of the block in TMEM buffer i
+    uint64_t p_full[2];       // softmax -> MMA: P of step g (buffer g & 1) written, O rescaled
+    uint64_t o_done;          // MMA -> all: every MMA issued so far (through P V of the step) completed
     uint32_t tmem;
     int item;
     int abort;
     int pad;
     uint32_t bitmap[kBitmapWords];
 };
+
+constexpr int kPAThreads = 160;   // 4 softmax warps (one query row per thread) + 1 TMA/MMA warp
+constexpr float kRescaleLog2 = 8.0f;   // lazy rescale: P stays below 2^8 between rescales
 
 template <int D>
 struct PAttnLayout {
@@ -478,13 +483,12 @@ struct PAttnLayout {
     static constexpr bool kPInK = kKVBytes >= kPBytes;         // P overwrites the consumed K block
     static constexpr uint32_t kOffK = kQBytes;
     static constexpr uint32_t kOffV = kOffK + 2 * kKVBytes;
-    static constexpr uint32_t kOffP = kOffV + 2 * kKVBytes;
-    static constexpr uint32_t kOffCtl = kOffP + (kPInK ? 0 : kPBytes);
+    static constexpr uint32_t kOffP = kOffV + 2 * kKVBytes;    // two P buffers when P does not fit in K
+    static constexpr uint32_t kOffCtl = kOffP + (kPInK ? 0 : 2 * kPBytes);
     static constexpr size_t kSmem = kOffCtl + sizeof(PAttnCtl) + 1024;   // + alignment slack
 };
 
-// Bounded wait that every thread of the CTA takes; a timeout is recorded once
-// and later waits of the CTA return at once.
+// Bounded wait; a timeout is recorded once and later waits of the CTA return at once.
 __device__ __forceinline__ void pwait(uint64_t* bar, uint32_t parity, PAttnCtl* ctl) {
     if (*reinterpret_cast<volatile int*>(&ctl->abort)) return;
     if (!mbar_wait_bounded(bar, parity)) {
@@ -493,8 +497,44 @@ __device__ __forceinline__ void pwait(uint64_t* bar, uint32_t parity, PAttnCtl* 
     }
 }
 
+__device__ __forceinline__ float fast_exp2(float x) {   // the SFU's 2^x (x = -inf gives +0)
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
+        "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]),
+        "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
+        "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Iterates the key offsets of an item's blocks: the causal tail in order, or the
+// set bits of the superblock bitmap in ascending order.
+struct BlockCursor {
+    bool tail;
+    int64_t k0, jb0;
+    int nwords, cw;
+    uint32_t cbits;
+    int k;
+    __device__ __forceinline__ int64_t next(const uint32_t* bitmap) {
+        if (tail) return k0 + static_cast<int64_t>(k++) * 64;
+        while (cbits == 0u && cw + 1 < nwords) cbits = bitmap[++cw];
+        const int bit = __ffs(cbits) - 1;
+        cbits &= cbits - 1u;
+        return (jb0 + cw * 32 + bit) * 64;
+    }
+};
+
 template <int D>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(kPAThreads, 2)
     attend_prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                           PAttnArgs a) {
     using Lay = PAttnLayout<D>;
@@ -506,16 +546,20 @@ __global__ void __launch_bounds__(128, 1)
     unsigned char* sK = base + Lay::kOffK;
     unsigned char* sV = base + Lay::kOffV;
     PAttnCtl* ctl = reinterpret_cast<PAttnCtl*>(base + Lay::kOffCtl);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool softmax_role = warp < 4;
 
     if (warp == 0) {
         umma::tmem_alloc(&ctl->tmem, 256);
         umma::tmem_relinquish();
     }
-    if (tid == 32) {
+    if (tid == 128) {
         mbar_init(&ctl->kv_full[0], 1);
         mbar_init(&ctl->kv_full[1], 1);
-        mbar_init(&ctl->s_done, 1);
+        mbar_init(&ctl->s_full[0], 1);
+        mbar_init(&ctl->s_full[1], 1);
+        mbar_init(&ctl->p_full[0], kTileRows);
+        mbar_init(&ctl->p_full[1], kTileRows);
         mbar_init(&ctl->o_done, 1);
         fence_mbar_init();
         ctl->abort = 0;
@@ -526,22 +570,24 @@ __global__ void __launch_bounds__(128, 1)
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem = ctl->tmem;
-    const uint32_t tS = tmem, tO = tmem + 64;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tO = tmem + 128;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     constexpr uint32_t kIdS = umma::idesc_bf16(128, 64, false);
     constexpr uint32_t kIdO = umma::idesc_bf16(128, D, true);
-    uint32_t ph_kv[2] = {0u, 0u}, ph_s = 0u, ph_o = 0u;
-    uint32_t gstep = 0;   // blocks processed by this CTA (buffer parity)
+    uint32_t gstep = 0;        // blocks processed by this CTA so far (barrier phases follow it)
     const int n_tail = a.slices * a.tiles;
     const int64_t n_sel = a.dense ? 0 : (a.hdr[2] < a.item_cap ? a.hdr[2] : a.item_cap);
     const int n_total = n_tail + static_cast<int>(n_sel);
+    auto p_buf = [&](uint32_t g) -> unsigned char* {
+        return Lay::kPInK ? sK + (g & 1u) * Lay::kKVBytes : base + Lay::kOffP + (g & 1u) * Lay::kPBytes;
+    };
 
     for (;;) {
         if (tid == 0) ctl->item = atomicAdd(&a.ctr[0], 1);
         __syncthreads();
         const int it = ctl->item;
         if (it >= n_total || *reinterpret_cast<volatile int*>(&ctl->abort)) break;
-        // ---------------- the item and this thread's row
+        // ---------------- the item and (softmax threads) this thread's row
         const bool tail = it < n_tail;
         int slice, r = 0, J = 0, selp = 0, nrows, row0 = 0;
         int64_t slot = 0;
@@ -569,25 +615,22 @@ __global__ void __launch_bounds__(128, 1)
         const bool seq_ok = N >= a.n_q && N <= a.N_cap && (a.dense || Ntree == N - a.n_q);
         if (!seq_ok && tid == 0) raise_status(ZHA_ERR_INVALID_ARG);
         if (!seq_ok) nrows = 0;
-        const bool row_ok = tid < nrows;
+        const bool row_ok = softmax_role && tid < nrows;
         const int64_t n1 = Ntree / a.B;
         const int64_t grow = prefill_sel_row(slice, r, a.Hkv, a.Hq, a.G, a.n_q);
         const int64_t t = N - a.n_q + r / a.G;
         const int32_t* list = a.sel + grow * a.sel_cap;
         const int lcnt = (!tail && row_ok) ? a.row_cnt[static_cast<int64_t>(slice) * a.R + r] : 0;
-        // block schedule (uniform over the CTA)
-        int64_t k0 = 0;
+        BlockCursor cur{};
+        cur.tail = tail;
         int nb = 0;
-        int lg = 0;
         if (tail) {
-            k0 = a.dense ? 0 : n1 * a.B;
+            cur.k0 = a.dense ? 0 : n1 * a.B;
             const int64_t tmax = N - a.n_q + (row0 + nrows - 1) / a.G;
-            nb = nrows > 0 ? static_cast<int>((tmax + 1 - k0 + 63) / 64) : 0;
-        } else {
-            lg = a.hdr[0];
+            nb = nrows > 0 ? static_cast<int>((tmax + 1 - cur.k0 + 63) / 64) : 0;
         }
-        // ---------------- Q rows -> swizzled K-major tile
-        {
+        // ---------------- Q rows -> swizzled K-major tile (softmax threads)
+        if (softmax_role) {
             const uint16_t* qrow = static_cast<const uint16_t*>(a.Q) + grow * D;
 #pragma unroll
             for (int c = 0; c < D / 8; ++c) {
@@ -597,183 +640,224 @@ __global__ void __launch_bounds__(128, 1)
             }
         }
         // ---------------- selected item: union bitmap of the superblock's blocks
-        int64_t jb0 = 0;
-        int nwords = 0;
         if (!tail) {
+            const int lg = a.hdr[0];
             const int64_t SB = 1ll << lg;
-            jb0 = static_cast<int64_t>(J) * SB;
-            const int64_t jend = min(jb0 + SB, n1);
-            nwords = static_cast<int>((jend - jb0 + 31) / 32);
-            for (int wi = tid; wi < nwords; wi += 128) ctl->bitmap[wi] = 0u;
+            cur.jb0 = static_cast<int64_t>(J) * SB;
+            const int64_t jend = min(cur.jb0 + SB, n1);
+            cur.nwords = static_cast<int>((jend - cur.jb0 + 31) / 32);
+            for (int wi = tid; wi < cur.nwords; wi += kPAThreads) ctl->bitmap[wi] = 0u;
             __syncthreads();
             if (tid == 0 && J == 0) atomicOr(&ctl->bitmap[0], 1u);   // the sink's block
             if (row_ok) {
                 for (int k = selp; k < lcnt && list[k] < jend; ++k) {   // ascending and >= jb0 by the plan
-                    const int64_t bi = list[k] - jb0;
+                    const int64_t bi = list[k] - cur.jb0;
                     atomicOr(&ctl->bitmap[bi >> 5], 1u << (bi & 31));
                 }
             }
             __syncthreads();
-            nb = 0;
             if (nrows > 0)
-                for (int wi = 0; wi < nwords; ++wi) nb += __popc(ctl->bitmap[wi]);
+                for (int wi = 0; wi < cur.nwords; ++wi) nb += __popc(ctl->bitmap[wi]);
+            cur.cbits = cur.nwords > 0 ? ctl->bitmap[0] : 0u;
         }
-        // the key offset of the block at position k of the schedule
-        int cw = 0;          // selected items: bitmap cursor (word, remaining bits)
-        uint32_t cbits = nwords > 0 ? ctl->bitmap[0] : 0u;
-        auto next_key = [&]() -> int64_t {   // call once per block, in order (selected items)
-            while (cbits == 0u && cw + 1 < nwords) cbits = ctl->bitmap[++cw];
-            const int bit = __ffs(cbits) - 1;
-            cbits &= cbits - 1u;
-            return (jb0 + cw * 32 + bit) * 64;
-        };
-        auto issue = [&](int64_t key0, uint32_t buf) {
-            unsigned char* kd = sK + buf * Lay::kKVBytes;
-            unsigned char* vd = sV + buf * Lay::kKVBytes;
-            mbar_arrive_expect_tx(&ctl->kv_full[buf], 2 * Lay::kKVBytes);
-#pragma unroll
-            for (int hh = 0; hh < H; ++hh) {
-                umma::tma_load_3d(kd + hh * 8192, &tmK, hh * 64, static_cast<int>(key0), slice, &ctl->kv_full[buf]);
-                umma::tma_load_3d(vd + hh * 8192, &tmV, hh * 64, static_cast<int>(key0), slice, &ctl->kv_full[buf]);
-            }
-        };
-        // first block
-        int64_t key_cur = 0, key_next = 0;
-        if (nb > 0) {
-            key_cur = tail ? k0 : next_key();
-            if (tid == 0) issue(key_cur, gstep & 1u);
-        }
-        umma::cp_async_wait_all();
+        if (softmax_role) umma::cp_async_wait_all();
         umma::fence_proxy_async_smem();
         __syncthreads();
 
-        float m = -1e30f, l = 0.f;
-        float o[D];
+        if (!softmax_role) {
+            // ================= TMA + MMA issue (one lane)
+            if (lane == 0 && nb > 0) {
+                int64_t keys[2];
+                auto issue = [&](int64_t key0, uint32_t buf) {
+                    unsigned char* kd = sK + buf * Lay::kKVBytes;
+                    unsigned char* vd = sV + buf * Lay::kKVBytes;
+                    mbar_arrive_expect_tx(&ctl->kv_full[buf], 2 * Lay::kKVBytes);
 #pragma unroll
-        for (int e = 0; e < D; ++e) o[e] = 0.f;
-
-        for (int k = 0; k < nb; ++k) {
-            const uint32_t buf = gstep & 1u;
-            // prefetch the next block into the other buffer (free: its last MMAs completed)
-            if (k + 1 < nb) {
-                key_next = tail ? k0 + static_cast<int64_t>(k + 1) * 64 : next_key();
-                if (tid == 0) issue(key_next, buf ^ 1u);
-            }
-            pwait(&ctl->kv_full[buf], ph_kv[buf], ctl);
-            ph_kv[buf] ^= 1u;
-            unsigned char* kb = sK + buf * Lay::kKVBytes;
-            unsigned char* vb = sV + buf * Lay::kKVBytes;
-            // keys past the end of the cache: zero their V rows (their weights are 0,
-            // but 0 * NaN would not be)
-            if (key_cur + 64 > N) {
-                const int valid = N > key_cur ? static_cast<int>(N - key_cur) : 0;
-                for (int idx = tid; idx < (64 - valid) * H * 8; idx += 128) {
-                    const int rr = valid + idx / (H * 8), rest = idx % (H * 8);
-                    *reinterpret_cast<uint4*>(vb + (rest >> 3) * 8192 + rr * 128 + ((rest & 7) << 4)) =
-                        make_uint4(0u, 0u, 0u, 0u);
+                    for (int hh = 0; hh < H; ++hh) {
+                        umma::tma_load_3d(kd + hh * 8192, &tmK, hh * 64, static_cast<int>(key0), slice, &ctl->kv_full[buf]);
+                        umma::tma_load_3d(vd + hh * 8192, &tmV, hh * 64, static_cast<int>(key0), slice, &ctl->kv_full[buf]);
+                    }
+                };
+                // waits for block (step g) in its buffer, zeroes V rows past the cache end
+                auto land = [&](uint32_t g, int64_t key0) {
+                    const uint32_t buf = g & 1u;
+                    pwait(&ctl->kv_full[buf], (g >> 1) & 1u, ctl);
+                    if (key0 + 64 > N) {
+                        unsigned char* vb = sV + buf * Lay::kKVBytes;
+                        const int valid = N > key0 ? static_cast<int>(N - key0) : 0;
+                        for (int idx = 0; idx < (64 - valid) * H * 8; ++idx) {
+                            const int rr = valid + idx / (H * 8), rest = idx % (H * 8);
+                            *reinterpret_cast<uint4*>(vb + (rest >> 3) * 8192 + rr * 128 + ((rest & 7) << 4)) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                        }
+                        umma::fence_proxy_async_smem();
+                    }
+                };
+                auto issue_s = [&](uint32_t g) {
+                    const unsigned char* kb = sK + (g & 1u) * Lay::kKVBytes;
+                    const uint32_t tS = tmem + (g & 1u) * 64;
+                    umma::fence_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t ad = umma::desc_sw128(smem_addr(sQ + (kk >> 2) * (kTileRows * 128) + (kk & 3) * 32), 16, 1024);
+                        const uint64_t bd = umma::desc_sw128(smem_addr(kb + (kk >> 2) * 8192 + (kk & 3) * 32), 16, 1024);
+                        umma::mma_bf16(tS, ad, bd, kIdS, kk > 0 ? 1u : 0u);
+                    }
+                    umma::commit(&ctl->s_full[g & 1u]);
+                };
+                const uint32_t g0 = gstep;
+                keys[0] = cur.next(ctl->bitmap);
+                issue(keys[0], g0 & 1u);
+                if (nb > 1) {
+                    keys[1] = cur.next(ctl->bitmap);
+                    issue(keys[1], (g0 + 1) & 1u);
                 }
+                land(g0, keys[0]);
+                issue_s(g0);
+                for (int k = 0; k < nb; ++k) {
+                    const uint32_t g = g0 + k;
+                    if (k + 1 < nb) {   // S of the next block overlaps this block's softmax
+                        land(g + 1, keys[(k + 1) & 1]);
+                        issue_s(g + 1);
+                    }
+                    pwait(&ctl->p_full[g & 1u], (g >> 1) & 1u, ctl);
+                    umma::fence_after_sync();
+                    const unsigned char* pb = p_buf(g);
+                    const unsigned char* vb = sV + (g & 1u) * Lay::kKVBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = umma::desc_sw128(smem_addr(pb + kk * 32), 16, 1024);
+                        const uint64_t bd = umma::desc_sw128(smem_addr(vb + kk * 2048), 8192, 1024);
+                        umma::mma_bf16(tO, ad, bd, kIdO, (k > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma::commit(&ctl->o_done);
+                    if (k + 2 < nb) {   // the block two ahead reuses this buffer once P V is done
+                        pwait(&ctl->o_done, g & 1u, ctl);
+                        keys[k & 1] = cur.next(ctl->bitmap);
+                        issue(keys[k & 1], g & 1u);
+                    }
+                }
+            }
+        } else {
+            // ================= masked online softmax, one query row per thread
+            float m_run = -1e30f, l = 0.f;   // log2 domain; P = 2^(x - m_run) <= 2^8
+            int64_t nsel_blk = (!tail && selp < lcnt) ? list[selp] : -1;
+            for (int k = 0; k < nb; ++k) {
+                const uint32_t g = gstep + k;
+                const int64_t key0 = cur.next(ctl->bitmap);
+                bool selected = false, sink_only = false;
+                if (!tail && row_ok) {
+                    const int64_t blk = key0 / 64;
+                    selected = nsel_blk == blk;
+                    if (selected) {
+                        ++selp;
+                        nsel_blk = selp < lcnt ? list[selp] : -1;
+                    }
+                    sink_only = !selected && blk == 0;
+                }
+                pwait(&ctl->s_full[g & 1u], (g >> 1) & 1u, ctl);
+                umma::fence_after_sync();
+                float sv[64];
+                umma::tmem_ld32(tmem + (g & 1u) * 64 + lane_base, sv);
+                umma::tmem_ld32(tmem + (g & 1u) * 64 + lane_base + 32, sv + 32);
+                float mx = -INFINITY;
+                if (tail) {
+                    const int64_t lim = row_ok ? t - key0 : -1;   // keys key0 + c with c <= lim
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) {
+                        sv[c] = c <= lim ? sv[c] * a.qscale : -INFINITY;
+                        mx = fmaxf(mx, sv[c]);
+                    }
+                } else {
+                    const int lim = selected ? 63 : (sink_only ? 0 : -1);
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) {
+                        sv[c] = c <= lim ? sv[c] * a.qscale : -INFINITY;
+                        mx = fmaxf(mx, sv[c]);
+                    }
+                }
+                // lazy rescale: move the reference only when the row max outgrows it by 2^8
+                bool resc = false;
+                float alpha = 1.f;
+                if (mx > m_run + kRescaleLog2) {
+                    if (l > 0.f) {
+                        resc = true;
+                        alpha = fast_exp2(m_run - mx);
+                        l *= alpha;
+                    }
+                    m_run = mx;
+                }
+                // P V of the previous block has completed (and with it every MMA issued
+                // before it, S of this block included) before O is touched or P overwrites
+                // this block's K.  (Relying on the S barrier alone for the overwrite raced:
+                // a few rows came out wrong in some runs.)
+                if (k > 0) pwait(&ctl->o_done, (g - 1) & 1u, ctl);
+                if (__any_sync(0xffffffffu, resc) && k > 0) {
+                    umma::fence_after_sync();
+#pragma unroll
+                    for (int q = 0; q < D / 32; ++q) {
+                        float ov[32];
+                        umma::tmem_ld32(tO + lane_base + q * 32, ov);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+                        tmem_st32(tO + lane_base + q * 32, ov);
+                    }
+                    tmem_wait_st();
+                }
+                float ps = 0.f;
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const float p0 = fast_exp2(sv[c] - m_run), p1 = fast_exp2(sv[c + 1] - m_run);
+                    ps += p0 + p1;
+                    const __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
+                    pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&pb2);
+                }
+                l += ps;
+                unsigned char* sP = p_buf(g);
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc)
+                    *reinterpret_cast<uint4*>(sP + tid * 128 + ((cc ^ (tid & 7)) << 4)) =
+                        make_uint4(pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
                 umma::fence_proxy_async_smem();
-                __syncthreads();
+                umma::fence_before_sync();
+                mbar_arrive(&ctl->p_full[g & 1u]);
             }
-            // S = Q K^T (128 x 64, fp32 in TMEM columns [0, 64))
-            if (tid == 0) {
+            // ---------------- this row's partial (or, dense, its output)
+            if (nb > 0) {
+                pwait(&ctl->o_done, (gstep + nb - 1) & 1u, ctl);
                 umma::fence_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t ad = umma::desc_sw128(smem_addr(sQ + (kk >> 2) * (kTileRows * 128) + (kk & 3) * 32), 16, 1024);
-                    const uint64_t bd = umma::desc_sw128(smem_addr(kb + (kk >> 2) * 8192 + (kk & 3) * 32), 16, 1024);
-                    umma::mma_bf16(tS, ad, bd, kIdS, kk > 0 ? 1u : 0u);
+                float* dst = nullptr;
+                float scale = 1.f;
+                if (row_ok) {
+                    if (a.dense) {
+                        dst = a.O + grow * D;
+                        scale = 1.0f / l;
+                    } else if (tail) {
+                        const int64_t gx = static_cast<int64_t>(slice) * a.R + r;
+                        a.tail_ml[gx] = make_float2(m_run, l);
+                        dst = a.tail_o + gx * D;
+                    } else {
+                        a.sel_ml[slot] = make_float2(m_run, l);
+                        dst = a.sel_o + slot * D;
+                    }
                 }
-                umma::commit(&ctl->s_done);
-            }
-            pwait(&ctl->s_done, ph_s, ctl);
-            ph_s ^= 1u;
-            umma::fence_after_sync();
-            // ---------------- masked online softmax of this thread's row
-            float sv[64];
-            umma::tmem_ld32(tS + lane_base, sv);
-            umma::tmem_ld32(tS + lane_base + 32, sv + 32);
-            bool selected = false, sink_only = false;
-            if (!tail && row_ok) {
-                const int64_t blk = key_cur / 64;
-                selected = selp < lcnt && list[selp] == blk;
-                if (selected) ++selp;
-                sink_only = !selected && blk == 0;
-            }
-            float mx = m;
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const bool ok = row_ok && (tail ? key_cur + c <= t : (selected || (sink_only && c == 0)));
-                sv[c] = ok ? sv[c] * a.qscale : -INFINITY;
-                mx = fmaxf(mx, sv[c]);
-            }
-            const float alpha = exp2f(m - mx);
-            float ps = 0.f;
-            uint32_t pk[32];
+                for (int q = 0; q < D / 32; ++q) {
+                    float ov[32];
+                    umma::tmem_ld32(tO + lane_base + q * 32, ov);
+                    if (dst) {
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-                const __nv_bfloat16 p0 = __float2bfloat16_rn(exp2f(sv[c] - mx));
-                const __nv_bfloat16 p1 = __float2bfloat16_rn(exp2f(sv[c + 1] - mx));
-                ps += __bfloat162float(p0) + __bfloat162float(p1);
-                pk[c >> 1] = static_cast<uint32_t>(__bfloat16_as_ushort(p0)) |
-                             (static_cast<uint32_t>(__bfloat16_as_ushort(p1)) << 16);
-            }
-            l = l * alpha + ps;
-            m = mx;
-            unsigned char* sP = Lay::kPInK ? kb : base + Lay::kOffP;
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc)
-                *reinterpret_cast<uint4*>(sP + tid * 128 + ((cc ^ (tid & 7)) << 4)) =
-                    make_uint4(pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
-            umma::fence_proxy_async_smem();
-            umma::fence_before_sync();
-            __syncthreads();
-            // O_blk = P V (128 x D, fp32 in TMEM columns [64, 64 + D))
-            if (tid == 0) {
-                umma::fence_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = umma::desc_sw128(smem_addr(sP + kk * 32), 16, 1024);
-                    const uint64_t bd = umma::desc_sw128(smem_addr(vb + kk * 2048), 8192, 1024);
-                    umma::mma_bf16(tO, ad, bd, kIdO, kk > 0 ? 1u : 0u);
+                        for (int e = 0; e < 32; e += 4)
+                            *reinterpret_cast<float4*>(dst + q * 32 + e) =
+                                make_float4(ov[e] * scale, ov[e + 1] * scale, ov[e + 2] * scale, ov[e + 3] * scale);
+                    }
                 }
-                umma::commit(&ctl->o_done);
+                umma::fence_before_sync();
             }
-            pwait(&ctl->o_done, ph_o, ctl);
-            ph_o ^= 1u;
-            umma::fence_after_sync();
-#pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
-                float ov[32];
-                umma::tmem_ld32(tO + lane_base + q * 32, ov);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) o[q * 32 + e] = fmaf(o[q * 32 + e], alpha, ov[e]);
-            }
-            umma::fence_before_sync();
-            ++gstep;
-            key_cur = key_next;
-        }
-        // ---------------- this row's partial (or, dense, its output)
-        if (row_ok && nb > 0) {
-            float* dst;
-            if (a.dense) {
-                dst = a.O + grow * D;
-                const float inv = 1.0f / l;
-#pragma unroll
-                for (int e = 0; e < D; ++e) o[e] *= inv;
-            } else if (tail) {
-                const int64_t gx = static_cast<int64_t>(slice) * a.R + r;
-                a.tail_ml[gx] = make_float2(m, l);
-                dst = a.tail_o + gx * D;
-            } else {
-                a.sel_ml[slot] = make_float2(m, l);
-                dst = a.sel_o + slot * D;
-            }
-#pragma unroll
-            for (int e = 0; e < D; e += 4)
-                *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
         }
         if (tid == 0 && nb > 0) atomicAdd(&a.steps[slice], nb);
+        gstep += nb;
         __syncthreads();
     }
     __syncthreads();

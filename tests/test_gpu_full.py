@@ -67,3 +67,30 @@ def test_decode_full_size_sampled(name):
     print(f"{name} sampled: {rep.exact_required}/{rep.queries} index sets checked bit-exact "
           f"({rep.low_margin} below the margin), mean keys read per head "
           f"{np.mean(rep.read_keys):.0f} ({np.mean(rep.read_keys) / w.N * 100:.2f}% of the cache)")
+
+
+def test_prefill_256k_full_size_sampled():
+    """The 256K chunked prefill (a 4096-query chunk over a tree on the first 262,144 keys,
+    32 query / 8 KV heads, d = 128, bf16) in the benchmark's launch configuration, checked on
+    sampled (sequence, KV head) slices and chunk queries against the oracle."""
+    from tests.test_gpu_prefill import TIGHT_OF_V, Prefill, check_prefill
+
+    w = W.WORKLOADS["prefill256k"]
+    Np, n_q = w.N, w.steps
+    data = W.planted(w, device="cuda", N_cap=Np + n_q, n_queries=n_q)
+    K, V = data["K"], data["V"]
+    K[:, :, Np:] = data["k_new"].permute(1, 2, 0, 3)
+    V[:, :, Np:] = data["v_new"].permute(1, 2, 0, 3)
+    Q = data["Q"].permute(1, 0, 2, 3).contiguous()
+    cfg = zha.Config(d=w.d, Hq=w.Hq, Hkv=w.Hkv, B=w.B, b=w.b, batch=w.batch, N_cap=Np + n_q, p=w.p)
+    pf = Prefill(cfg, K, V, Q, data["qref"], Np, n_q)
+    zha.get_status(clear=True)
+    pf.build()
+    pf.run()
+    rep = check_prefill(pf, [(0, 0), (0, 5)], [0, 1, 63, 64, 2047, n_q - 1], w.p)
+    rep.check()
+    assert rep.exact_required >= rep.queries // 2, rep
+    assert torch.isfinite(pf.O).all()
+    assert_status_clean()
+    print(f"prefill256k sampled: {rep.exact_required}/{rep.queries} index sets checked bit-exact, "
+          f"max error over the GPU's set {rep.max_err_gpu_set:.2e} (bound {TIGHT_OF_V:.2e} of max|v|)")
