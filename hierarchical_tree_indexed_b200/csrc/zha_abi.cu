@@ -72,7 +72,7 @@ int validate(const zha_config* c) {
     if (G != 1 && G != 2 && G != 4) return fail(ZHA_ERR_UNSUPPORTED, "Hq/Hkv=%d: groups of 1, 2 or 4 query heads", G);
     if (c->Hkv > 32) return fail(ZHA_ERR_UNSUPPORTED, "Hkv=%d > 32", c->Hkv);
     if (c->B < 1) return fail(ZHA_ERR_INVALID_ARG, "B=%d", c->B);
-    if (c->B > 64) return fail(ZHA_ERR_UNSUPPORTED, "B=%d > 64", c->B);
+    if (c->B > 256) return fail(ZHA_ERR_UNSUPPORTED, "B=%d > 256", c->B);
     if (c->b < 2 || c->b > 32) return fail(c->b < 2 ? ZHA_ERR_INVALID_ARG : ZHA_ERR_UNSUPPORTED, "b=%d: branching must be 2..32", c->b);
     if (c->R < 1) return fail(ZHA_ERR_INVALID_ARG, "R=%d", c->R);
     if (c->R != 1) return fail(ZHA_ERR_UNSUPPORTED, "R=%d: the GPU path keeps one reference query per node", c->R);
@@ -135,7 +135,7 @@ int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
     w->par_cap = std::max<int64_t>(t.ncap[0], 1);
     w->kb_cap = (w->cand_cap + 31) / 32;
     w->sel_cap = std::max<int64_t>(t.ncap[0], 1);
-    w->item_cap = t.ncap[0] + 2 + (c->N_cap + kAttRows - 1) / kAttRows;
+    w->item_cap = t.ncap[0] * ((c->B + kAttRows - 1) / kAttRows) + 2 + (c->N_cap + kAttRows - 1) / kAttRows;
     w->words = (t.ncap[0] + 31) / 32;
     size_t off = 0;
     w->off_scores = off;   off = align256(off + sizeof(float) * ctas * w->cand_cap);
@@ -499,7 +499,7 @@ int run_pattn_t(const zha_config* c, const PAttnArgs& a, const void* K, const vo
     ZHA_TRY(allow_smem(kern, PAttnLayout<D>::kSmem));
     DevInfo di;
     ZHA_TRY(dev_info(&di));
-    kern<<<2 * di.sms, 128, PAttnLayout<D>::kSmem, st>>>(mk, mv, a);
+    kern<<<2 * di.sms, kPAThreads, PAttnLayout<D>::kSmem, st>>>(mk, mv, a);
     return check_launch("attend_prefill");
 }
 

@@ -223,16 +223,22 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
                     if (!ok) break;
                     StageDesc& d = sm.desc[slot];
                     {   // every lane writes the masks of rows 2*lane, 2*lane+1: the item holding row r
-                        // is the first fitting lane whose inclusive row count exceeds r
-                        const uint32_t fitm = __ballot_sync(0xffffffffu, fit && cc > 0);
+                        // is the first fitting lane whose inclusive row count exceeds r, found by a
+                        // binary search over the fitting lanes (incl is non-decreasing across them)
                         uint32_t pair = 0;
 #pragma unroll
                         for (int k = 0; k < 2; ++k) {
                             const int r = 2 * lane + k;
-                            const uint32_t over = __ballot_sync(0xffffffffu, incl > r) & fitm;
-                            const int owner = over ? __ffs(over) - 1 : 0;
-                            const uint32_t mo = __shfl_sync(0xffffffffu, m, owner);
-                            if (over && r < rows) pair |= (mo & 0xffu) << (8 * k);
+                            int lo = pos, hi = pos + n_fit - 1;   // incl(hi) = rows > r whenever r < rows
+#pragma unroll
+                            for (int step = 0; step < 5; ++step) {
+                                const int mid = (lo + hi) >> 1;
+                                const int im = __shfl_sync(0xffffffffu, incl, mid);
+                                if (im > r) hi = mid;
+                                else lo = mid + 1 < hi ? mid + 1 : hi;
+                            }
+                            const uint32_t mo = __shfl_sync(0xffffffffu, m, lo);
+                            if (r < rows) pair |= (mo & 0xffu) << (8 * k);
                         }
                         reinterpret_cast<uint16_t*>(d.mask)[lane] = static_cast<uint16_t>(pair);
                     }

@@ -76,11 +76,12 @@ __device__ void plan_group(const PlanArgs& a, int g, uint32_t* bits, int* scan) 
     // compaction of the union, ascending: thread owns words [w0, w1)
     const int64_t per = (words + kPlanThreads - 1) / kPlanThreads;
     const int64_t w0 = min(words, tid * per), w1 = min(words, w0 + per);
+    const int nsplit = (a.B + kItemRowsMax - 1) / kItemRowsMax;   // items per block (B > 64)
     int c = 0;
     for (int64_t wd = w0; wd < w1; ++wd) {
         uint32_t o = 0;
         for (int h = 0; h < G; ++h) o |= bits[h * a.words + wd];
-        c += __popc(o);
+        c += __popc(o) * nsplit;
     }
     int total;
     int pos = block_exclusive_scan<kPlanThreads / 32>(c, scan, &total);
@@ -93,12 +94,13 @@ __device__ void plan_group(const PlanArgs& a, int g, uint32_t* bits, int* scan) 
             o &= o - 1;
             uint32_t m = 0;
             for (int h = 0; h < G; ++h) m |= ((bits[h * a.words + wd] >> bit) & 1u) << h;
-            out[pos++] = make_item((wd * 32 + bit) * a.B, a.B, m);
+            for (int st = 0; st < a.B; st += kItemRowsMax)
+                out[pos++] = make_item((wd * 32 + bit) * a.B + st, min(kItemRowsMax, a.B - st), m);
         }
     }
     if (tid == 0) {
         int n = total;
-        int64_t rows = static_cast<int64_t>(total) * a.B;
+        int64_t rows = static_cast<int64_t>(total / nsplit) * a.B;
         if (n1 >= 1) {   // sink: key 0 for the heads whose block 0 is not in the union
             uint32_t m0 = 0;
             for (int h = 0; h < G; ++h) m0 |= (bits[h * a.words] & 1u) << h;

@@ -74,7 +74,7 @@ typedef struct zha_config {
     int32_t d;        /* head dim: 64 or 128                                  */
     int32_t Hq;       /* query heads                                          */
     int32_t Hkv;      /* KV heads; Hq/Hkv in {1, 2, 4}                        */
-    int32_t B;        /* leaf block, 1..64                                    */
+    int32_t B;        /* leaf block, 1..256 (chunked prefill: 64)             */
     int32_t b;        /* branching factor, 2..32                              */
     int32_t R;        /* reference queries per node (GPU path: 1)             */
     int32_t dtype;    /* zha_dtype of K, V, Q, k_new, v_new                   */
