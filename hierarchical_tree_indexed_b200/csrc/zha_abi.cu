@@ -51,7 +51,7 @@ int fail(int code, const char* fmt, ...) {
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct TreeLayout {
-    int Lcap;
+    int Lcap, R;
     int64_t ncap[kMaxLevels];
     size_t off_ntree, off_qref, off_khat[kMaxLevels], off_bhat[kMaxLevels], total;
 };
@@ -75,7 +75,7 @@ int validate(const zha_config* c) {
     if (c->B > 256) return fail(ZHA_ERR_UNSUPPORTED, "B=%d > 256", c->B);
     if (c->b < 2 || c->b > 32) return fail(c->b < 2 ? ZHA_ERR_INVALID_ARG : ZHA_ERR_UNSUPPORTED, "b=%d: branching must be 2..32", c->b);
     if (c->R < 1) return fail(ZHA_ERR_INVALID_ARG, "R=%d", c->R);
-    if (c->R != 1) return fail(ZHA_ERR_UNSUPPORTED, "R=%d: the GPU path keeps one reference query per node", c->R);
+    if (c->R > 16) return fail(ZHA_ERR_UNSUPPORTED, "R=%d: at most 16 reference queries per node", c->R);
     if (c->dtype != ZHA_F32 && c->dtype != ZHA_BF16) return fail(ZHA_ERR_INVALID_ARG, "dtype=%d", c->dtype);
     if (c->batch < 1) return fail(ZHA_ERR_INVALID_ARG, "batch=%d", c->batch);
     if (c->N_cap < 1 || c->N_cap > (int64_t{1} << 31) - 128) return fail(ZHA_ERR_INVALID_ARG, "N_cap=%lld", (long long)c->N_cap);
@@ -95,6 +95,7 @@ int tree_layout(const zha_config* c, TreeLayout* t) {
     ZHA_TRY(validate(c));
     int64_t n[kMaxLevels];
     t->Lcap = tree_levels(c->N_cap, c->B, c->b, c->L_fixed, n);
+    t->R = c->R;
     const int64_t slices = static_cast<int64_t>(c->batch) * c->Hkv;
     size_t off = 0;
     t->off_ntree = off;
@@ -123,6 +124,7 @@ TreeDev tree_view(const TreeLayout& t, void* tree) {
         v.ncap[l] = t.ncap[l];
     }
     v.Lcap = t.Lcap;
+    v.R = t.R;
     return v;
 }
 
@@ -226,10 +228,10 @@ int run_build(const zha_config* c, const TreeLayout& lay, const void* K, const i
     const int64_t slices = static_cast<int64_t>(c->batch) * c->Hkv;
     build_set_count_kernel<<<static_cast<unsigned>(cdiv(c->batch, 128)), 128, 0, st>>>(a.tree, N, c->batch, c->N_cap);
     ZHA_TRY(check_launch("build_set_count"));
-    build_leaf_kernel<T, D><<<static_cast<unsigned>(cdiv(slices * lay.ncap[0] * 32, 256)), 256, 0, st>>>(a);
+    build_leaf_kernel<T, D><<<static_cast<unsigned>(cdiv(slices * lay.ncap[0] * lay.R * 32, 256)), 256, 0, st>>>(a);
     ZHA_TRY(check_launch("build_leaf"));
     for (int l = 2; l <= lay.Lcap; ++l) {
-        build_upper_kernel<D><<<static_cast<unsigned>(cdiv(slices * lay.ncap[l - 1] * 32, 256)), 256, 0, st>>>(a, l);
+        build_upper_kernel<D><<<static_cast<unsigned>(cdiv(slices * lay.ncap[l - 1] * lay.R * 32, 256)), 256, 0, st>>>(a, l);
         ZHA_TRY(check_launch("build_upper"));
     }
     return ZHA_OK;
@@ -255,7 +257,7 @@ bool plan_fits_route(const zha_config* c, const WsLayout& wl);
 
 template <typename T, int D, int NVR>
 int run_route_t(const RouteArgs& a, int ctas, cudaStream_t st) {
-    auto kern = route_decode_kernel<T, D, NVR>;
+    auto kern = a.tree.R > 1 ? route_decode_kernel<T, D, NVR, true> : route_decode_kernel<T, D, NVR, false>;
     ZHA_TRY(allow_smem(kern, sizeof(RouteSmem)));
     kern<<<ctas, kRouteThreads, sizeof(RouteSmem), st>>>(a);
     return check_launch("route");
@@ -433,7 +435,7 @@ int make_kv_map(const zha_config* c, const void* base, CUtensorMap* map) {
 
 template <int D, int NVR>
 int run_proute_t(const PRouteArgs& a, int64_t rows, cudaStream_t st) {
-    auto kern = route_prefill_kernel<uint16_t, D, NVR>;
+    auto kern = a.tree.R > 1 ? route_prefill_kernel<uint16_t, D, NVR, true> : route_prefill_kernel<uint16_t, D, NVR, false>;
     ZHA_TRY(allow_smem(kern, sizeof(PRouteSmem)));
     DevInfo di;
     ZHA_TRY(dev_info(&di));

@@ -12,7 +12,10 @@
 //   F   = LSE_i z_i,  khat = sum_i softmax(z)_i x_i,  bhat = F - scale * qhat . khat.
 // One warp computes one summary with a streaming (online) softmax over 16-byte
 // row loads; build and append call the same routine, so an appended tree is
-// bitwise identical to a rebuilt one.  R = 1 (one reference query per node).
+// bitwise identical to a rebuilt one.  With R reference queries per node (planes
+// r = 0..R-1), every plane of a node is its own tangent; above level 1 a child's
+// estimate is its best plane, max_p (scale q.khat_p + bhat_p) (ties to the lower
+// plane), and its pooled key is that plane's khat.
 #pragma once
 
 #include "zha_common.cuh"
@@ -114,6 +117,56 @@ __device__ void summarize_rows(const T* __restrict__ rows, const float* __restri
     }
 }
 
+// One warp: the summary at reference query q of `cnt` children with R planes each
+// (child c, plane p at kh[(c * R + p) * D], bh[c * R + p]): each child enters with
+// its best plane's estimate and key.
+template <int D>
+__device__ void summarize_children_planes(const float* __restrict__ kh, const float* __restrict__ bh, int cnt,
+                                          int R, const float* __restrict__ q, float scale,
+                                          float* __restrict__ khat_out, float* __restrict__ bhat_out) {
+    constexpr int VF = D / 32;
+    const int lane = threadIdx.x & 31;
+    float qv[VF];
+#pragma unroll
+    for (int e = 0; e < VF; ++e) qv[e] = q[lane * VF + e] * scale;
+    float m = -INFINITY, l = 0.f, acc[VF];
+#pragma unroll
+    for (int e = 0; e < VF; ++e) acc[e] = 0.f;
+    for (int c = 0; c < cnt; ++c) {
+        float best = -INFINITY;
+        int bp = 0;
+        for (int pl = 0; pl < R; ++pl) {
+            float x[VF];
+            load_n<float, VF>(kh + (static_cast<int64_t>(c) * R + pl) * D + lane * VF, x);
+            float dd = 0.f;
+#pragma unroll
+            for (int e = 0; e < VF; ++e) dd = fmaf(qv[e], x[e], dd);
+            const float t = warp_sum(dd) + bh[static_cast<int64_t>(c) * R + pl];
+            if (t > best) { best = t; bp = pl; }
+        }
+        float x[VF];
+        load_n<float, VF>(kh + (static_cast<int64_t>(c) * R + bp) * D + lane * VF, x);
+        const float mn = fmaxf(m, best);
+        const float alpha = expf(m - mn);
+        const float wgt = expf(best - mn);
+        l = l * alpha + wgt;
+#pragma unroll
+        for (int e = 0; e < VF; ++e) acc[e] = fmaf(wgt, x[e], acc[e] * alpha);
+        m = mn;
+    }
+    const float inv = 1.f / l;
+    float pd = 0.f;
+#pragma unroll
+    for (int e = 0; e < VF; ++e) {
+        acc[e] *= inv;
+        pd = fmaf(qv[e], acc[e], pd);
+    }
+    pd = warp_sum(pd);
+#pragma unroll
+    for (int e = 0; e < VF; ++e) khat_out[lane * VF + e] = acc[e];
+    if (lane == 0) *bhat_out = m + logf(l) - pd;
+}
+
 struct BuildArgs {
     TreeDev tree;
     const void* K;      // [batch][Hkv][N_cap][d]
@@ -123,10 +176,13 @@ struct BuildArgs {
     float scale;
 };
 
-// Level 1: one warp per (sequence, KV head, leaf block).
+// Level 1: one warp per (sequence, KV head, leaf block, plane).
 template <typename T, int D>
 __global__ void __launch_bounds__(256) build_leaf_kernel(BuildArgs a) {
-    const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int R = a.tree.R;
+    const int64_t gw0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int pl = static_cast<int>(gw0 % R);
+    const int64_t gw = gw0 / R;
     const int64_t n1cap = a.tree.ncap[0];
     const int64_t slice = gw / n1cap, j = gw % n1cap;
     if (slice >= static_cast<int64_t>(a.batch) * a.Hkv) return;
@@ -138,30 +194,34 @@ __global__ void __launch_bounds__(256) build_leaf_kernel(BuildArgs a) {
     }
     if (j >= N / a.B) return;
     const T* rows = static_cast<const T*>(a.K) + (slice * a.N_cap + j * a.B) * D;
-    const float* q = a.tree.qref + static_cast<int64_t>(h) * a.tree.Lcap * D;
-    float* kh = a.tree.khat[0] + (slice * n1cap + j) * D;
-    float* bh = a.tree.bhat[0] + slice * n1cap + j;
+    const float* q = a.tree.qref + (static_cast<int64_t>(h) * a.tree.Lcap * R + pl) * D;
+    float* kh = a.tree.khat[0] + ((slice * n1cap + j) * R + pl) * D;
+    float* bh = a.tree.bhat[0] + (slice * n1cap + j) * R + pl;
     summarize_rows<T, D>(rows, nullptr, a.B, q, a.scale, kh, bh);
 }
 
 // Level l >= 2: one warp per (sequence, KV head, node) over its children at l-1.
 template <int D>
 __device__ __forceinline__ void summarize_node(const TreeDev& t, int64_t slice, int h, int l, int64_t i,
-                                               int64_t n_child, int b, float scale) {
+                                               int64_t n_child, int b, float scale, int pl = 0) {
+    const int R = t.R;
     const int64_t c0 = i * b;
     const int cnt = static_cast<int>(min(static_cast<int64_t>(b), n_child - c0));
     const int64_t cc = t.ncap[l - 2];
-    const float* rows = t.khat[l - 2] + (slice * cc + c0) * D;
-    const float* bias = t.bhat[l - 2] + slice * cc + c0;
-    const float* q = t.qref + (static_cast<int64_t>(h) * t.Lcap + (l - 1)) * D;
-    float* kh = t.khat[l - 1] + (slice * t.ncap[l - 1] + i) * D;
-    float* bh = t.bhat[l - 1] + slice * t.ncap[l - 1] + i;
-    summarize_rows<float, D>(rows, bias, cnt, q, scale, kh, bh);
+    const float* rows = t.khat[l - 2] + (slice * cc + c0) * R * D;
+    const float* bias = t.bhat[l - 2] + (slice * cc + c0) * R;
+    const float* q = t.qref + ((static_cast<int64_t>(h) * t.Lcap + (l - 1)) * R + pl) * D;
+    float* kh = t.khat[l - 1] + ((slice * t.ncap[l - 1] + i) * R + pl) * D;
+    float* bh = t.bhat[l - 1] + (slice * t.ncap[l - 1] + i) * R + pl;
+    if (R == 1) summarize_rows<float, D>(rows, bias, cnt, q, scale, kh, bh);
+    else summarize_children_planes<D>(rows, bias, cnt, R, q, scale, kh, bh);
 }
 
 template <int D>
 __global__ void __launch_bounds__(256) build_upper_kernel(BuildArgs a, int l) {
-    const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t gw0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int pl = static_cast<int>(gw0 % a.tree.R);
+    const int64_t gw = gw0 / a.tree.R;
     const int64_t ncap = a.tree.ncap[l - 1];
     const int64_t slice = gw / ncap, i = gw % ncap;
     if (slice >= static_cast<int64_t>(a.batch) * a.Hkv) return;
@@ -171,7 +231,7 @@ __global__ void __launch_bounds__(256) build_upper_kernel(BuildArgs a, int l) {
     if (N < 0 || N > a.N_cap) return;
     const int L = tree_levels(N, a.B, a.b, a.L_fixed, n);
     if (L < 0 || l > L || i >= n[l - 1]) return;
-    summarize_node<D>(a.tree, slice, h, l, i, n[l - 2], a.b, a.scale);
+    summarize_node<D>(a.tree, slice, h, l, i, n[l - 2], a.b, a.scale, pl);
 }
 
 __global__ void build_set_count_kernel(TreeDev t, const int32_t* N, int batch, int64_t N_cap) {
@@ -225,10 +285,14 @@ __global__ void append_kernel(AppendArgs a) {
             __syncwarp();
             __threadfence_block();
             const int64_t j = N1 / a.B - 1;
-            const float* q = a.tree.qref + static_cast<int64_t>(h) * a.tree.Lcap * D;
+            const int R = a.tree.R;
             const T* rows = static_cast<const T*>(a.K) + (slice * a.N_cap + j * a.B) * D;
-            summarize_rows<T, D>(rows, nullptr, a.B, q, a.scale, a.tree.khat[0] + (slice * a.tree.ncap[0] + j) * D,
-                                 a.tree.bhat[0] + slice * a.tree.ncap[0] + j);
+            for (int pl = 0; pl < R; ++pl) {
+                const float* q = a.tree.qref + (static_cast<int64_t>(h) * a.tree.Lcap * R + pl) * D;
+                summarize_rows<T, D>(rows, nullptr, a.B, q, a.scale,
+                                     a.tree.khat[0] + ((slice * a.tree.ncap[0] + j) * R + pl) * D,
+                                     a.tree.bhat[0] + (slice * a.tree.ncap[0] + j) * R + pl);
+            }
             int64_t n0[kMaxLevels], n1[kMaxLevels];
             const int L0 = tree_levels(N, a.B, a.b, a.L_fixed, n0);
             const int L1 = tree_levels(N1, a.B, a.b, a.L_fixed, n1);
@@ -239,11 +303,11 @@ __global__ void append_kernel(AppendArgs a) {
                 idx /= a.b;
                 if (l > L0) {
                     for (int64_t i = 0; i < n1[l - 1]; ++i) {
-                        summarize_node<D>(a.tree, slice, h, l, i, n1[l - 2], a.b, a.scale);
+                        for (int pl = 0; pl < R; ++pl) summarize_node<D>(a.tree, slice, h, l, i, n1[l - 2], a.b, a.scale, pl);
                         __syncwarp();
                     }
                 } else {
-                    summarize_node<D>(a.tree, slice, h, l, idx, n1[l - 2], a.b, a.scale);
+                    for (int pl = 0; pl < R; ++pl) summarize_node<D>(a.tree, slice, h, l, idx, n1[l - 2], a.b, a.scale, pl);
                 }
             }
         }

@@ -44,6 +44,7 @@ struct TreeDev {
     float* bhat[kMaxLevels];    // level l-1: [batch][Hkv][ncap][R]
     int64_t ncap[kMaxLevels];
     int Lcap;
+    int R;                      // reference queries (planes) per node
 };
 
 // ---------------------------------------------------------------- elements

@@ -143,7 +143,7 @@ __device__ int warp_top_p(const float* sc, int nc, float p, int32_t* out, NodeOf
 }
 
 // One warp per (sequence, query, query head) row, rows taken in a grid-stride loop.
-template <typename T, int D, int NVR>
+template <typename T, int D, int NVR, bool MP>
 __global__ void __launch_bounds__(kPRThreads, 2) route_prefill_kernel(PRouteArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     PRouteSmem& sm = *reinterpret_cast<PRouteSmem*>(smem_raw);
@@ -191,19 +191,33 @@ __global__ void __launch_bounds__(kPRThreads, 2) route_prefill_kernel(PRouteArgs
             scored += nc - (par[np - 1] == last_parent ? b - (nl - last_parent * b) : 0);
             float* sc = nc <= kPRScores ? sm.sc[w] : spill_sc;
             const int64_t ncap = a.tree.ncap[l - 1];
-            const float* kh = a.tree.khat[l - 1] + slice * ncap * D;
-            const float* bh = a.tree.bhat[l - 1] + slice * ncap;
+            const int R = a.tree.R;
+            const float* kh = a.tree.khat[l - 1] + slice * ncap * R * D;
+            const float* bh = a.tree.bhat[l - 1] + slice * ncap * R;
             for (int pi = 0; pi < np; pi += 2) {
                 const int64_t c0 = static_cast<int64_t>(par[pi]) * b;
                 const int cnt0 = static_cast<int>(min(static_cast<int64_t>(b), nl - c0));
+                if constexpr (!MP) {
+                    if (pi + 1 < np) {
+                        const int64_t c1 = static_cast<int64_t>(par[pi + 1]) * b;
+                        const int cnt1 = static_cast<int>(min(static_cast<int64_t>(b), nl - c1));
+                        scan_children2<D, NVR>(kh + c0 * D, bh + c0, cnt0, kh + c1 * D, bh + c1, cnt1, b, qv,
+                                               sc + static_cast<int64_t>(pi) * b, sc + static_cast<int64_t>(pi + 1) * b);
+                    } else {
+                        scan_children<D, NVR>(kh + c0 * D, bh + c0, cnt0, b, qv, sc + static_cast<int64_t>(pi) * b);
+                    }
+                    continue;
+                }
                 if (pi + 1 < np) {
                     const int64_t c1 = static_cast<int64_t>(par[pi + 1]) * b;
                     const int cnt1 = static_cast<int>(min(static_cast<int64_t>(b), nl - c1));
-                    scan_children2<D, NVR>(kh + c0 * D, bh + c0, cnt0, kh + c1 * D, bh + c1, cnt1, b, qv,
-                                           sc + static_cast<int64_t>(pi) * b, sc + static_cast<int64_t>(pi + 1) * b);
-                } else {
-                    scan_children<D, NVR>(kh + c0 * D, bh + c0, cnt0, b, qv, sc + static_cast<int64_t>(pi) * b);
+                    for (int pl = 0; pl < R; ++pl)
+                        scan_children<D, NVR>(kh + (c1 * R + pl) * D, bh + c1 * R + pl, cnt1, b, qv,
+                                              sc + static_cast<int64_t>(pi + 1) * b, R * D, R, pl == 0);
                 }
+                for (int pl = 0; pl < R; ++pl)
+                    scan_children<D, NVR>(kh + (c0 * R + pl) * D, bh + c0 * R + pl, cnt0, b, qv,
+                                          sc + static_cast<int64_t>(pi) * b, R * D, R, pl == 0);
             }
             __syncwarp();
             const int nxt = nc <= kPRParents ? (cur == 0 ? 1 : 0) : (cur == 2 ? 3 : 2);

@@ -313,9 +313,13 @@ __device__ int top_p_select(const float* sc, int nc, float p, int32_t* out, Rout
 // One warp scores the `cnt` (<= b <= NVR) children of one parent: rows of D fp32
 // starting at kh, biases at bh.  NVR dot products are reduced together: after
 // the halving steps lane holds row (lane >> (5 - log2 NVR)) of the block.
+// With R planes per node, child r's plane p sits at kh[(r * R + p) * D]: the caller
+// passes the plane's first row, rs = R * D and bs = R, and calls once per plane with
+// first = (p == 0); later planes keep the max (the node's score is the max over planes).
 template <int D, int NVR>
 __device__ __forceinline__ void scan_children(const float* __restrict__ kh, const float* __restrict__ bh,
-                                              int cnt, int b, const float* qv, float* __restrict__ out) {
+                                              int cnt, int b, const float* qv, float* __restrict__ out,
+                                              int rs = D, int bs = 1, bool first = true) {
     constexpr int VF = D / 32;
     const int lane = threadIdx.x & 31;
     float v[NVR];
@@ -323,7 +327,7 @@ __device__ __forceinline__ void scan_children(const float* __restrict__ kh, cons
     for (int r = 0; r < NVR; ++r) {
         float x[VF];
         if (r < cnt) {
-            load_n<float, VF>(kh + static_cast<int64_t>(r) * D + lane * VF, x);
+            load_n<float, VF>(kh + static_cast<int64_t>(r) * rs + lane * VF, x);
         } else {
 #pragma unroll
             for (int e = 0; e < VF; ++e) x[e] = 0.f;
@@ -355,7 +359,10 @@ __device__ __forceinline__ void scan_children(const float* __restrict__ kh, cons
     constexpr int low = 5 - H;
     if ((lane & ((1 << low) - 1)) == 0) {
         const int r = (lane >> low) & (NVR - 1);
-        if (r < b) out[r] = r < cnt ? v[0] + bh[r] : -INFINITY;
+        if (r < b) {
+            const float t = r < cnt ? v[0] + bh[static_cast<int64_t>(r) * bs] : -INFINITY;
+            out[r] = first ? t : fmaxf(out[r], t);
+        }
     }
 }
 
@@ -365,17 +372,18 @@ template <int D, int NVR>
 __device__ __forceinline__ void scan_children2(const float* __restrict__ kh0, const float* __restrict__ bh0, int cnt0,
                                                const float* __restrict__ kh1, const float* __restrict__ bh1, int cnt1,
                                                int b, const float* qv, float* __restrict__ out0,
-                                               float* __restrict__ out1) {
+                                               float* __restrict__ out1, int rs = D, int bs = 1,
+                                               bool first = true) {
     constexpr int VF = D / 32;
     const int lane = threadIdx.x & 31;
     float x0[NVR][VF], x1[NVR][VF];
 #pragma unroll
     for (int r = 0; r < NVR; ++r) {
-        if (r < cnt0) load_n<float, VF>(kh0 + static_cast<int64_t>(r) * D + lane * VF, x0[r]);
+        if (r < cnt0) load_n<float, VF>(kh0 + static_cast<int64_t>(r) * rs + lane * VF, x0[r]);
         else
 #pragma unroll
             for (int e = 0; e < VF; ++e) x0[r][e] = 0.f;
-        if (r < cnt1) load_n<float, VF>(kh1 + static_cast<int64_t>(r) * D + lane * VF, x1[r]);
+        if (r < cnt1) load_n<float, VF>(kh1 + static_cast<int64_t>(r) * rs + lane * VF, x1[r]);
         else
 #pragma unroll
             for (int e = 0; e < VF; ++e) x1[r][e] = 0.f;
@@ -417,14 +425,16 @@ __device__ __forceinline__ void scan_children2(const float* __restrict__ kh0, co
     if ((lane & ((1 << low) - 1)) == 0) {
         const int r = (lane >> low) & (NVR - 1);
         if (r < b) {
-            out0[r] = r < cnt0 ? v0[0] + bh0[r] : -INFINITY;
-            out1[r] = r < cnt1 ? v1[0] + bh1[r] : -INFINITY;
+            const float t0 = r < cnt0 ? v0[0] + bh0[static_cast<int64_t>(r) * bs] : -INFINITY;
+            const float t1 = r < cnt1 ? v1[0] + bh1[static_cast<int64_t>(r) * bs] : -INFINITY;
+            out0[r] = first ? t0 : fmaxf(out0[r], t0);
+            out1[r] = first ? t1 : fmaxf(out1[r], t1);
         }
     }
 }
 
 // The top-down walk of one decode query (the body of route_decode_kernel).
-template <typename T, int D, int NVR>
+template <typename T, int D, int NVR, bool MP>
 __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, int cta, int64_t row, int64_t slice,
                                            int64_t N, int64_t Ntree) {
     constexpr int VF = D / 32;   // fp32 summary elements per lane
@@ -462,21 +472,35 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
         float* sc = nc <= kScoresSmem ? sm.scores : ws_sc;
         const int32_t* par = bufs[cur];
         const int64_t ncap = a.tree.ncap[l - 1];
-        const float* kh = a.tree.khat[l - 1] + slice * ncap * D;
-        const float* bh = a.tree.bhat[l - 1] + slice * ncap;
-        // ---- scan: one warp per kept parent, its b child rows of D fp32
+        const int R = a.tree.R;
+        const float* kh = a.tree.khat[l - 1] + slice * ncap * R * D;
+        const float* bh = a.tree.bhat[l - 1] + slice * ncap * R;
+        // ---- scan: one warp per kept parent, its b child rows of D fp32 (per plane, max over planes)
         for (int pi = w; pi < np; pi += 2 * kRouteWarps) {
             const int pj = pi + kRouteWarps;   // a second parent in the same round, if any
             const int64_t c0 = static_cast<int64_t>(par[pi]) * b;
             const int cnt0 = static_cast<int>(min(static_cast<int64_t>(b), nl - c0));
+            if constexpr (!MP) {
+                if (pj < np) {
+                    const int64_t c1 = static_cast<int64_t>(par[pj]) * b;
+                    const int cnt1 = static_cast<int>(min(static_cast<int64_t>(b), nl - c1));
+                    scan_children2<D, NVR>(kh + c0 * D, bh + c0, cnt0, kh + c1 * D, bh + c1, cnt1, b, qv,
+                                           sc + static_cast<int64_t>(pi) * b, sc + static_cast<int64_t>(pj) * b);
+                } else {
+                    scan_children<D, NVR>(kh + c0 * D, bh + c0, cnt0, b, qv, sc + static_cast<int64_t>(pi) * b);
+                }
+                continue;
+            }
             if (pj < np) {
                 const int64_t c1 = static_cast<int64_t>(par[pj]) * b;
                 const int cnt1 = static_cast<int>(min(static_cast<int64_t>(b), nl - c1));
-                scan_children2<D, NVR>(kh + c0 * D, bh + c0, cnt0, kh + c1 * D, bh + c1, cnt1, b, qv,
-                                       sc + static_cast<int64_t>(pi) * b, sc + static_cast<int64_t>(pj) * b);
-            } else {
-                scan_children<D, NVR>(kh + c0 * D, bh + c0, cnt0, b, qv, sc + static_cast<int64_t>(pi) * b);
+                for (int pl = 0; pl < R; ++pl)
+                    scan_children<D, NVR>(kh + (c1 * R + pl) * D, bh + c1 * R + pl, cnt1, b, qv,
+                                          sc + static_cast<int64_t>(pj) * b, R * D, R, pl == 0);
             }
+            for (int pl = 0; pl < R; ++pl)
+                scan_children<D, NVR>(kh + (c0 * R + pl) * D, bh + c0 * R + pl, cnt0, b, qv,
+                                      sc + static_cast<int64_t>(pi) * b, R * D, R, pl == 0);
         }
         __syncthreads();
         // ---- top-p cut and compaction of the kept node ids
@@ -511,7 +535,9 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
 
 // One CTA per (sequence, query head): the whole top-down walk of one decode query.
 // NVR = b rounded up to a power of two (4, 8, 16 or 32).
-template <typename T, int D, int NVR>
+// MP: nodes carry several reference-query planes (R > 1); R = 1 compiles the
+// single-plane scan alone.
+template <typename T, int D, int NVR, bool MP>
 __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     RouteSmem& sm = *reinterpret_cast<RouteSmem*>(smem_raw);
@@ -527,7 +553,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
     if (!valid) {
         if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.sel_count[row] = 0; a.cand[row] = 0; }
     } else {
-        route_walk<T, D, NVR>(a, sm, cta, row, slice, N, Ntree);
+        route_walk<T, D, NVR, MP>(a, sm, cta, row, slice, N, Ntree);
     }
     if (a.fuse_plan) {
         // the last of the group's G query-head CTAs builds the group's gather plan

@@ -55,7 +55,7 @@ def test_sizes_and_levels(lib):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(d=96), 2), (dict(R=2), 2), (dict(Hq=30), 1), (dict(Hq=64), 2), (dict(B=0), 1),
+    (dict(d=96), 2), (dict(R=17), 2), (dict(Hq=30), 1), (dict(Hq=64), 2), (dict(B=0), 1),
     (dict(B=512), 2), (dict(b=1), 1), (dict(b=64), 2), (dict(batch=0), 1), (dict(N_cap=0), 1),
     (dict(p=0.0), 1), (dict(p=float("nan")), 1), (dict(L_fixed=17), 1), (dict(scale=-1.0), 1),
 ])

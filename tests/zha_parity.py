@@ -52,11 +52,11 @@ def compare_tree(cfg: zha.Config, tree: torch.Tensor, ot: O.Tree, s: int, h: int
         n = ot.n[l - 1]
         if n == 0:
             continue
-        g_k = kh[s, h, :n, 0].double().cpu().numpy()
-        g_b = bh[s, h, :n, 0].double().cpu().numpy()
+        g_k = kh[s, h, :n].double().cpu().numpy()        # [n][R][d], every plane
+        g_b = bh[s, h, :n].double().cpu().numpy()
         o_k, o_b = ot.level(l)
-        dk = np.max(np.abs(g_k - o_k[:, 0]))
-        db = np.max(np.abs(g_b - o_b[:, 0]))
+        dk = np.max(np.abs(g_k - o_k))
+        db = np.max(np.abs(g_b - o_b))
         assert dk <= atol and db <= atol, f"level {l}: khat err {dk:.3g}, bhat err {db:.3g}"
 
 
