@@ -39,7 +39,9 @@ namespace zha {
 // ======================================================================== routing
 constexpr int kPRThreads = 256;
 constexpr int kPRWarps = kPRThreads / 32;
-constexpr int kPRScores = 2048;     // per-warp candidate scores in shared memory
+constexpr int kPRScores = 1536;     // per-warp candidate scores in shared memory
+constexpr int kPRBins = 256;        // per-warp mass histogram of the binned cut (1/32 nat bins)
+constexpr int kPRMembers = 64;      // crossing-bin members ranked exactly in shared memory
 constexpr int kPRParents = 512;     // per-warp parent ids, per buffer
 constexpr int kPRSpillWarps = 2 * 160 * kPRWarps;   // warps with a workspace spill area (grid cap)
 
@@ -61,6 +63,9 @@ struct PRouteArgs {
 struct PRouteSmem {
     float sc[kPRWarps][kPRScores];
     int32_t par[kPRWarps][2][kPRParents];
+    unsigned long long hist[kPRWarps][kPRBins];
+    unsigned long long mem_key[kPRWarps][kPRMembers];   // (score key << 32) | ~slot of a member
+    unsigned long long mem_mass[kPRWarps][kPRMembers];
 };
 
 // Top-p cut of one warp over sc[0..nc): the same kept set as top_p_select (the
@@ -142,6 +147,106 @@ __device__ int warp_top_p(const float* sc, int nc, float p, int32_t* out, NodeOf
     return cnt;
 }
 
+// The same cut as warp_top_p, found with a histogram: one pass sums the fixed-point
+// masses into bins of 1/32 nat below the max score (bins are monotone in the score,
+// so bin order is the sorted order up to the order inside a bin); a warp scan finds
+// the bin where the cumulative mass reaches ceil(p * total); only that bin's members
+// are ranked exactly (score, then slot), by comparing each against the others.
+// Falls back to warp_top_p when the crossing bin holds more than kPRMembers.
+template <typename NodeOf>
+__device__ int warp_top_p_binned(const float* sc, int nc, float p, int32_t* out, NodeOf node_of,
+                                 unsigned long long* hist, unsigned long long* mkey,
+                                 unsigned long long* mmass) {
+    const int lane = threadIdx.x & 31;
+    if (p >= 1.0f) return warp_top_p(sc, nc, p, out, node_of);
+    float mx = -INFINITY;
+    for (int i = lane; i < nc; i += 32) mx = fmaxf(mx, sc[i]);
+    mx = warp_max(mx);
+    if (mx == -INFINITY) return 0;
+    auto bin_of = [mx](float s) -> int {
+        const float x = (mx - s) * 32.0f;
+        return x >= static_cast<float>(kPRBins - 1) ? kPRBins - 1 : static_cast<int>(x);
+    };
+#pragma unroll
+    for (int k = 0; k < kPRBins / 32; ++k) hist[lane + 32 * k] = 0ull;
+    __syncwarp();
+    for (int i = lane; i < nc; i += 32) {
+        const float s = sc[i];
+        if (s != -INFINITY) atomicAdd(&hist[bin_of(s)], score_mass(s, mx));
+    }
+    __syncwarp();
+    // lane j owns bins [8j, 8j+8): its sum, then an inclusive scan over lanes
+    unsigned long long own[kPRBins / 32], ls = 0;
+#pragma unroll
+    for (int k = 0; k < kPRBins / 32; ++k) {
+        own[k] = hist[lane * (kPRBins / 32) + k];
+        ls += own[k];
+    }
+    unsigned long long incl = ls;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const unsigned long long tot = __shfl_sync(0xffffffffu, incl, 31);
+    unsigned long long target =
+        static_cast<unsigned long long>(ceil(static_cast<double>(p) * static_cast<double>(tot)));
+    if (target < 1) target = 1;
+    if (target > tot) target = tot;
+    const int J = __ffs(__ballot_sync(0xffffffffu, incl >= target)) - 1;   // lane holding the crossing bin
+    unsigned long long run = __shfl_sync(0xffffffffu, incl - ls, J);        // mass of the bins before lane J's
+    int cbin = 0;
+    unsigned long long above = 0;
+#pragma unroll
+    for (int k = 0; k < kPRBins / 32; ++k) {   // inside lane J's 8 bins (uniform: broadcast each)
+        const unsigned long long bk = __shfl_sync(0xffffffffu, own[k], J);
+        if (run < target && run + bk >= target) { cbin = J * (kPRBins / 32) + k; above = run; }
+        run += bk;
+    }
+    // gather the crossing bin's members
+    int nm = 0;
+    for (int base = 0; base < nc; base += 32) {
+        const int i = base + lane;
+        const float s = i < nc ? sc[i] : -INFINITY;
+        const bool mem = s != -INFINITY && bin_of(s) == cbin;
+        const uint32_t bal = __ballot_sync(0xffffffffu, mem);
+        const int at = nm + __popc(bal & ((1u << lane) - 1u));
+        if (mem && at < kPRMembers) {
+            mkey[at] = (static_cast<unsigned long long>(score_key(s)) << 32) | (0xffffffffu - static_cast<uint32_t>(i));
+            mmass[at] = score_mass(s, mx);
+        }
+        nm += __popc(bal);
+    }
+    if (nm > kPRMembers) return warp_top_p(sc, nc, p, out, node_of);
+    __syncwarp();
+    const unsigned long long need = target - above;
+    // member k is kept iff the mass of the members ordered before it is below `need`;
+    // the order is by the key (score, then lower slot first: ~slot)
+    int cnt = 0;
+    for (int base = 0; base < nc; base += 32) {
+        const int i = base + lane;
+        const float s = i < nc ? sc[i] : -INFINITY;
+        bool keep = false;
+        if (s != -INFINITY) {
+            const int bn = bin_of(s);
+            if (bn < cbin) {
+                keep = true;
+            } else if (bn == cbin) {
+                const unsigned long long myk =
+                    (static_cast<unsigned long long>(score_key(s)) << 32) | (0xffffffffu - static_cast<uint32_t>(i));
+                unsigned long long before = 0;
+                for (int m = 0; m < nm; ++m)
+                    if (mkey[m] > myk) before += mmass[m];
+                keep = before < need;
+            }
+        }
+        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) out[cnt + __popc(bal & ((1u << lane) - 1u))] = node_of(i);
+        cnt += __popc(bal);
+    }
+    return cnt;
+}
+
 // One warp per (sequence, query, query head) row, rows taken in a grid-stride loop.
 template <typename T, int D, int NVR, bool MP>
 __global__ void __launch_bounds__(kPRThreads, 2) route_prefill_kernel(PRouteArgs a) {
@@ -153,12 +258,16 @@ __global__ void __launch_bounds__(kPRThreads, 2) route_prefill_kernel(PRouteArgs
     const int nw = gridDim.x * kPRWarps;
     const int G = a.Hq / a.Hkv;
     const int b = a.b;
-    const int64_t rows = static_cast<int64_t>(a.batch) * a.n_q * a.Hq;
+    // rows < 2^31 (the workspace layout bounds batch * n_q * Hq far below that)
+    const int rows = a.batch * a.n_q * a.Hq;
+    const int per_seq = a.n_q * a.Hq;
     float* spill_sc = a.spill_sc + static_cast<int64_t>(gw) * a.cand_cap;
     int32_t* spill_par = a.spill_par + static_cast<int64_t>(gw) * 2 * a.par_cap;
-    for (int64_t x = gw; x < rows; x += nw) {
-        const int s = static_cast<int>(x / (static_cast<int64_t>(a.n_q) * a.Hq));
-        const int hq = static_cast<int>(x % a.Hq);
+    int cached_s = -1, L = 0;
+    int64_t n[kMaxLevels];
+    for (int x = gw; x < rows; x += nw) {
+        const int s = x / per_seq;
+        const int hq = x % a.Hq;
         const int64_t slice = static_cast<int64_t>(s) * a.Hkv + hq / G;
         const int64_t N = a.N[s];
         const int64_t Ntree = a.tree.n_tree[s];
@@ -171,11 +280,13 @@ __global__ void __launch_bounds__(kPRThreads, 2) route_prefill_kernel(PRouteArgs
             continue;
         }
         float qv[VF];
-        load_n<T, VF>(static_cast<const T*>(a.Q) + x * D + lane * VF, qv);
+        load_n<T, VF>(static_cast<const T*>(a.Q) + static_cast<int64_t>(x) * D + lane * VF, qv);
 #pragma unroll
         for (int e = 0; e < VF; ++e) qv[e] *= a.scale;
-        int64_t n[kMaxLevels];
-        const int L = tree_levels(Ntree, a.B, a.b, a.L_fixed, n);
+        if (s != cached_s) {   // the geometry of this sequence's tree, once per sequence
+            L = tree_levels(Ntree, a.B, a.b, a.L_fixed, n);
+            cached_s = s;
+        }
         int32_t* bufs[4] = {sm.par[w][0], sm.par[w][1], spill_par, spill_par + a.par_cap};
         int cur = 0;
         int np = static_cast<int>((n[L - 1] + b - 1) / b);
@@ -191,7 +302,7 @@ __global__ void __launch_bounds__(kPRThreads, 2) route_prefill_kernel(PRouteArgs
             scored += nc - (par[np - 1] == last_parent ? b - (nl - last_parent * b) : 0);
             float* sc = nc <= kPRScores ? sm.sc[w] : spill_sc;
             const int64_t ncap = a.tree.ncap[l - 1];
-            const int R = a.tree.R;
+            const int R = MP ? a.tree.R : 1;
             const float* kh = a.tree.khat[l - 1] + slice * ncap * R * D;
             const float* bh = a.tree.bhat[l - 1] + slice * ncap * R;
             for (int pi = 0; pi < np; pi += 2) {
@@ -223,11 +334,12 @@ __global__ void __launch_bounds__(kPRThreads, 2) route_prefill_kernel(PRouteArgs
             const int nxt = nc <= kPRParents ? (cur == 0 ? 1 : 0) : (cur == 2 ? 3 : 2);
             auto node_of = [par, b](int i) { return static_cast<int32_t>(par[i / b] * b + i % b); };
             np = nc <= 64 ? top_p_small(sc, nc, a.p[l - 1], bufs[nxt], node_of)
-                          : warp_top_p(sc, nc, a.p[l - 1], bufs[nxt], node_of);
+                          : warp_top_p_binned(sc, nc, a.p[l - 1], bufs[nxt], node_of, sm.hist[w], sm.mem_key[w],
+                                              sm.mem_mass[w]);
             __syncwarp();
             cur = nxt;
         }
-        int32_t* out = a.sel + x * a.sel_cap;
+        int32_t* out = a.sel + static_cast<int64_t>(x) * a.sel_cap;
         const int ncopy = min(np, a.sel_cap);
         for (int i = lane; i < ncopy; i += 32) out[i] = bufs[cur][i];
         if (lane == 0) {

@@ -472,7 +472,7 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
         float* sc = nc <= kScoresSmem ? sm.scores : ws_sc;
         const int32_t* par = bufs[cur];
         const int64_t ncap = a.tree.ncap[l - 1];
-        const int R = a.tree.R;
+        const int R = MP ? a.tree.R : 1;
         const float* kh = a.tree.khat[l - 1] + slice * ncap * R * D;
         const float* bh = a.tree.bhat[l - 1] + slice * ncap * R;
         // ---- scan: one warp per kept parent, its b child rows of D fp32 (per plane, max over planes)
