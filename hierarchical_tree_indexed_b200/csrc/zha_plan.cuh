@@ -94,13 +94,17 @@ __device__ void plan_group(const PlanArgs& a, int g, uint32_t* bits, int* scan) 
             o &= o - 1;
             uint32_t m = 0;
             for (int h = 0; h < G; ++h) m |= ((bits[h * a.words + wd] >> bit) & 1u) << h;
-            for (int st = 0; st < a.B; st += kItemRowsMax)
-                out[pos++] = make_item((wd * 32 + bit) * a.B + st, min(kItemRowsMax, a.B - st), m);
+            if (nsplit == 1) {
+                out[pos++] = make_item((wd * 32 + bit) * a.B, a.B, m);
+            } else {
+                for (int st = 0; st < a.B; st += kItemRowsMax)
+                    out[pos++] = make_item((wd * 32 + bit) * a.B + st, min(kItemRowsMax, a.B - st), m);
+            }
         }
     }
     if (tid == 0) {
         int n = total;
-        int64_t rows = static_cast<int64_t>(total / nsplit) * a.B;
+        int64_t rows = static_cast<int64_t>(nsplit == 1 ? total : total / nsplit) * a.B;
         if (n1 >= 1) {   // sink: key 0 for the heads whose block 0 is not in the union
             uint32_t m0 = 0;
             for (int h = 0; h < G; ++h) m0 |= (bits[h * a.words] & 1u) << h;
