@@ -486,6 +486,61 @@ def prefill_main(args, rank, w):
     torch.cuda.synchronize()
     t_dense = sum(a_.elapsed_time(b_) for a_, b_ in dense_ev[1:]) / 4 / 1e3
     dense_flops = sum(Np + i + 1 for i in range(n_q)) * w.batch * w.Hq * w.d * 4
+    # the pages' U_p(W), with S_p(q) read as the routed set: the union of the blocks the last W
+    # chunk queries selected, as a fraction of the prefix's blocks (mean over (sequence, query head))
+    n1 = Np // w.B
+    coverage = {}
+    for W_ in (1, 16, 256, n_q):
+        fr = []
+        for s_ in range(w.batch):
+            for hq in range(w.Hq):
+                c = cnt[s_, n_q - W_:, hq].to(torch.int64)
+                ids = sel[s_, n_q - W_:, hq]
+                mask = torch.arange(ids.shape[1], device=dev)[None, :] < c[:, None]
+                u = torch.zeros(n1, dtype=torch.bool, device=dev)
+                u[ids[mask].long()] = True
+                fr.append(u.sum().item() / n1)
+        coverage[str(W_)] = sum(fr) / len(fr)
+    # causal chunk insertion: the chunk in block-aligned sub-chunks; before each, zha_extend indexes
+    # the chunk's blocks completed so far, so query t routes over exactly the blocks before its own
+    causal = None
+    if w.batch == 1 and Np % w.B == 0:
+        subs = [(i0, min(i0 + w.B, n_q)) for i0 in range(0, n_q, w.B)]
+        ws_sub = zha.alloc_workspace(cfg, w.B, device=dev)
+        Oc = torch.zeros_like(O)
+        N_tree = [torch.full((1,), Np + i0, dtype=torch.int32, device=dev) for i0, _ in subs]
+        N_end = [torch.full((1,), Np + i1, dtype=torch.int32, device=dev) for _, i1 in subs]
+
+        def causal_chunk():
+            zha.build(cfg, K, qref, N_tree[0], tree)
+            for k, (i0, i1) in enumerate(subs):
+                if k:
+                    zha.extend(cfg, K, N_tree[k], tree)
+                zha.route(cfg, tree, Q[:, i0:i1], N_end[k], sel[:, i0:i1], cnt[:, i0:i1], ws_sub, n_q=i1 - i0)
+                zha.attend(cfg, K, V, tree, Q[:, i0:i1], N_end[k], sel[:, i0:i1], cnt[:, i0:i1], Oc[:, i0:i1],
+                           ws_sub, n_q=i1 - i0)
+        causal_chunk()
+        torch.cuda.synchronize()
+        gc_ = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gc_, stream=s):
+            causal_chunk()
+        torch.cuda.synchronize()
+        cev = []
+        for _ in range(4):
+            flush.zero_()
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream); gc_.replay(); b_.record(stream)
+            cev.append((a_, b_))
+        torch.cuda.synchronize()
+        bits = zha.get_status(clear=True)
+        if bits:
+            raise RuntimeError(f"device status after the causal chunk: {zha.status_names(bits)}")
+        t_c = sum(a_.elapsed_time(b_) for a_, b_ in cev[1:]) / 3 / 1e3
+        causal = {"ms_per_chunk": t_c * 1e3, "queries_per_s": n_q / t_c, "sub_chunks": len(subs),
+                  "note": "tree rebuilt on the prefix then extended block by block (zha_extend), each sub-chunk "
+                          "routed and attended over the tree of the keys before it; timed including the rebuild"}
+        del gc_
+        zha.build(cfg, K, qref, torch.full((w.batch,), Np, dtype=torch.int32, device=dev), tree)
     # end to end: host Q and chunk K/V in, O out, through the public calls
     e2e = None
     if not args.no_e2e:
@@ -536,6 +591,8 @@ def prefill_main(args, rank, w):
                          "issued_tflops": issued_tflops},
             "phases_ms": {"route": t_route / K_steps * 1e3, "attend": t_att / K_steps * 1e3},
             "keys_per_row": keys / (w.batch * n_q * w.Hq),
+            "coverage_U_W": coverage,
+            "causal_chunk": causal,
             "dense_baseline": {"ms_per_step": t_dense * 1e3, "tflops": dense_flops / t_dense / 1e12,
                                "queries_per_s": w.batch * n_q / t_dense,
                                "speedup_of_tree": t_dense / (t_max / K_steps)},

@@ -59,7 +59,7 @@ struct TreeLayout {
 struct WsLayout {
     int64_t cand_cap, par_cap, kb_cap, sel_cap, item_cap, words;
     size_t off_scores, off_parents, off_sel, off_count, off_items, off_nitems, off_ml, off_acc, off_counters;
-    size_t off_rows, off_cand, off_sched, off_ballot, off_grp;
+    size_t off_rows, off_cand, off_ballot, off_grp;
     size_t total;
 };
 
@@ -128,6 +128,14 @@ TreeDev tree_view(const TreeLayout& t, void* tree) {
     return v;
 }
 
+// The decode kernels clear their own per-group counters when they finish, so these
+// must hold zero between calls.  They sit at the front of every workspace layout,
+// decode and prefill alike, and no prefill call writes there: a workspace moves
+// between decode and chunks of any length without being zeroed again.
+size_t ws_counter_bytes(const zha_config* c) {
+    return 2 * align256(sizeof(uint32_t) * static_cast<size_t>(c->batch) * c->Hkv);
+}
+
 int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
     if (n_q != 1) return fail(ZHA_ERR_UNSUPPORTED, "n_q=%d: decode takes one query per sequence", n_q);
     const int64_t groups = static_cast<int64_t>(c->batch) * c->Hkv;
@@ -140,6 +148,8 @@ int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
     w->item_cap = t.ncap[0] * ((c->B + kAttRows - 1) / kAttRows) + 2 + (c->N_cap + kAttRows - 1) / kAttRows;
     w->words = (t.ncap[0] + 31) / 32;
     size_t off = 0;
+    w->off_counters = off; off = align256(off + sizeof(uint32_t) * groups);
+    w->off_grp = off;      off = align256(off + sizeof(uint32_t) * groups);
     w->off_scores = off;   off = align256(off + sizeof(float) * ctas * w->cand_cap);
     w->off_parents = off;  off = align256(off + sizeof(int32_t) * ctas * 2 * w->par_cap);
     w->off_sel = off;      off = align256(off + sizeof(int32_t) * ctas * w->sel_cap);
@@ -148,12 +158,9 @@ int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
     w->off_nitems = off;   off = align256(off + sizeof(int32_t) * groups);
     w->off_ml = off;       off = align256(off + sizeof(float2) * groups * kSplitMax * G);
     w->off_acc = off;      off = align256(off + sizeof(float) * groups * kSplitMax * G * c->d);
-    w->off_counters = off; off = align256(off + sizeof(uint32_t) * groups);
     w->off_rows = off;     off = align256(off + sizeof(int32_t) * groups);
     w->off_cand = off;     off = align256(off + sizeof(int32_t) * ctas);
-    w->off_sched = off;    off = align256(off + sizeof(uint32_t) * 2);
     w->off_ballot = off;   off = align256(off + sizeof(uint32_t) * ctas * 2 * w->kb_cap);
-    w->off_grp = off;      off = align256(off + sizeof(uint32_t) * groups);
     w->total = off;
     if (static_cast<size_t>(G) * w->words * 4 > 200 * 1024)
         return fail(ZHA_ERR_UNSUPPORTED, "N_cap too large for the on-chip union bitmap");
@@ -235,6 +242,29 @@ int run_build(const zha_config* c, const TreeLayout& lay, const void* K, const i
         ZHA_TRY(check_launch("build_upper"));
     }
     return ZHA_OK;
+}
+
+// Extension: leaves and ancestors that change, then the new count (the kernels read the old one).
+template <typename T, int D>
+int run_extend(const zha_config* c, const TreeLayout& lay, const void* K, const int32_t* N, void* tree,
+               cudaStream_t st) {
+    BuildArgs a{};
+    a.tree = tree_view(lay, tree);
+    a.K = K;
+    a.N = N;
+    a.batch = c->batch; a.Hkv = c->Hkv; a.B = c->B; a.b = c->b; a.L_fixed = c->L_fixed;
+    a.incremental = 1;
+    a.N_cap = c->N_cap;
+    a.scale = scale_of(c);
+    const int64_t slices = static_cast<int64_t>(c->batch) * c->Hkv;
+    build_leaf_kernel<T, D><<<static_cast<unsigned>(cdiv(slices * lay.ncap[0] * lay.R * 32, 256)), 256, 0, st>>>(a);
+    ZHA_TRY(check_launch("extend_leaf"));
+    for (int l = 2; l <= lay.Lcap; ++l) {
+        build_upper_kernel<D><<<static_cast<unsigned>(cdiv(slices * lay.ncap[l - 1] * lay.R * 32, 256)), 256, 0, st>>>(a, l);
+        ZHA_TRY(check_launch("extend_upper"));
+    }
+    extend_set_count_kernel<<<static_cast<unsigned>(cdiv(c->batch, 128)), 128, 0, st>>>(a.tree, N, c->batch, c->N_cap);
+    return check_launch("extend_set_count");
 }
 
 template <typename T, int D>
@@ -382,11 +412,12 @@ int pf_layout(const zha_config* c, int n_q, const TreeLayout& t, PfLayout* p) {
     p->pair_cap = p->rows * kPairsPerRow;
     p->item_cap = p->slices * ((p->R * kPairsPerRow + kTileRows - 1) / kTileRows + p->nJ_cap);
     const size_t D = static_cast<size_t>(c->d);
-    size_t off = 0;
+    size_t off = ws_counter_bytes(c);
     p->off_spill_sc = off;  off = align256(off + sizeof(float) * kPRSpillWarps * p->cand_cap);
     p->off_spill_par = off; off = align256(off + sizeof(int32_t) * kPRSpillWarps * 2 * p->par_cap);
     p->off_cand = off;      off = align256(off + sizeof(int32_t) * p->rows);
     p->off_totals = off;    off = align256(off + sizeof(unsigned long long) * p->slices * kSBOpts);
+    p->off_steps = off;     off = align256(off + sizeof(int32_t) * p->slices);
     p->off_hdr = off;       off = align256(off + sizeof(int32_t) * 8);
     p->off_ctr = off;       off = align256(off + sizeof(int32_t) * 2);
     p->off_row_cnt = off;   off = align256(off + sizeof(int32_t) * p->rows);
@@ -400,7 +431,6 @@ int pf_layout(const zha_config* c, int n_q, const TreeLayout& t, PfLayout* p) {
     p->off_tail_o = off;    off = align256(off + sizeof(float) * p->rows * D);
     p->off_sel_ml = off;    off = align256(off + sizeof(float2) * p->pair_cap);
     p->off_sel_o = off;     off = align256(off + sizeof(float) * p->pair_cap * D);
-    p->off_steps = off;     off = align256(off + sizeof(int32_t) * p->slices);
     p->total = off;
     return ZHA_OK;
 }
@@ -505,6 +535,15 @@ int run_pattn_t(const zha_config* c, const PAttnArgs& a, const void* K, const vo
     return check_launch("attend_prefill");
 }
 
+// The pair totals, step counters, plan header and item counters sit side by side and
+// start every chunk at zero, whatever an earlier call with another n_q (hence another
+// layout of the same workspace) left in these bytes.
+int pf_reset(const PfLayout& pl, void* ws, cudaStream_t st) {
+    ZHA_CUDA(cudaMemsetAsync(static_cast<char*>(ws) + pl.off_totals, 0,
+                             pl.off_ctr + sizeof(int32_t) * 2 - pl.off_totals, st));
+    return ZHA_OK;
+}
+
 int run_pattn(const zha_config* c, const PAttnArgs& a, const void* K, const void* V, cudaStream_t st) {
     return c->d == 128 ? run_pattn_t<128>(c, a, K, V, st) : run_pattn_t<64>(c, a, K, V, st);
 }
@@ -529,7 +568,7 @@ int run_prefill_attend(const zha_config* c, const TreeLayout& lay, const PfLayou
     p.sel_cap = sel_cap; p.n_q = n_q; p.Hq = c->Hq; p.Hkv = c->Hkv; p.G = c->Hq / c->Hkv; p.B = c->B;
     p.R = static_cast<int>(pl.R); p.slices = static_cast<int>(pl.slices);
     const int chunks = static_cast<int>(pl.slices) * kPlanChunks;
-    ZHA_CUDA(cudaMemsetAsync(at<int32_t>(ws, pl.off_steps), 0, sizeof(int32_t) * pl.slices, st));
+    ZHA_TRY(pf_reset(pl, ws, st));
     prefill_count_kernel<<<chunks, 256, 0, st>>>(p);
     prefill_choose_kernel<<<1, 1024, 0, st>>>(p);
     prefill_pairs_kernel<<<chunks, 256, 0, st>>>(p);
@@ -683,10 +722,10 @@ int zha_workspace_stats(const zha_config* cfg, int32_t n_q, size_t* rows_offset,
 
 int zha_workspace_init(const zha_config* cfg, void* ws, size_t ws_bytes, zha_stream_t stream) {
     TreeLayout t;
-    WsLayout w;
     ZHA_TRY(tree_layout(cfg, &t));
-    ZHA_TRY(ws_layout(cfg, 1, t, &w));
-    ZHA_TRY(check_ws(w, ws, ws_bytes));
+    ZHA_TRY(need(ws, "ws"));
+    if (ws_bytes < ws_counter_bytes(cfg))
+        return fail(ZHA_ERR_WORKSPACE, "workspace of %zu B < %zu B", ws_bytes, ws_counter_bytes(cfg));
     ZHA_CUDA(cudaMemsetAsync(ws, 0, ws_bytes, stream));
     return ZHA_OK;
 }
@@ -702,6 +741,15 @@ int zha_build(const zha_config* cfg, const void* K, const float* Qref, const int
     const size_t qbytes = sizeof(float) * static_cast<size_t>(cfg->Hkv) * t.Lcap * cfg->R * cfg->d;
     ZHA_CUDA(cudaMemcpyAsync(static_cast<char*>(tree) + t.off_qref, Qref, qbytes, cudaMemcpyDeviceToDevice, stream));
     return ZHA_DISPATCH(cfg, run_build, cfg, t, K, N, tree, stream);
+}
+
+int zha_extend(const zha_config* cfg, const void* K, const int32_t* N, void* tree, zha_stream_t stream) {
+    TreeLayout t;
+    ZHA_TRY(tree_layout(cfg, &t));
+    ZHA_TRY(need(K, "K"));
+    ZHA_TRY(need(N, "N"));
+    ZHA_TRY(need(tree, "tree"));
+    return ZHA_DISPATCH(cfg, run_extend, cfg, t, K, N, tree, stream);
 }
 
 int zha_append(const zha_config* cfg, void* K, void* V, const void* k_new, const void* v_new, int32_t* N,
@@ -843,7 +891,7 @@ int zha_dense(const zha_config* cfg, const void* K, const void* V, const void* Q
         ZHA_TRY(need(Q, "Q"));
         ZHA_TRY(need(N, "N"));
         ZHA_TRY(need(O, "O"));
-        ZHA_CUDA(cudaMemsetAsync(at<int32_t>(ws, p.off_steps), 0, sizeof(int32_t) * p.slices, stream));
+        ZHA_TRY(pf_reset(p, const_cast<void*>(ws), stream));
         const PAttnArgs a = pattn_args(cfg, p, t, nullptr, Q, n_q, N, nullptr, nullptr, 0, O, ws, 1);
         return run_pattn(cfg, a, K, V, stream);
     }

@@ -172,9 +172,22 @@ struct BuildArgs {
     const void* K;      // [batch][Hkv][N_cap][d]
     const int32_t* N;   // [batch]
     int batch, Hkv, B, b, L_fixed;
+    int incremental;    // 1: the tree already indexes tree.n_tree[s] keys; summarise only what changes
     int64_t N_cap;
     float scale;
 };
+
+// Extending a tree from n_old to N keys changes the leaf blocks from floor(n_old/B)
+// on, and at level l only their ancestors (node index = leaf index / b^(l-1)) and
+// any level the old tree did not have.  Returns the first node of level l to redo.
+__device__ __forceinline__ int64_t first_changed(int64_t n_old, int l, int B, int b, int L_fixed) {
+    int64_t no[kMaxLevels];
+    const int L_old = tree_levels(n_old, B, b, L_fixed, no);
+    if (l > L_old) return 0;
+    int64_t first = n_old / B;
+    for (int k = 1; k < l; ++k) first /= b;
+    return first;
+}
 
 // Level 1: one warp per (sequence, KV head, leaf block, plane).
 template <typename T, int D>
@@ -193,6 +206,10 @@ __global__ void __launch_bounds__(256) build_leaf_kernel(BuildArgs a) {
         return;
     }
     if (j >= N / a.B) return;
+    if (a.incremental) {
+        const int64_t n_old = a.tree.n_tree[s];
+        if (N < n_old || j < n_old / a.B) return;   // shrinking is refused by the count kernel
+    }
     const T* rows = static_cast<const T*>(a.K) + (slice * a.N_cap + j * a.B) * D;
     const float* q = a.tree.qref + (static_cast<int64_t>(h) * a.tree.Lcap * R + pl) * D;
     float* kh = a.tree.khat[0] + ((slice * n1cap + j) * R + pl) * D;
@@ -231,12 +248,24 @@ __global__ void __launch_bounds__(256) build_upper_kernel(BuildArgs a, int l) {
     if (N < 0 || N > a.N_cap) return;
     const int L = tree_levels(N, a.B, a.b, a.L_fixed, n);
     if (L < 0 || l > L || i >= n[l - 1]) return;
+    if (a.incremental) {
+        const int64_t n_old = a.tree.n_tree[s];
+        if (N < n_old || i < first_changed(n_old, l, a.B, a.b, a.L_fixed)) return;
+    }
     summarize_node<D>(a.tree, slice, h, l, i, n[l - 2], a.b, a.scale, pl);
 }
 
 __global__ void build_set_count_kernel(TreeDev t, const int32_t* N, int batch, int64_t N_cap) {
     const int s = blockIdx.x * blockDim.x + threadIdx.x;
     if (s < batch) t.n_tree[s] = (N[s] >= 0 && N[s] <= N_cap) ? N[s] : 0;
+}
+
+// After an extension: the tree now indexes N[s] keys (a shorter N is refused).
+__global__ void extend_set_count_kernel(TreeDev t, const int32_t* N, int batch, int64_t N_cap) {
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= batch) return;
+    if (N[s] < t.n_tree[s] || N[s] > N_cap) raise_status(ZHA_ERR_INVALID_ARG);
+    else t.n_tree[s] = N[s];
 }
 
 struct AppendArgs {

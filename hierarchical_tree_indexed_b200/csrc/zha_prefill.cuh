@@ -434,7 +434,8 @@ __global__ void __launch_bounds__(256) prefill_count_kernel(PPlanArgs a) {
     if (threadIdx.x < kSBOpts && acc[threadIdx.x]) atomicAdd(&a.totals[slice * kSBOpts + threadIdx.x], acc[threadIdx.x]);
 }
 
-// Picks SB, clears the per-superblock counters and the pair totals.
+// Picks SB and clears the per-superblock counters.  The pair totals it reads are
+// zeroed on the stream before the count kernel of every plan.
 __global__ void __launch_bounds__(1024) prefill_choose_kernel(PPlanArgs a) {
     __shared__ int s_log2;
     if (threadIdx.x == 0) {
@@ -455,7 +456,6 @@ __global__ void __launch_bounds__(1024) prefill_choose_kernel(PPlanArgs a) {
     for (int64_t i = threadIdx.x; i < static_cast<int64_t>(a.slices) * a.nJ_cap; i += blockDim.x) {
         if (i % a.nJ_cap < nJ) a.jcount[i] = 0;
     }
-    for (int i = threadIdx.x; i < a.slices * kSBOpts; i += blockDim.x) a.totals[i] = 0;
 }
 
 // Pairs per row at the chosen SB, and rows per superblock.

@@ -39,7 +39,7 @@ class ZhaConfig(ctypes.Structure):
 
 
 EXPORTS = ["zha_levels_cap", "zha_tree_bytes", "zha_tree_level", "zha_tree_count_offset", "zha_workspace_bytes", "zha_workspace_init", "zha_workspace_stats", "zha_build",
-           "zha_append", "zha_route", "zha_attend", "zha_attend_noalloc", "zha_decode", "zha_dense", "zha_get_status",
+           "zha_extend", "zha_append", "zha_route", "zha_attend", "zha_attend_noalloc", "zha_decode", "zha_dense", "zha_get_status",
            "zha_last_error"]
 
 
@@ -63,6 +63,7 @@ def lib():
         "zha_workspace_init": [C, P, SZ, P],
         "zha_workspace_stats": [C, I32, P, P],
         "zha_build": [C, P, P, P, P, P],
+        "zha_extend": [C, P, P, P, P],
         "zha_append": [C, P, P, P, P, P, P, P],
         "zha_route": [C, P, P, I32, P, P, P, I32, P, SZ, P],
         "zha_attend": [C, P, P, P, P, I32, P, P, P, I32, P, P, SZ, P],
@@ -200,6 +201,11 @@ def build(cfg: Config, K, qref, N, tree, stream=None):
     q = qref[:, :Lc].contiguous()
     _check(lib().zha_build(ctypes.byref(cfg.c()), _ptr(K), _ptr(q), _ptr(N), _ptr(tree), _stream(stream)))
     return q   # keep alive until the copy has run
+
+
+def extend(cfg: Config, K, N, tree, stream=None):
+    """Grows the tree to index keys [0, N[s]) already written into K (see include/zha.h)."""
+    _check(lib().zha_extend(ctypes.byref(cfg.c()), _ptr(K), _ptr(N), _ptr(tree), _stream(stream)))
 
 
 def append(cfg: Config, K, V, k_new, v_new, N, tree, stream=None):

@@ -105,7 +105,8 @@ int zha_tree_count_offset(const zha_config *cfg, size_t *offset);
  * for n_q queries per sequence (decode: n_q = 1; a chunked prefill: n_q > 1,
  * which takes bf16 K/V/Q, leaf blocks of B = 64 and at most 262144 leaf blocks,
  * else ZHA_ERR_UNSUPPORTED).  The workspace must be zeroed once after allocation
- * (zha_workspace_init); calls leave it reusable. */
+ * (zha_workspace_init); calls leave it reusable by any later call whose own
+ * size it covers, decode and chunks of any length alike, in any order. */
 int zha_workspace_bytes(const zha_config *cfg, int32_t n_q, size_t *bytes);
 int zha_workspace_init(const zha_config *cfg, void *ws, size_t ws_bytes, zha_stream_t stream);
 
@@ -129,6 +130,17 @@ int zha_workspace_stats(const zha_config *cfg, int32_t n_q, size_t *rows_offset,
  */
 int zha_build(const zha_config *cfg, const void *K, const float *Qref, const int32_t *N,
               void *tree, zha_stream_t stream);
+
+/*
+ * zha_extend -- grow the tree to index keys [0, N[s]) of every sequence s whose
+ * rows the caller has already written into K (for instance a prefill chunk):
+ * the new complete leaf blocks are summarised, then their ancestors and any new
+ * level ([EoQ] "the tree is built on the fly as the context grows").  The
+ * result is bitwise equal to zha_build at N.  N[s] below the tree's current
+ * count, or above N_cap, sets ZHA_ERR_INVALID_ARG on the device and leaves
+ * that sequence's count unchanged.
+ */
+int zha_extend(const zha_config *cfg, const void *K, const int32_t *N, void *tree, zha_stream_t stream);
 
 /*
  * zha_append -- decode-time growth ([EoQ] "the tree is built on the fly as the

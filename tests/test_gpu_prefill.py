@@ -202,3 +202,86 @@ def test_prefill_is_deterministic():
     torch.cuda.synchronize()
     assert torch.equal(first[1], pf.cnt) and torch.equal(first[0], pf.sel)
     assert torch.equal(first[2], pf.O)
+
+
+def test_causal_chunk_insertion_matches_decode_semantics():
+    """The chunk's own blocks inserted causally: the chunk runs in block-aligned sub-chunks and
+    zha_extend indexes the blocks completed before each, so query t routes over the tree of the
+    keys [0, floor(t/B) B) and attends to its own block up to t -- what decoding it token by token
+    would do."""
+    Np, n_q, B = 12800, 150, 64            # the prefix ends on a block boundary
+    w, cfg, K, V, Q, qref = make_case(batch=1, Hkv=2, G=4, d=128, Np=Np, n_q=n_q, p=0.95, M=8)
+    pf = Prefill(cfg, K, V, Q, qref, Np, n_q)
+    ws_sub = zha.alloc_workspace(cfg, B)
+    zha.get_status(clear=True)
+    pf.build()
+    for i0 in range(0, n_q, B):
+        i1 = min(i0 + B, n_q)
+        if i0:
+            zha.extend(cfg, pf.K, torch.full((1,), Np + i0, dtype=torch.int32, device="cuda"), pf.tree)
+        N_end = torch.full((1,), Np + i1, dtype=torch.int32, device="cuda")
+        zha.route(cfg, pf.tree, Q[:, i0:i1], N_end, pf.sel[:, i0:i1], pf.cnt[:, i0:i1], ws_sub, n_q=i1 - i0)
+        zha.attend(cfg, pf.K, pf.V, pf.tree, Q[:, i0:i1], N_end, pf.sel[:, i0:i1], pf.cnt[:, i0:i1],
+                   pf.O[:, i0:i1], ws_sub, n_q=i1 - i0)
+    torch.cuda.synchronize()
+    sel, cnt, out = pf.sel.cpu(), pf.cnt.cpu(), pf.O.cpu()
+    rep = Report()
+    for h in range(cfg.Hkv):
+        Kh, Vh = pf.K[0, h].cpu(), pf.V[0, h].cpu()
+        for i in (0, 63, 64, 100, n_q - 1):
+            t = Np + i
+            ot = oracle_tree(Kh, (t // B) * B, cfg, pf.qref[h].cpu())
+            hs = slice(h * cfg.G, (h + 1) * cfg.G)
+            check_queries(cfg, ot, Kh, Vh, [t] * cfg.G, pf.Q[0, i, hs].cpu().float(), sel[0, i, hs], cnt[0, i, hs],
+                          out[0, i, hs].numpy(), 0.95, rep, tight_of_v=TIGHT_OF_V)
+    rep.check()
+    assert rep.exact_required >= rep.queries // 2, rep
+    assert_status_clean()
+
+
+def test_workspace_reused_across_chunk_lengths():
+    """One workspace serves chunks of different lengths and then decoding: its layout depends
+    on n_q, so what a longer chunk left in it must reach neither a shorter chunk nor a decode
+    step (both bit-identical to a fresh workspace)."""
+    Np, n_q, short = 9000 + 5, 200, 37
+    w, cfg, K, V, Q, qref = make_case(batch=2, Hkv=2, G=2, d=128, Np=Np, n_q=n_q, p=0.95, M=8)
+    pf = Prefill(cfg, K, V, Q, qref, Np, n_q)
+    zha.get_status(clear=True)
+    pf.build()
+    pf.run()
+    Qs = Q[:, :short].contiguous()
+    N_s = torch.full((cfg.batch,), Np + short, dtype=torch.int32, device="cuda")
+
+    def run(ws):
+        sel = torch.zeros((cfg.batch, short, cfg.Hq, pf.sel_cap), dtype=torch.int32, device="cuda")
+        cnt = torch.zeros((cfg.batch, short, cfg.Hq), dtype=torch.int32, device="cuda")
+        out = torch.zeros((cfg.batch, short, cfg.Hq, cfg.d), dtype=torch.float32, device="cuda")
+        zha.route(cfg, pf.tree, Qs, N_s, sel, cnt, ws, n_q=short)
+        zha.attend(cfg, pf.K, pf.V, pf.tree, Qs, N_s, sel, cnt, out, ws, n_q=short)
+        return sel, cnt, out
+
+    reused = run(pf.ws)
+    fresh = run(zha.alloc_workspace(cfg, short))
+    torch.cuda.synchronize()
+    for a, b in zip(reused, fresh):
+        assert torch.equal(a, b)
+
+    # then a decode step on the same workspace
+    assert pf.ws.numel() >= zha.workspace_bytes(cfg, 1)
+    Qd = Q[:, :1].contiguous()
+    N_d = torch.full((cfg.batch,), Np + 1, dtype=torch.int32, device="cuda")
+
+    def decode(ws):
+        sel = torch.zeros((cfg.batch, 1, cfg.Hq, pf.sel_cap), dtype=torch.int32, device="cuda")
+        cnt = torch.zeros((cfg.batch, 1, cfg.Hq), dtype=torch.int32, device="cuda")
+        out = torch.zeros((cfg.batch, 1, cfg.Hq, cfg.d), dtype=torch.float32, device="cuda")
+        zha.route(cfg, pf.tree, Qd, N_d, sel, cnt, ws)
+        zha.attend(cfg, pf.K, pf.V, pf.tree, Qd, N_d, sel, cnt, out, ws)
+        return sel, cnt, out
+
+    reused = decode(pf.ws)
+    fresh = decode(zha.alloc_workspace(cfg, 1))
+    torch.cuda.synchronize()
+    for a, b in zip(reused, fresh):
+        assert torch.equal(a, b)
+    assert_status_clean()
