@@ -12,7 +12,7 @@ planted-cluster synthetic keys and queries.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference]
 
 Prints one JSON line on rank 0.  Times are CUDA-event device times on the
-launching stream (max over ranks); L2 is flushed (256 MiB write) before every
+launching stream (max over ranks); L2 is flushed (256 MiB write, then a 256 MiB read) before every
 timed step, outside the events.
 """
 from __future__ import annotations
@@ -38,7 +38,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 UNIT = "queries/s"
 FALLBACK_HBM_GBS = 6650.0
 POOL = 64                 # distinct (q, k_new, v_new) sets cycled through by the steps
+E2E_WARMUP = 3            # untimed end-to-end steps before the timed ones
 ATTEND_SOURCES = ["hierarchical_tree_indexed_b200/csrc/zha_attend.cuh",
+                  "hierarchical_tree_indexed_b200/csrc/zha_attend_tc.cuh",
+                  "hierarchical_tree_indexed_b200/csrc/zha_umma.cuh",
                   "hierarchical_tree_indexed_b200/csrc/zha_common.cuh"]
 
 
@@ -74,8 +77,27 @@ def config_dict(w, world: int) -> dict:
     return {"workload": f"{w.name}: batch {w.batch} per GPU, {w.Hq} query / {w.Hkv} KV heads, d {w.d}, "
                         f"bf16 K/V, N={w.N}, leaf block {w.B}, branching {w.b}, p={w.p}",
             "global_batch": w.batch * world, "seq_len": w.N, "parallelism": f"dp{world}",
-            "kv_dtype": w.dtype, "l2": "flushed (256 MiB write) before every timed step; KV 16 GiB > L2",
+            "kv_dtype": w.dtype,
+            "l2": L2Flush.NOTE + f"; KV {w.batch * w.Hkv * w.N * w.d * 2 * (2 if w.dtype == 'bf16' else 4) / 2**30:.1f} GiB > L2",
             "step": "append + route (plan fused) + attend, each phase one CUDA graph"}
+
+
+class L2Flush:
+    """Flushes L2 between timed steps: writes a 256 MiB buffer (twice L2), then reads another
+    256 MiB buffer, so that L2 holds neither the step's inputs nor dirty lines that the timed
+    kernels would have to write back to HBM.  Runs outside the timed region."""
+    NOTE = "flushed before every timed step (256 MiB write, then 256 MiB read of another buffer: no dirty lines left)"
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+        self.out = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        import torch
+        self.w.zero_()
+        torch.sum(self.r, dim=0, out=self.out)
 
 
 def measured_peaks(key: str = "hbm_gbs") -> tuple[float, str]:
@@ -292,7 +314,7 @@ class DecodeRun:
         for k in range(steps):
             self.load(self.step)
             self.step += 1
-            flush.zero_()
+            flush()
             e = ev[k]
             e[0].record(stream)
             g_app.replay()
@@ -314,7 +336,7 @@ class DecodeRun:
         stream = torch.cuda.current_stream()
         evs = []
         for _ in range(reps + 2):
-            flush.zero_()
+            flush()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream); self.g_dense.replay(); b.record(stream)
             evs.append((a, b))
@@ -343,7 +365,7 @@ def sweep(args, rank):
     dev = torch.device("cuda", rank.local)
     torch.cuda.set_device(dev)
     base = W.WORKLOADS["decode1m"]
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     points = []
     for n in [int(x) for x in args.sweep.split(",")]:
         w = dataclasses.replace(base, N=n, n_clusters=max(1, n // 2048), batch=args.batch or 1)
@@ -434,7 +456,7 @@ def prefill_main(args, rank, w):
         graphs.append(g)
     torch.cuda.synchronize()
     g_route, g_att, g_dense = graphs
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     for _ in range(args.warmup):
         g_route.replay(); g_att.replay()
     torch.cuda.synchronize()
@@ -449,7 +471,7 @@ def prefill_main(args, rank, w):
     time.sleep(0.25)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_steps)]
     for k in range(K_steps):
-        flush.zero_()
+        flush()
         e = ev[k]
         e[0].record(stream); g_route.replay(); e[1].record(stream); g_att.replay(); e[2].record(stream)
     torch.cuda.synchronize()
@@ -479,7 +501,7 @@ def prefill_main(args, rank, w):
     # dense causal prefill, same kernel without the selection
     dense_ev = []
     for _ in range(5):
-        flush.zero_()
+        flush()
         a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a_.record(stream); g_dense.replay(); b_.record(stream)
         dense_ev.append((a_, b_))
@@ -527,7 +549,7 @@ def prefill_main(args, rank, w):
         torch.cuda.synchronize()
         cev = []
         for _ in range(4):
-            flush.zero_()
+            flush()
             a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a_.record(stream); gc_.replay(); b_.record(stream)
             cev.append((a_, b_))
@@ -549,10 +571,11 @@ def prefill_main(args, rank, w):
         kh = K[:, :, Np:].cpu().pin_memory()
         vh = V[:, :, Np:].cpu().pin_memory()
         oh = torch.empty_like(O, device="cpu").pin_memory()
-        torch.cuda.synchronize()
         a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a_.record(stream)
-        for _ in range(e2e_steps):
+        for k in range(E2E_WARMUP + e2e_steps):
+            if k == E2E_WARMUP:   # untimed warm-up steps first
+                torch.cuda.synchronize()
+                a_.record(stream)
             Q.copy_(qh, non_blocking=True)
             K[:, :, Np:].copy_(kh, non_blocking=True)
             V[:, :, Np:].copy_(vh, non_blocking=True)
@@ -565,7 +588,7 @@ def prefill_main(args, rank, w):
         e2e = {"value": w.batch * n_q * e2e_steps * rank.world / t_e2e, "unit": UNIT,
                "h2d_bytes_per_step": qh.numel() * 2 + kh.numel() * 2 + vh.numel() * 2,
                "d2h_bytes_per_step": oh.numel() * 4, "steps": e2e_steps,
-               "note": "zha_route + zha_attend per chunk (not graphed), pinned host Q, chunk K/V and O"}
+               "note": "zha_route + zha_attend per chunk (not graphed) after 3 untimed chunks, pinned host Q, chunk K/V and O"}
     cpu = None
     if rank.leader and rank.world == 1 and not args.no_cpu_baseline:
         per_head, done, setup = oracle_sample(w, args.cpu_seconds)
@@ -582,7 +605,7 @@ def prefill_main(args, rank, w):
                                    f"bf16, prefix N={Np} in the tree, chunk of {n_q} causal queries, leaf block "
                                    f"{w.B}, branching {w.b}, p={w.p}",
                        "global_batch": w.batch * rank.world, "seq_len": N_cap, "parallelism": f"dp{rank.world}",
-                       "l2": "flushed (256 MiB write) before every timed step",
+                       "l2": L2Flush.NOTE,
                        "step": "zha_route + zha_attend of one chunk, each one CUDA graph"},
             "roofline": {"bound": "tensor", "kernel": "attend phase (plan + attend_prefill_kernel + merge)",
                          "achieved": att_tflops, "peak": peak, "unit": "TFLOP/s", "frac": att_tflops / peak,
@@ -628,9 +651,9 @@ def main():
     w = workload(args)
     K_steps, W_steps = args.steps, args.warmup
     e2e_steps = 0 if args.no_e2e else min(K_steps, 500)
-    N_cap = w.N + W_steps + K_steps + e2e_steps + 8
+    N_cap = w.N + W_steps + K_steps + E2E_WARMUP + e2e_steps + 8
     run = DecodeRun(w, dev, N_cap, rank)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     for _ in range(W_steps):
         run.load(run.step)
         run.step += 1
@@ -672,12 +695,13 @@ def main():
         qh.copy_(run.Qp.reshape(POOL, w.batch, 1, w.Hq, w.d).cpu())
         kh = run.knp.cpu().pin_memory()
         vh = run.vnp.cpu().pin_memory()
-        oh = torch.empty((e2e_steps, w.batch, 1, w.Hq, w.d), dtype=torch.float32).pin_memory()
-        torch.cuda.synchronize()
-        D.barrier(rank, dev)
+        oh = torch.empty((E2E_WARMUP + e2e_steps, w.batch, 1, w.Hq, w.d), dtype=torch.float32).pin_memory()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for k in range(e2e_steps):
+        for k in range(E2E_WARMUP + e2e_steps):
+            if k == E2E_WARMUP:   # untimed warm-up steps first
+                torch.cuda.synchronize()
+                D.barrier(rank, dev)
+                a.record(stream)
             j = k % POOL
             run.q_in.copy_(qh[j], non_blocking=True)
             run.k_in.copy_(kh[j], non_blocking=True)
@@ -690,7 +714,7 @@ def main():
         e2e = {"value": w.batch * e2e_steps * rank.world / t_e2e, "unit": UNIT,
                "h2d_bytes_per_step": (run.q_in.numel() + run.k_in.numel() + run.v_in.numel()) * es,
                "d2h_bytes_per_step": run.O.numel() * 4, "steps": e2e_steps,
-               "note": "zha_decode per step (not graphed), pinned host inputs/outputs, L2 not flushed"}
+               "note": "zha_decode per step (not graphed) after 3 untimed steps, pinned host inputs/outputs, L2 not flushed"}
         run.check_status("the e2e steps")
 
     cpu = None
@@ -708,7 +732,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": config_dict(w, rank.world),
             "hbm_gbs": step_gbs, "hbm_frac_of_peak": step_gbs / peak,
-            "roofline": {"bound": "hbm", "kernel": "attend_kernel", "achieved": att_gbs, "peak": peak,
+            "roofline": {"bound": "hbm", "kernel": run.zha.attend_kernel(run.cfg), "achieved": att_gbs, "peak": peak,
                          "unit": "GB/s", "frac": att_gbs / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} copy bandwidth", "algorithmic_bytes_per_launch": attend_bytes,
                          "kernel_source_sha256_16": khash},

@@ -20,6 +20,7 @@
 #include "zha_plan.cuh"
 #include "zha_route.cuh"
 #include "zha_attend.cuh"
+#include "zha_attend_tc.cuh"
 #include "zha_prefill.cuh"
 
 using namespace zha;
@@ -319,6 +320,35 @@ int run_route(const zha_config* c, const TreeLayout& lay, const WsLayout& wl, co
 }
 
 // ---------------------------------------------------------------- attend
+int make_kv_map(const zha_config* c, const void* base, CUtensorMap* map);
+int make_q_map(const zha_config* c, const void* base, int64_t rows, CUtensorMap* map);
+
+int attend_grid(const DevInfo& di) { return std::min(di.sms, kSplitMax); }   // a group has at most `grid` partials
+
+// The tensor-core decode attention takes bf16, d = 128 and leaf blocks of whole 64-key
+// tiles (items then start on a block and a 64-key box holds each); other shapes, or
+// more groups than its shared memory holds, run on attend_kernel.
+bool attend_tc_fits(const zha_config* c, const DevInfo& di) {
+    return c->dtype == ZHA_BF16 && c->d == 128 && c->B % 64 == 0 &&
+           tc_smem_bytes(c->batch * c->Hkv, attend_grid(di)) <= static_cast<size_t>(di.smem_optin);
+}
+
+template <int G>
+int run_attend_tc(const zha_config* c, const AttendArgs& a, cudaStream_t st) {
+    CUtensorMap mk, mv, mq;
+    ZHA_TRY(make_kv_map(c, a.K, &mk));
+    ZHA_TRY(make_kv_map(c, a.V, &mv));
+    ZHA_TRY(make_q_map(c, a.Q, static_cast<int64_t>(c->batch) * a.n_q * c->Hq, &mq));
+    auto kern = attend_tc_kernel<G>;
+    DevInfo di;
+    ZHA_TRY(dev_info(&di));
+    const int grid = attend_grid(di);
+    const size_t smem = tc_smem_bytes(a.groups, grid);
+    ZHA_TRY(allow_smem(kern, smem));
+    kern<<<grid, kTCThreads, smem, st>>>(mk, mv, mq, a);
+    return check_launch("attend_tc");
+}
+
 template <typename T, int D, int G>
 int run_attend_t(const AttendArgs& a, cudaStream_t st) {
     auto kern = attend_kernel<T, D, G>;
@@ -347,6 +377,15 @@ int run_attend(const zha_config* c, const WsLayout& wl, const void* K, const voi
     a.item_cap = wl.item_cap; a.N_cap = c->N_cap;
     a.groups = c->batch * c->Hkv; a.Hq = c->Hq; a.Hkv = c->Hkv; a.n_q = 1;
     a.qscale = scale_of(c) * 1.4426950408889634f;
+    DevInfo di;
+    ZHA_TRY(dev_info(&di));
+    if (attend_tc_fits(c, di)) {
+        switch (c->Hq / c->Hkv) {
+            case 1: return run_attend_tc<1>(c, a, st);
+            case 2: return run_attend_tc<2>(c, a, st);
+            default: return run_attend_tc<4>(c, a, st);
+        }
+    }
     switch (c->Hq / c->Hkv) {
         case 1: return run_attend_t<T, D, 1>(a, st);
         case 2: return run_attend_t<T, D, 2>(a, st);
@@ -437,19 +476,25 @@ int pf_layout(const zha_config* c, int n_q, const TreeLayout& t, PfLayout* p) {
 
 // Tiled TMA map over K or V viewed as [batch*Hkv][N_cap][d] bf16, boxes of 64 keys x 64
 // columns with the 128-byte swizzle the tensor-core operands expect.
-int make_kv_map(const zha_config* c, const void* base, CUtensorMap* map) {
+int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
     static std::mutex mu;
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-    {
-        std::lock_guard<std::mutex> lk(mu);
-        if (!encode) {
-            void* fn = nullptr;
-            cudaDriverEntryPointQueryResult q;
-            ZHA_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
-            if (q != cudaDriverEntryPointSuccess || !fn) return fail(ZHA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-            encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-        }
+    std::lock_guard<std::mutex> lk(mu);
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        ZHA_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+        if (q != cudaDriverEntryPointSuccess || !fn) return fail(ZHA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
+    *out = encode;
+    return ZHA_OK;
+}
+
+// bf16 K or V cache [batch*Hkv][N_cap][d] as boxes of 64 dims x 64 keys, 128-byte swizzle.
+int make_kv_map(const zha_config* c, const void* base, CUtensorMap* map) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    ZHA_TRY(tensor_map_encoder(&encode));
     if (reinterpret_cast<uintptr_t>(base) % 16) return fail(ZHA_ERR_INVALID_ARG, "K/V must be 16-byte aligned");
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(c->d), static_cast<cuuint64_t>(c->N_cap),
                                 static_cast<cuuint64_t>(c->batch) * c->Hkv};
@@ -457,6 +502,22 @@ int make_kv_map(const zha_config* c, const void* base, CUtensorMap* map) {
     const cuuint32_t box[3] = {64, 64, 1};
     const cuuint32_t estride[3] = {1, 1, 1};
     const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                              estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ZHA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return ZHA_OK;
+}
+
+// bf16 queries [rows][d] as boxes of 64 dims x 16 rows, 128-byte swizzle.
+int make_q_map(const zha_config* c, const void* base, int64_t rows, CUtensorMap* map) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    ZHA_TRY(tensor_map_encoder(&encode));
+    if (reinterpret_cast<uintptr_t>(base) % 16) return fail(ZHA_ERR_INVALID_ARG, "Q must be 16-byte aligned");
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(c->d), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(c->d) * 2};
+    const cuuint32_t box[2] = {64, 16};
+    const cuuint32_t estride[2] = {1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                               estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(ZHA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -717,6 +778,24 @@ int zha_workspace_stats(const zha_config* cfg, int32_t n_q, size_t* rows_offset,
     ZHA_TRY(ws_layout(cfg, n_q, t, &w));
     *rows_offset = w.off_rows;
     *cand_offset = w.off_cand;
+    return ZHA_OK;
+}
+
+int zha_attend_kernel(const zha_config* cfg, int32_t n_q, int32_t* kind) {
+    TreeLayout t;
+    ZHA_TRY(need(kind, "kind"));
+    ZHA_TRY(tree_layout(cfg, &t));
+    if (n_q > 1) {
+        PfLayout p;
+        ZHA_TRY(pf_layout(cfg, n_q, t, &p));
+        *kind = 2;
+        return ZHA_OK;
+    }
+    WsLayout w;
+    ZHA_TRY(ws_layout(cfg, n_q, t, &w));
+    DevInfo di;
+    ZHA_TRY(dev_info(&di));
+    *kind = attend_tc_fits(cfg, di) ? 1 : 0;
     return ZHA_OK;
 }
 

@@ -1,0 +1,551 @@
+// zha_attend_tc.cuh -- decode attention over the routed key set on the
+// 5th-generation tensor cores (sm_100a): bf16 K/V/Q, head dim 128, leaf blocks
+// of a whole multiple of 64 keys.
+//
+// Pages: [HTI] "Subquadratic Attention with a Hierarchical Tree-Structured
+// Indexer", Methodology / Routing: o(q) = Attn(q, K_I, V_I) over I(q) = {0} u
+// (kept level-1 chunks) u C_cur(q), computed exactly as dense attention over
+// those keys ([EoQ] "Zyphra Hierarchical Attention: The End of Quadratic
+// Attention?", A query's path).
+//
+// The same work as attend_kernel (zha_attend.cuh) -- the same plan (items of at
+// most 64 keys with a head mask, concatenated over the groups and cut into one
+// contiguous piece per CTA), the same partials and the same group merge -- with
+// the arithmetic of a piece on the tensor cores.  Two items form a pair of 128
+// key rows:
+//   S^T  = K Q^T     M = 128 keys, N = 16 (the group's G query heads, the rest
+//                    ignored), K = 128 dims; A = K tile K-major, B = Q K-major
+//   O^T += V^T P^T   M = 128 dims, N = 16, K = 128 keys; A = the V tile read
+//                    MN-major (dims contiguous), B = P^T K-major
+// P enters as two bf16 parts, hi = bf16(P) in column h and lo = bf16(P - hi)
+// in column 4 + h, so P = hi + lo to 2^-18 relative and the output keeps fp32
+// accuracy although the tensor cores take bf16; O = column h + column 4 + h.
+// Warps 0-3: softmax (thread i owns key row i of a pair, and dimension i of O);
+// warp 4: TMA producer; warp 5: TMEM owner and MMA issue (one lane).  The
+// online softmax runs in log2 units; O is rescaled lazily, only when a head's
+// running max outgrows its reference by 2^8.
+// Every wait is bounded: a timeout raises ZHA_ERR_TIMEOUT, marks the CTA
+// aborted, and all later waits return at once, so the kernel always ends.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "zha_attend.cuh"
+#include "zha_umma.cuh"
+
+namespace zha {
+
+constexpr int kTCStages = 3;                                   // pairs of items in flight
+constexpr int kTCThreads = 192;
+constexpr uint32_t kTCKBytes = 2 * 128 * 128;                  // 128 keys x 128 dims, two 64-dim spans
+constexpr uint32_t kTCSpan = 128 * 128;                        // one 64-dim span of a pair
+constexpr uint32_t kTCItem = 64 * 128;                         // one item's rows inside a span
+constexpr uint32_t kTCQBytes = 2 * 16 * 128;                   // 16 query rows x 128 dims
+constexpr uint32_t kTCStageBytes = 2 * kTCKBytes + kTCQBytes;  // K, V, Q of a pair
+constexpr uint32_t kTCPBytes = 2 * 16 * 128;                   // P^T: 16 rows x 128 keys
+constexpr uint32_t kTCOffP = kTCStages * kTCStageBytes;
+constexpr uint32_t kTCOffCtl = kTCOffP + 2 * kTCPBytes;
+constexpr uint32_t kTCTmemCols = 64;                           // S: 2 x 16 columns; O: 16 columns at 32
+constexpr float kTCRescaleLog2 = 8.0f;                         // lazy rescale: P stays below 2^8 between rescales
+
+struct TcDesc {
+    int n0, n1;                // keys of the pair's items (n1 = 0: one item); n0 < 0: no more work
+    uint32_t heads0, heads1;   // head masks of the two items
+    int group, split;
+    int flags;                 // bit 0: last pair of this CTA's piece of the group; bit 1: first pair
+    int pad;
+};
+
+struct TcCtl {
+    uint64_t kv_full[kTCStages];   // TMA -> all: K, V, Q of the pair landed (and its descriptor written)
+    uint64_t kv_empty[kTCStages];  // MMA -> TMA: P V of the pair completed
+    uint64_t s_full[2];            // MMA -> softmax: S^T of pair g in TMEM buffer g & 1
+    uint64_t s_free[2];            // softmax -> MMA: S^T buffer read
+    uint64_t p_full[2];            // softmax -> MMA: P^T of pair g written, O rescaled
+    uint64_t o_done[2];            // MMA -> softmax: P V of pair g (and every MMA before it) completed
+    uint64_t mx[2];                // softmax warps: pair maxima exchanged
+    uint64_t ep[3];                // softmax warps: partial sums exchanged / partial stored / merge decided
+    uint64_t mg[2];                // softmax warps: a merge's (max, sum) gathered / weights computed
+    uint64_t fin;                  // MMA lane: every MMA it issued completed
+    TcDesc desc[kTCStages];
+    uint32_t tmem;
+    int abort;
+    int last_flag, sp;
+    int red[2][4][4];              // [pair parity][warp][head] order-mapped maxima
+    float lsum[4][4];              // [warp][head] softmax sums
+    float mL[4];                   // [head] a merge's total sum
+    int scan[8];
+    int prefix[1];                 // [groups + 1] first global item of each group; then the merge's
+                                   // (max, sum) -> (weight, sum) of every partial, float2 [grid][4]
+};
+
+__host__ __device__ constexpr size_t tc_merge_offset(int groups) {   // from the start of TcCtl, 8-aligned
+    return (sizeof(TcCtl) + sizeof(int) * static_cast<size_t>(groups) + 7) & ~static_cast<size_t>(7);
+}
+__host__ __device__ constexpr size_t tc_smem_bytes(int groups, int grid) {
+    return kTCOffCtl + tc_merge_offset(groups) + sizeof(float2) * 4 * static_cast<size_t>(grid) + 1024;   // + alignment slack
+}
+
+// Bounded wait; a timeout is recorded once and later waits of the CTA return at once.
+__device__ __forceinline__ bool twait(uint64_t* bar, uint32_t parity, TcCtl* ctl) {
+    if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
+    if (mbar_wait_bounded(bar, parity)) return true;
+    *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+    raise_status(ZHA_ERR_TIMEOUT);
+    return false;
+}
+__device__ __forceinline__ bool tc_aborted(TcCtl* ctl) { return *reinterpret_cast<volatile int*>(&ctl->abort) != 0; }
+
+// Order-preserving map of floats (no NaN) to int, for the integer warp max.
+__device__ __forceinline__ int ord_of(float x) {
+    const int i = __float_as_int(x);
+    return i >= 0 ? i : i ^ 0x7fffffff;
+}
+__device__ __forceinline__ float of_ord(int k) { return __int_as_float(k >= 0 ? k : k ^ 0x7fffffff); }
+
+template <int G>
+__global__ void __launch_bounds__(kTCThreads, 1)
+    attend_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmQ, AttendArgs a) {
+    constexpr int D = 128;
+    static_assert(G >= 1 && G <= 4, "at most 4 query heads per KV head");
+    extern __shared__ __align__(1024) unsigned char tc_smem[];
+    const uint32_t raw_s = smem_addr(tc_smem);
+    unsigned char* base = tc_smem + (((raw_s + 1023u) & ~1023u) - raw_s);
+    unsigned char* sP = base + kTCOffP;
+    TcCtl* ctl = reinterpret_cast<TcCtl*>(base + kTCOffCtl);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    auto stage = [&](int s) { return base + static_cast<uint32_t>(s) * kTCStageBytes; };
+
+    // ---- prefix[g] = first global item of group g; barriers; TMEM; P^T rows 8..15 stay zero
+    {
+        int carry = 0;
+        for (int b0 = 0; b0 < a.groups; b0 += kTCThreads) {
+            const int g = b0 + tid;
+            const int n = g < a.groups ? a.n_items[g] : 0;
+            int tot;
+            const int x = block_exclusive_scan<kTCThreads / 32>(n, ctl->scan, &tot);
+            if (g < a.groups) ctl->prefix[g] = carry + x;
+            carry += tot;
+        }
+        if (tid == 0) {
+            ctl->prefix[a.groups] = carry;
+            for (int i = 0; i < kTCStages; ++i) {
+                mbar_init(&ctl->kv_full[i], 1);
+                mbar_init(&ctl->kv_empty[i], 1);
+            }
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(&ctl->s_full[i], 1);
+                mbar_init(&ctl->s_free[i], 128);
+                mbar_init(&ctl->p_full[i], 128);
+                mbar_init(&ctl->o_done[i], 1);
+                mbar_init(&ctl->mx[i], 4);
+            }
+            mbar_init(&ctl->ep[0], 4);
+            mbar_init(&ctl->ep[1], 4);
+            mbar_init(&ctl->ep[2], 1);
+            mbar_init(&ctl->mg[0], 4);
+            mbar_init(&ctl->mg[1], 4);
+            mbar_init(&ctl->fin, 1);
+            fence_mbar_init();
+            ctl->abort = 0;
+            umma::prefetch_tensormap(&tmK);
+            umma::prefetch_tensormap(&tmV);
+            umma::prefetch_tensormap(&tmQ);
+        }
+        for (int x = tid; x < static_cast<int>(2 * kTCPBytes / 16); x += kTCThreads)
+            reinterpret_cast<uint4*>(sP)[x] = make_uint4(0u, 0u, 0u, 0u);
+        if (warp == 5) {
+            umma::tmem_alloc(&ctl->tmem, kTCTmemCols);
+            umma::tmem_relinquish();
+        }
+        umma::fence_proxy_async_smem();
+        umma::fence_before_sync();
+        __syncthreads();
+        umma::fence_after_sync();
+    }
+    const uint32_t tmem = ctl->tmem;
+    const int64_t I = ctl->prefix[a.groups];
+    const int C = gridDim.x;
+    const int64_t ch = I > 0 ? (I + C - 1) / C : 1;   // items per CTA: one contiguous piece each
+
+    if (warp == 4) {
+        // ================= TMA producer: this CTA's piece, two items per pair
+        int fills = 0;     // pairs posted (lane 0's count is the one used)
+        bool ok = true;
+        auto acquire = [&](int f) -> bool {
+            return f < kTCStages || twait(&ctl->kv_empty[f % kTCStages], ((f / kTCStages) - 1) & 1, ctl);
+        };
+        const int64_t j = blockIdx.x;
+        if (j * ch < I) {
+            const int64_t x_end = min(I, (j + 1) * ch);
+            int g = 0;
+            for (int64_t x = j * ch; x < x_end && ok;) {
+                while (ctl->prefix[g + 1] <= x) ++g;   // the group holding item x
+                const int64_t g0 = ctl->prefix[g], g1 = ctl->prefix[g + 1];
+                const int64_t seg_end = min(x_end, g1);
+                const int i0 = static_cast<int>(x - g0), nseg = static_cast<int>(seg_end - x);
+                // CTAs start at different points of their segments (the order of the keys does
+                // not matter to the softmax), so concurrent CTAs stream different address patterns
+                const int rot = static_cast<int>((static_cast<uint32_t>(blockIdx.x) * 2654435761u) %
+                                                 static_cast<uint32_t>(nseg));
+                const int s = g / a.Hkv, kv = g % a.Hkv;
+                const int qrow = (s * a.n_q + (a.n_q - 1)) * a.Hq + kv * G;
+                const int2* its = a.items + static_cast<int64_t>(g) * a.item_cap;
+                auto item_at = [&](int v) {   // the segment's v-th item in this CTA's order
+                    v += rot;
+                    if (v >= nseg) v -= nseg;
+                    return its[i0 + v];
+                };
+                int2 nx = make_int2(0, 0);    // the next batch of 32 items
+                if (lane < nseg) nx = item_at(lane);
+                for (int vb = 0; vb < nseg && ok; vb += 32) {
+                    const int avail = min(32, nseg - vb);
+                    const int2 it = nx;
+                    nx = make_int2(0, 0);
+                    if (vb + 32 + lane < nseg) nx = item_at(vb + 32 + lane);
+                    int c = it.y & 0xffff;
+                    if (lane < avail && (c < 1 || c > 64)) {
+                        raise_status(ZHA_ERR_INVALID_ARG);
+                        c = 0;
+                    }
+                    const uint32_t m = static_cast<uint32_t>(it.y) >> 16;
+                    for (int p = 0; p < avail; p += 2) {
+                        const bool two = p + 1 < avail;
+                        const int q1 = two ? p + 1 : p;
+                        const int st0 = __shfl_sync(0xffffffffu, it.x, p);
+                        const int st1 = __shfl_sync(0xffffffffu, it.x, q1);
+                        const int c0 = __shfl_sync(0xffffffffu, c, p);
+                        const int c1 = two ? __shfl_sync(0xffffffffu, c, q1) : 0;
+                        const uint32_t m0 = __shfl_sync(0xffffffffu, m, p);
+                        const uint32_t m1 = __shfl_sync(0xffffffffu, m, q1);
+                        int posted = 0;
+                        if (lane == 0 && acquire(fills)) {
+                            const int slot = fills % kTCStages;
+                            TcDesc& d = ctl->desc[slot];
+                            d.n0 = c0;
+                            d.n1 = c1;
+                            d.heads0 = c0 > 0 ? m0 : 0u;
+                            d.heads1 = c1 > 0 ? m1 : 0u;
+                            d.group = g;
+                            d.split = blockIdx.x;
+                            d.flags = (vb + p + 2 >= nseg ? 1 : 0) | (vb + p == 0 ? 2 : 0);
+                            unsigned char* sb = stage(slot);
+                            uint64_t* bar = &ctl->kv_full[slot];
+                            const uint32_t bytes = (c0 > 0 ? 2 * kTCSpan : 0u) + (c1 > 0 ? 2 * kTCSpan : 0u) + kTCQBytes;
+                            mbar_arrive_expect_tx(bar, bytes);
+                            // an item's 64 rows from its first key (rows past the cache's end
+                            // read as zeros), both 64-dim spans, K and V
+                            if (c0 > 0) {
+                                umma::tma_load_3d(sb, &tmK, 0, st0, g, bar);
+                                umma::tma_load_3d(sb + kTCSpan, &tmK, 64, st0, g, bar);
+                                umma::tma_load_3d(sb + kTCKBytes, &tmV, 0, st0, g, bar);
+                                umma::tma_load_3d(sb + kTCKBytes + kTCSpan, &tmV, 64, st0, g, bar);
+                            }
+                            if (c1 > 0) {
+                                umma::tma_load_3d(sb + kTCItem, &tmK, 0, st1, g, bar);
+                                umma::tma_load_3d(sb + kTCSpan + kTCItem, &tmK, 64, st1, g, bar);
+                                umma::tma_load_3d(sb + kTCKBytes + kTCItem, &tmV, 0, st1, g, bar);
+                                umma::tma_load_3d(sb + kTCKBytes + kTCSpan + kTCItem, &tmV, 64, st1, g, bar);
+                            }
+                            umma::tma_load_2d(sb + 2 * kTCKBytes, &tmQ, 0, qrow, bar);
+                            umma::tma_load_2d(sb + 2 * kTCKBytes + kTCQBytes / 2, &tmQ, 64, qrow, bar);
+                            posted = 1;
+                        }
+                        ok = __shfl_sync(0xffffffffu, posted, 0) != 0;
+                        if (!ok) break;
+                        ++fills;
+                    }
+                }
+                x = seg_end;
+            }
+        }
+        if (lane == 0) {
+            if (ok && acquire(fills)) {   // sentinel: no pair follows
+                ctl->desc[fills % kTCStages].n0 = -1;
+                mbar_arrive(&ctl->kv_full[fills % kTCStages]);
+                ++fills;
+            }
+            // the loads of the last pairs have landed before the CTA may exit
+            for (int f = fills > kTCStages ? fills - kTCStages : 0; f < fills; ++f)
+                mbar_wait_bounded(&ctl->kv_full[f % kTCStages], (f / kTCStages) & 1);
+        }
+    } else if (warp == 5) {
+        // ================= MMA issue (one lane): S^T and P V of the pairs in order
+        if (lane == 0) {
+            constexpr uint32_t kIdS = umma::idesc_bf16_ab(128, 16, false, false);
+            constexpr uint32_t kIdO = umma::idesc_bf16_ab(128, 16, true, false);
+            const uint32_t tO = tmem + 32;
+            auto pv = [&](uint32_t h) {   // P^T of pair h is written
+                const int slot = static_cast<int>(h % kTCStages);
+                umma::fence_after_sync();
+                const bool first = (ctl->desc[slot].flags & 2) != 0;
+                const unsigned char* vb = stage(slot) + kTCKBytes;
+                const unsigned char* pb = sP + (h & 1u) * kTCPBytes;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {   // 16 keys per step
+                    const uint64_t ad = umma::desc_sw128(smem_addr(vb + kk * 2048), kTCSpan, 1024);
+                    const uint64_t bd = umma::desc_sw128(smem_addr(pb + (kk >> 2) * 2048 + (kk & 3) * 32), 16, 1024);
+                    umma::mma_bf16(tO, ad, bd, kIdO, (kk > 0 || !first) ? 1u : 0u);
+                }
+                umma::commit(&ctl->o_done[h & 1u]);
+                umma::commit(&ctl->kv_empty[slot]);
+            };
+            // S^T of pair gs as soon as its tiles landed and its TMEM buffer is free; P V of pair
+            // gp as soon as its softmax is done -- polled, so that neither waits on the other and
+            // a pair's stage is released right after its own softmax.
+            uint32_t gs = 0, gp = 0;
+            bool no_more = false;
+            uint64_t t_last = global_timer_ns();
+            for (uint32_t idle = 0;;) {
+                bool progress = false;
+                if (!no_more) {
+                    const int slot = static_cast<int>(gs % kTCStages);
+                    if (mbar_test_wait(&ctl->kv_full[slot], (gs / kTCStages) & 1u)) {
+                        if (ctl->desc[slot].n0 < 0) {
+                            no_more = true;
+                        } else if (gs < 2 || mbar_test_wait(&ctl->s_free[gs & 1u], ((gs - 2) >> 1) & 1u)) {
+                            umma::fence_after_sync();
+                            const unsigned char* kb = stage(slot);
+                            const unsigned char* qb = kb + 2 * kTCKBytes;
+                            const uint32_t tS = tmem + (gs & 1u) * 16;
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk) {   // 16 dims per step
+                                const uint64_t ad = umma::desc_sw128(smem_addr(kb + (kk >> 2) * kTCSpan + (kk & 3) * 32), 16, 1024);
+                                const uint64_t bd = umma::desc_sw128(smem_addr(qb + (kk >> 2) * (kTCQBytes / 2) + (kk & 3) * 32), 16, 1024);
+                                umma::mma_bf16(tS, ad, bd, kIdS, kk > 0 ? 1u : 0u);
+                            }
+                            umma::commit(&ctl->s_full[gs & 1u]);
+                            ++gs;
+                            progress = true;
+                        }
+                    }
+                }
+                if (gp < gs && mbar_test_wait(&ctl->p_full[gp & 1u], (gp >> 1) & 1u)) {
+                    pv(gp);
+                    ++gp;
+                    progress = true;
+                }
+                if (no_more && gp == gs) break;
+                if (progress) {
+                    idle = 0;
+                    t_last = global_timer_ns();
+                } else if ((++idle & 1023u) == 0) {
+                    if (tc_aborted(ctl)) break;
+                    if (global_timer_ns() - t_last > 2000000000ull) {
+                        *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+                        raise_status(ZHA_ERR_TIMEOUT);
+                        break;
+                    }
+                }
+            }
+            umma::commit(&ctl->fin);
+            mbar_wait_bounded(&ctl->fin, 0);
+        }
+    } else {
+        // ================= softmax warps 0-3
+        const int i = tid;   // key row i of each pair; dimension i of O
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        float m_ref[4], l[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            m_ref[h] = -INFINITY;
+            l[h] = 0.f;
+        }
+        uint32_t e = 0, nm = 0;   // epilogues and merges so far
+        float2* mbuf = reinterpret_cast<float2*>(reinterpret_cast<unsigned char*>(ctl) + tc_merge_offset(a.groups));
+        for (uint32_t g = 0;; ++g) {
+            if (tc_aborted(ctl)) break;
+            const int slot = static_cast<int>(g % kTCStages);
+            twait(&ctl->kv_full[slot], (g / kTCStages) & 1u, ctl);
+            if (tc_aborted(ctl)) break;
+            const TcDesc d = ctl->desc[slot];
+            if (d.n0 < 0) break;
+            const bool first = (d.flags & 2) != 0, last = (d.flags & 1) != 0;
+            const int n = i < 64 ? d.n0 : d.n1;
+            const uint32_t hm = i < 64 ? d.heads0 : d.heads1;
+            const bool vrow = (i & 63) < n;
+            if (first) {
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    m_ref[h] = -INFINITY;
+                    l[h] = 0.f;
+                }
+            }
+            if (!vrow) {   // the tensor cores read every V row of the pair: rows outside the items are zeroed
+                unsigned char* vr = stage(slot) + kTCKBytes + i * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    reinterpret_cast<uint4*>(vr)[c] = make_uint4(0u, 0u, 0u, 0u);
+                    reinterpret_cast<uint4*>(vr + kTCSpan)[c] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            twait(&ctl->s_full[g & 1u], (g >> 1) & 1u, ctl);
+            umma::fence_after_sync();
+            float sv[4];
+            umma::tmem_ld4(tmem + (g & 1u) * 16 + lane_base, sv);
+            umma::fence_before_sync();
+            mbar_arrive(&ctl->s_free[g & 1u]);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) sv[h] = (h < G && vrow && ((hm >> h) & 1u)) ? sv[h] * a.qscale : -INFINITY;
+            // the pair's max per head over the four warps
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const int k = __reduce_max_sync(0xffffffffu, ord_of(sv[h]));
+                if (lane == 0) ctl->red[g & 1u][warp][h] = k;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->mx[g & 1u]);
+            twait(&ctl->mx[g & 1u], (g >> 1) & 1u, ctl);
+            bool resc = false;
+            float alpha[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                int k = ctl->red[g & 1u][0][h];
+#pragma unroll
+                for (int ww = 1; ww < 4; ++ww) k = max(k, ctl->red[g & 1u][ww][h]);
+                const float tmax = of_ord(k);
+                alpha[h] = 1.f;
+                if (tmax > m_ref[h] + kTCRescaleLog2) {   // lazy: move the reference only by more than 2^8
+                    if (m_ref[h] != -INFINITY) {
+                        alpha[h] = exp2f(m_ref[h] - tmax);
+                        l[h] *= alpha[h];
+                        resc = true;
+                    }
+                    m_ref[h] = tmax;
+                }
+            }
+            // P V of pair g - 2 has read the P buffer this pair writes
+            if (g >= 2) twait(&ctl->o_done[g & 1u], ((g - 2) >> 1) & 1u, ctl);
+            if (resc) {   // uniform: every thread sees the same maxima; never on a piece's first pair
+                twait(&ctl->o_done[(g - 1) & 1u], ((g - 1) >> 1) & 1u, ctl);
+                umma::fence_after_sync();
+                float o[8];
+                umma::tmem_ld8(tmem + 32 + lane_base, o);
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    o[h] *= alpha[h];
+                    o[4 + h] *= alpha[h];
+                }
+                umma::tmem_st8(tmem + 32 + lane_base, o);
+            }
+            // P^T, K-major 128-byte swizzle: row n (head part), key i -> span i / 64, chunk (i % 64) / 8
+            unsigned char* pb = sP + (g & 1u) * kTCPBytes + (i >> 6) * 2048;
+            const int kc = (i & 63) >> 3, kb = (i & 7) * 2;
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float p = sv[h] == -INFINITY ? 0.f : exp2f(sv[h] - m_ref[h]);
+                l[h] += p;
+                const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
+                *reinterpret_cast<__nv_bfloat16*>(pb + h * 128 + ((kc ^ h) << 4) + kb) = hi;
+                *reinterpret_cast<__nv_bfloat16*>(pb + (4 + h) * 128 + ((kc ^ (4 + h)) << 4) + kb) = lo;
+            }
+            umma::fence_proxy_async_smem();   // P^T and the zeroed V rows, for the tensor cores
+            umma::fence_before_sync();
+            mbar_arrive(&ctl->p_full[g & 1u]);
+
+            if (last) {
+                // ---- this CTA's partial of the group: (max, sum) per head and O^T, unnormalised
+                twait(&ctl->o_done[g & 1u], (g >> 1) & 1u, ctl);
+                umma::fence_after_sync();
+                float o[8];
+                umma::tmem_ld8(tmem + 32 + lane_base, o);
+                umma::fence_before_sync();
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float sum = warp_sum(l[h]);
+                    if (lane == 0) ctl->lsum[warp][h] = sum;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->ep[0]);
+                twait(&ctl->ep[0], e & 1u, ctl);
+                const int grp = d.group, split = d.split;
+                const int64_t pbase = (static_cast<int64_t>(grp) * kSplitMax + split) * G;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float L = (ctl->lsum[0][h] + ctl->lsum[1][h]) + (ctl->lsum[2][h] + ctl->lsum[3][h]);
+                    if (i == 0) a.part_ml[pbase + h] = make_float2(m_ref[h], L);
+                    a.part_acc[(pbase + h) * D + i] = o[h] + o[4 + h];
+                }
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->ep[1]);
+                if (i == 0) {
+                    twait(&ctl->ep[1], e & 1u, ctl);
+                    const int sp = partials_of(ctl->prefix[grp], ctl->prefix[grp + 1], ch, C);
+                    const uint32_t done = atomicAdd(&a.counters[grp], 1u);
+                    ctl->last_flag = done == static_cast<uint32_t>(sp - 1);
+                    ctl->sp = sp;
+                    mbar_arrive(&ctl->ep[2]);
+                }
+                twait(&ctl->ep[2], e & 1u, ctl);
+                if (ctl->last_flag) {
+                    // ---- this CTA closes the group: merge its partials into O.  The (max, sum)
+                    // pairs go to shared memory in parallel; warp h turns them into the weights
+                    // 2^(m_k - M_h) and the total sum; thread i then sums dimension i over the
+                    // partials with independent loads.
+                    __threadfence();
+                    const int sp = ctl->sp;
+                    const int s = grp / a.Hkv, kv = grp % a.Hkv;
+                    const int64_t pb0 = static_cast<int64_t>(grp) * kSplitMax * G;
+                    const int slot0 = static_cast<int>((ctl->prefix[grp] / ch) % C);   // partial k at slot (slot0+k) % C
+                    for (int x = i; x < sp * G; x += 128) {
+                        const int k = x / G, h = x % G;
+                        mbuf[k * 4 + h] = __ldcg(&a.part_ml[pb0 + ((slot0 + k) % C) * G + h]);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ctl->mg[0]);
+                    twait(&ctl->mg[0], nm & 1u, ctl);
+                    if (warp < G) {
+                        const int h = warp;
+                        float M = -INFINITY;
+                        for (int k = lane; k < sp; k += 32) M = fmaxf(M, mbuf[k * 4 + h].x);
+                        M = warp_max(M);
+                        float Ls = 0.f;
+                        for (int k = lane; k < sp; k += 32) {
+                            const float2 ml = mbuf[k * 4 + h];
+                            const float f = M == -INFINITY ? 0.f : exp2f(ml.x - M);
+                            mbuf[k * 4 + h].x = f;
+                            Ls = fmaf(f, ml.y, Ls);
+                        }
+                        Ls = warp_sum(Ls);
+                        if (lane == 0) ctl->mL[h] = Ls;
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ctl->mg[1]);
+                    twait(&ctl->mg[1], nm & 1u, ctl);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float* src = a.part_acc + (pb0 + h) * D + i;
+                        auto at_k = [&](int k) { return src + static_cast<int64_t>((slot0 + k) % C) * G * D; };
+                        float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+                        int k = 0;
+                        for (; k + 4 <= sp; k += 4) {
+                            const float x0 = __ldcg(at_k(k)), x1 = __ldcg(at_k(k + 1));
+                            const float x2 = __ldcg(at_k(k + 2)), x3 = __ldcg(at_k(k + 3));
+                            o0 = fmaf(mbuf[k * 4 + h].x, x0, o0);
+                            o1 = fmaf(mbuf[(k + 1) * 4 + h].x, x1, o1);
+                            o2 = fmaf(mbuf[(k + 2) * 4 + h].x, x2, o2);
+                            o3 = fmaf(mbuf[(k + 3) * 4 + h].x, x3, o3);
+                        }
+                        for (; k < sp; ++k) o0 = fmaf(mbuf[k * 4 + h].x, __ldcg(at_k(k)), o0);
+                        const float Ls = ctl->mL[h];
+                        const int64_t orow = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + h;
+                        a.O[orow * D + i] = Ls > 0.f ? ((o0 + o1) + (o2 + o3)) / Ls : 0.f;
+                    }
+                    if (i == 0) a.counters[grp] = 0u;
+                    ++nm;
+                }
+                ++e;
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 5) {
+        umma::fence_after_sync();
+        umma::tmem_dealloc(tmem, kTCTmemCols);
+    }
+}
+
+}  // namespace zha

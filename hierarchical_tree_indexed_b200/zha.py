@@ -38,7 +38,7 @@ class ZhaConfig(ctypes.Structure):
                 ("p", ctypes.c_float * MAX_LEVELS)]
 
 
-EXPORTS = ["zha_levels_cap", "zha_tree_bytes", "zha_tree_level", "zha_tree_count_offset", "zha_workspace_bytes", "zha_workspace_init", "zha_workspace_stats", "zha_build",
+EXPORTS = ["zha_levels_cap", "zha_tree_bytes", "zha_tree_level", "zha_tree_count_offset", "zha_workspace_bytes", "zha_workspace_init", "zha_workspace_stats", "zha_attend_kernel", "zha_build",
            "zha_extend", "zha_append", "zha_route", "zha_attend", "zha_attend_noalloc", "zha_decode", "zha_dense", "zha_get_status",
            "zha_last_error"]
 
@@ -62,6 +62,7 @@ def lib():
         "zha_workspace_bytes": [C, I32, P],
         "zha_workspace_init": [C, P, SZ, P],
         "zha_workspace_stats": [C, I32, P, P],
+        "zha_attend_kernel": [C, I32, P],
         "zha_build": [C, P, P, P, P, P],
         "zha_extend": [C, P, P, P, P],
         "zha_append": [C, P, P, P, P, P, P, P],
@@ -187,6 +188,16 @@ def workspace_stats_view(cfg: Config, ws: torch.Tensor, n_q: int = 1) -> tuple[t
 
 def alloc_tree(cfg: Config, device="cuda") -> torch.Tensor:
     return torch.zeros(tree_bytes(cfg), dtype=torch.uint8, device=device)
+
+
+ATTEND_KERNELS = ("attend_kernel", "attend_tc_kernel", "attend_prefill_kernel")
+
+
+def attend_kernel(cfg: Config, n_q: int = 1) -> str:
+    """Name of the attention kernel zha_attend runs for this configuration on the current device."""
+    k = ctypes.c_int32()
+    _check(lib().zha_attend_kernel(ctypes.byref(cfg.c()), n_q, ctypes.byref(k)))
+    return ATTEND_KERNELS[k.value]
 
 
 def alloc_workspace(cfg: Config, n_q: int = 1, device="cuda", stream=None) -> torch.Tensor:

@@ -118,6 +118,13 @@ int zha_workspace_init(const zha_config *cfg, void *ws, size_t ws_bytes, zha_str
  * by the last zha_route). */
 int zha_workspace_stats(const zha_config *cfg, int32_t n_q, size_t *rows_offset, size_t *cand_offset);
 
+/* Which attention kernel zha_attend (and zha_decode, zha_attend_noalloc) runs for
+ * cfg and n_q: *kind = 0 for the CUDA-core decode kernel, 1 for the tensor-core
+ * decode kernel (bf16, d = 128, B a multiple of 64, when its shared memory fits
+ * the current device), 2 for the tensor-core prefill kernel (n_q > 1).  Reads the
+ * current device's limits; launches nothing. */
+int zha_attend_kernel(const zha_config *cfg, int32_t n_q, int32_t *kind);
+
 /*
  * zha_build -- build the whole tree over keys [0, N[s]) of every sequence s.
  * [HTI] Tree Construction: each complete block of B keys gets, for its

@@ -199,6 +199,51 @@ def test_short_caches(N):
     assert_status_clean()
 
 
+def test_attend_kernel_selection():
+    """bf16, d = 128 and leaf blocks of whole 64-key tiles run the tensor-core decode kernel;
+    every other decode shape the CUDA-core one; chunks the prefill kernel."""
+    base = dict(d=128, Hq=8, Hkv=2, B=64, b=16, batch=2, N_cap=70144, p=0.95)
+    assert zha.attend_kernel(zha.Config(**base)) == "attend_tc_kernel"
+    assert zha.attend_kernel(zha.Config(**{**base, "B": 256})) == "attend_tc_kernel"
+    assert zha.attend_kernel(zha.Config(**{**base, "Hq": 2})) == "attend_tc_kernel"
+    assert zha.attend_kernel(zha.Config(**{**base, "dtype": "f32"})) == "attend_kernel"
+    assert zha.attend_kernel(zha.Config(**{**base, "d": 64})) == "attend_kernel"
+    assert zha.attend_kernel(zha.Config(**{**base, "B": 16})) == "attend_kernel"
+    assert zha.attend_kernel(zha.Config(**base), n_q=64) == "attend_prefill_kernel"
+
+
+@pytest.mark.parametrize("G", [4, 2])
+def test_nan_past_the_cache_end_never_reaches_the_output(G):
+    """The tensor-core kernel loads whole 64-key tiles, past the cache's end too: rows there hold
+    NaN here, and the output must still equal attention over the index set (scores of rows
+    outside an item are masked by selection, their V rows zeroed before P V)."""
+    d, Hkv, batch = 128, 2, 2
+    Hq = G * Hkv
+    N = [1000 + 17, 640 + 1]
+    N_cap = 1100
+    K, V, Q, qref = planted_inputs("test", batch, Hq, Hkv, d, max(N), N_cap, 4, 1)
+    for s in range(batch):
+        K[s, :, N[s]:] = float("nan")
+        V[s, :, N[s]:] = float("nan")
+    cfg = zha.Config(d=d, Hq=Hq, Hkv=Hkv, B=64, b=16, batch=batch, N_cap=N_cap, p=0.95)
+    assert zha.attend_kernel(cfg) == "attend_tc_kernel"
+    dec = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), N)
+    dec.build()
+    dec.route_attend(Q[0].reshape(batch, 1, Hq, d).contiguous().cuda())
+    sel, cnt, o = dec.results()
+    assert torch.isfinite(o).all()
+    rep = Report()
+    for s in range(batch):
+        for h in range(Hkv):
+            ot = oracle_tree(K[s, h], N[s], cfg, qref[h])
+            hs = range(h * G, (h + 1) * G)
+            check_queries(cfg, ot, K[s, h], V[s, h], N[s] - 1, Q[0, s, h * G:(h + 1) * G],
+                          [sel[s, 0, x].numpy() for x in hs], [int(cnt[s, 0, x]) for x in hs],
+                          [o[s, 0, x].numpy() for x in hs], 0.95, rep)
+    rep.check()
+    assert_status_clean()
+
+
 # ---------------------------------------------------------------- append == rebuild
 
 @pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
