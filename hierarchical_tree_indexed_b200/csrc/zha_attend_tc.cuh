@@ -46,6 +46,7 @@ constexpr uint32_t kTCPBytes = 2 * 16 * 128;                   // P^T: 16 rows x
 constexpr uint32_t kTCOffP = kTCStages * kTCStageBytes;
 constexpr uint32_t kTCOffCtl = kTCOffP + 2 * kTCPBytes;
 constexpr uint32_t kTCTmemCols = 64;                           // S: 2 x 16 columns; O: 16 columns at 32
+constexpr int kTCRegPartials = 8;                              // a merge of at most this many partials runs from registers
 constexpr float kTCRescaleLog2 = 8.0f;                         // lazy rescale: P stays below 2^8 between rescales
 
 struct TcDesc {
@@ -66,6 +67,7 @@ struct TcCtl {
     uint64_t mx[2];                // softmax warps: pair maxima exchanged
     uint64_t ep[3];                // softmax warps: partial sums exchanged / partial stored / merge decided
     uint64_t mg[2];                // softmax warps: a merge's (max, sum) gathered / weights computed
+    uint64_t pre_ready;            // producer -> softmax: prefix[] written
     uint64_t fin;                  // MMA lane: every MMA it issued completed
     TcDesc desc[kTCStages];
     uint32_t tmem;
@@ -74,7 +76,6 @@ struct TcCtl {
     int red[2][4][4];              // [pair parity][warp][head] order-mapped maxima
     float lsum[4][4];              // [warp][head] softmax sums
     float mL[4];                   // [head] a merge's total sum
-    int scan[8];
     int prefix[1];                 // [groups + 1] first global item of each group; then the merge's
                                    // (max, sum) -> (weight, sum) of every partial, float2 [grid][4]
 };
@@ -95,6 +96,13 @@ __device__ __forceinline__ bool twait(uint64_t* bar, uint32_t parity, TcCtl* ctl
     return false;
 }
 __device__ __forceinline__ bool tc_aborted(TcCtl* ctl) { return *reinterpret_cast<volatile int*>(&ctl->abort) != 0; }
+
+// atomicAdd with acquire-release semantics at GPU scope; returns the old value.
+__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
 
 // Order-preserving map of floats (no NaN) to int, for the integer warp max.
 __device__ __forceinline__ int ord_of(float x) {
@@ -117,60 +125,71 @@ __global__ void __launch_bounds__(kTCThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     auto stage = [&](int s) { return base + static_cast<uint32_t>(s) * kTCStageBytes; };
 
-    // ---- prefix[g] = first global item of group g; barriers; TMEM; P^T rows 8..15 stay zero
-    {
-        int carry = 0;
-        for (int b0 = 0; b0 < a.groups; b0 += kTCThreads) {
-            const int g = b0 + tid;
-            const int n = g < a.groups ? a.n_items[g] : 0;
-            int tot;
-            const int x = block_exclusive_scan<kTCThreads / 32>(n, ctl->scan, &tot);
-            if (g < a.groups) ctl->prefix[g] = carry + x;
-            carry += tot;
+    // ---- barriers; TMEM; P^T rows 8..15 stay zero.  The group prefix is the producer's
+    // first job (published through pre_ready), so its first loads go out without a block scan.
+    if (tid == 0) {
+        for (int i = 0; i < kTCStages; ++i) {
+            mbar_init(&ctl->kv_full[i], 1);
+            mbar_init(&ctl->kv_empty[i], 1);
         }
-        if (tid == 0) {
-            ctl->prefix[a.groups] = carry;
-            for (int i = 0; i < kTCStages; ++i) {
-                mbar_init(&ctl->kv_full[i], 1);
-                mbar_init(&ctl->kv_empty[i], 1);
-            }
-            for (int i = 0; i < 2; ++i) {
-                mbar_init(&ctl->s_full[i], 1);
-                mbar_init(&ctl->s_free[i], 128);
-                mbar_init(&ctl->p_full[i], 128);
-                mbar_init(&ctl->o_done[i], 1);
-                mbar_init(&ctl->mx[i], 4);
-            }
-            mbar_init(&ctl->ep[0], 4);
-            mbar_init(&ctl->ep[1], 4);
-            mbar_init(&ctl->ep[2], 1);
-            mbar_init(&ctl->mg[0], 4);
-            mbar_init(&ctl->mg[1], 4);
-            mbar_init(&ctl->fin, 1);
-            fence_mbar_init();
-            ctl->abort = 0;
-            umma::prefetch_tensormap(&tmK);
-            umma::prefetch_tensormap(&tmV);
-            umma::prefetch_tensormap(&tmQ);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl->s_full[i], 1);
+            mbar_init(&ctl->s_free[i], 128);
+            mbar_init(&ctl->p_full[i], 128);
+            mbar_init(&ctl->o_done[i], 1);
+            mbar_init(&ctl->mx[i], 4);
         }
-        for (int x = tid; x < static_cast<int>(2 * kTCPBytes / 16); x += kTCThreads)
-            reinterpret_cast<uint4*>(sP)[x] = make_uint4(0u, 0u, 0u, 0u);
-        if (warp == 5) {
-            umma::tmem_alloc(&ctl->tmem, kTCTmemCols);
-            umma::tmem_relinquish();
-        }
-        umma::fence_proxy_async_smem();
-        umma::fence_before_sync();
-        __syncthreads();
-        umma::fence_after_sync();
+        mbar_init(&ctl->ep[0], 4);
+        mbar_init(&ctl->ep[1], 4);
+        mbar_init(&ctl->ep[2], 1);
+        mbar_init(&ctl->mg[0], 4);
+        mbar_init(&ctl->mg[1], 4);
+        mbar_init(&ctl->pre_ready, 1);
+        mbar_init(&ctl->fin, 1);
+        fence_mbar_init();
+        ctl->abort = 0;
+        umma::prefetch_tensormap(&tmK);
+        umma::prefetch_tensormap(&tmV);
+        umma::prefetch_tensormap(&tmQ);
     }
+    for (int x = tid; x < static_cast<int>(2 * kTCPBytes / 16); x += kTCThreads)
+        reinterpret_cast<uint4*>(sP)[x] = make_uint4(0u, 0u, 0u, 0u);
+    if (warp == 5) {
+        umma::tmem_alloc(&ctl->tmem, kTCTmemCols);
+        umma::tmem_relinquish();
+    }
+    umma::fence_proxy_async_smem();
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
     const uint32_t tmem = ctl->tmem;
-    const int64_t I = ctl->prefix[a.groups];
     const int C = gridDim.x;
-    const int64_t ch = I > 0 ? (I + C - 1) / C : 1;   // items per CTA: one contiguous piece each
 
     if (warp == 4) {
         // ================= TMA producer: this CTA's piece, two items per pair
+        // prefix[g] = first global item of group g: lane l sums a run of groups, a warp scan
+        // places the runs, lane l writes its run's prefixes
+        const int per = (a.groups + 31) / 32;
+        const int r0 = min(a.groups, lane * per), r1 = min(a.groups, r0 + per);
+        int run = 0;
+#pragma unroll 4
+        for (int g = r0; g < r1; ++g) run += a.n_items[g];
+        int incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int acc = incl - run;
+        for (int g = r0; g < r1; ++g) {
+            ctl->prefix[g] = acc;
+            acc += a.n_items[g];
+        }
+        const int64_t I = __shfl_sync(0xffffffffu, incl, 31);
+        if (lane == 0) ctl->prefix[a.groups] = static_cast<int>(I);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->pre_ready);
+        const int64_t ch = I > 0 ? (I + C - 1) / C : 1;   // items per CTA: one contiguous piece each
         int fills = 0;     // pairs posted (lane 0's count is the one used)
         bool ok = true;
         auto acquire = [&](int f) -> bool {
@@ -352,6 +371,9 @@ __global__ void __launch_bounds__(kTCThreads, 1)
             m_ref[h] = -INFINITY;
             l[h] = 0.f;
         }
+        twait(&ctl->pre_ready, 0, ctl);   // the group prefix (first read by an epilogue)
+        const int64_t I = ctl->prefix[a.groups];
+        const int64_t ch = I > 0 ? (I + C - 1) / C : 1;
         uint32_t e = 0, nm = 0;   // epilogues and merges so far
         float2* mbuf = reinterpret_cast<float2*>(reinterpret_cast<unsigned char*>(ctl) + tc_merge_offset(a.groups));
         for (uint32_t g = 0;; ++g) {
@@ -468,13 +490,15 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                     if (i == 0) a.part_ml[pbase + h] = make_float2(m_ref[h], L);
                     a.part_acc[(pbase + h) * D + i] = o[h] + o[4 + h];
                 }
-                __threadfence();
+                // the CTA's stores are ordered before thread 0's count by the barrier; the count's
+                // release publishes them at GPU scope, and its acquire makes the other CTAs'
+                // partials visible to this CTA (through the barrier that follows) when it merges
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ctl->ep[1]);
                 if (i == 0) {
                     twait(&ctl->ep[1], e & 1u, ctl);
                     const int sp = partials_of(ctl->prefix[grp], ctl->prefix[grp + 1], ch, C);
-                    const uint32_t done = atomicAdd(&a.counters[grp], 1u);
+                    const uint32_t done = atomic_add_acq_rel_gpu(&a.counters[grp], 1u);
                     ctl->last_flag = done == static_cast<uint32_t>(sp - 1);
                     ctl->sp = sp;
                     mbar_arrive(&ctl->ep[2]);
@@ -483,13 +507,24 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                 if (ctl->last_flag) {
                     // ---- this CTA closes the group: merge its partials into O.  The (max, sum)
                     // pairs go to shared memory in parallel; warp h turns them into the weights
-                    // 2^(m_k - M_h) and the total sum; thread i then sums dimension i over the
-                    // partials with independent loads.
-                    __threadfence();
+                    // 2^(m_k - M_h) and the total sum; thread i sums dimension i over the
+                    // partials from registers, kTCRegPartials partials per round of loads (the
+                    // first round issued together with the (max, sum) loads).
                     const int sp = ctl->sp;
                     const int s = grp / a.Hkv, kv = grp % a.Hkv;
                     const int64_t pb0 = static_cast<int64_t>(grp) * kSplitMax * G;
                     const int slot0 = static_cast<int>((ctl->prefix[grp] / ch) % C);   // partial k at slot (slot0+k) % C
+                    float xr[kTCRegPartials][G];
+                    auto load_round = [&](int k0) {
+#pragma unroll
+                        for (int k = 0; k < kTCRegPartials; ++k)
+#pragma unroll
+                            for (int h = 0; h < G; ++h)
+                                xr[k][h] = k0 + k < sp
+                                    ? __ldcg(a.part_acc + ((pb0 + static_cast<int64_t>((slot0 + k0 + k) % C) * G + h) * D + i))
+                                    : 0.f;
+                    };
+                    load_round(0);
                     for (int x = i; x < sp * G; x += 128) {
                         const int k = x / G, h = x % G;
                         mbuf[k * 4 + h] = __ldcg(&a.part_ml[pb0 + ((slot0 + k) % C) * G + h]);
@@ -515,24 +550,22 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&ctl->mg[1]);
                     twait(&ctl->mg[1], nm & 1u, ctl);
+                    float o[G];
+#pragma unroll
+                    for (int h = 0; h < G; ++h) o[h] = 0.f;
+                    for (int k0 = 0; k0 < sp; k0 += kTCRegPartials) {
+                        if (k0 > 0) load_round(k0);
+#pragma unroll
+                        for (int k = 0; k < kTCRegPartials; ++k)
+                            if (k0 + k < sp)
+#pragma unroll
+                                for (int h = 0; h < G; ++h) o[h] = fmaf(mbuf[(k0 + k) * 4 + h].x, xr[k][h], o[h]);
+                    }
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
-                        const float* src = a.part_acc + (pb0 + h) * D + i;
-                        auto at_k = [&](int k) { return src + static_cast<int64_t>((slot0 + k) % C) * G * D; };
-                        float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-                        int k = 0;
-                        for (; k + 4 <= sp; k += 4) {
-                            const float x0 = __ldcg(at_k(k)), x1 = __ldcg(at_k(k + 1));
-                            const float x2 = __ldcg(at_k(k + 2)), x3 = __ldcg(at_k(k + 3));
-                            o0 = fmaf(mbuf[k * 4 + h].x, x0, o0);
-                            o1 = fmaf(mbuf[(k + 1) * 4 + h].x, x1, o1);
-                            o2 = fmaf(mbuf[(k + 2) * 4 + h].x, x2, o2);
-                            o3 = fmaf(mbuf[(k + 3) * 4 + h].x, x3, o3);
-                        }
-                        for (; k < sp; ++k) o0 = fmaf(mbuf[k * 4 + h].x, __ldcg(at_k(k)), o0);
                         const float Ls = ctl->mL[h];
                         const int64_t orow = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + h;
-                        a.O[orow * D + i] = Ls > 0.f ? ((o0 + o1) + (o2 + o3)) / Ls : 0.f;
+                        a.O[orow * D + i] = Ls > 0.f ? o[h] / Ls : 0.f;
                     }
                     if (i == 0) a.counters[grp] = 0u;
                     ++nm;
