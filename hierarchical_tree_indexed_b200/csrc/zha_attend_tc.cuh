@@ -97,13 +97,6 @@ __device__ __forceinline__ bool twait(uint64_t* bar, uint32_t parity, TcCtl* ctl
 }
 __device__ __forceinline__ bool tc_aborted(TcCtl* ctl) { return *reinterpret_cast<volatile int*>(&ctl->abort) != 0; }
 
-// atomicAdd with acquire-release semantics at GPU scope; returns the old value.
-__device__ __forceinline__ uint32_t atomic_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
-    uint32_t old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
-}
-
 // Order-preserving map of floats (no NaN) to int, for the integer warp max.
 __device__ __forceinline__ int ord_of(float x) {
     const int i = __float_as_int(x);

@@ -14,6 +14,7 @@ namespace zha {
 
 constexpr int kPlanThreads = 512;
 constexpr int kItemRowsMax = 64;   // rows of one item (and of one attention stage)
+constexpr int kPlanSpec = 4;       // selection entries per thread loaded with the counts
 
 // item: x = first key, y = key count | head mask << 16
 __device__ __forceinline__ int2 make_item(int64_t start, int count, uint32_t mask) {
@@ -35,11 +36,15 @@ struct PlanArgs {
 
 // The gather plan of group g (one (sequence, KV head)), computed by one block of
 // kPlanThreads threads.  bits: shared memory for G * a.words words; scan: kPlanThreads/32+1 ints.
-__device__ void plan_group(const PlanArgs& a, int g, uint32_t* bits, int* scan) {
+// N, Ntree: the sequence's key count and tree count when the caller has them (else < 0).
+__device__ void plan_group(const PlanArgs& a, int g, uint32_t* bits, int* scan, int64_t N = -1, int64_t Ntree = -1) {
     const int s = g / a.Hkv, kv = g % a.Hkv, tid = threadIdx.x;
     const int G = a.G;
     const uint32_t all = (1u << G) - 1u;
-    const int64_t N = a.N[s], Ntree = a.n_tree[s];
+    if (N < 0) {
+        N = a.N[s];
+        Ntree = a.n_tree[s];
+    }
     if (N < 1 || N > a.N_cap || Ntree > N) {
         if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.n_items[g] = 0; a.rows[g] = 0; }
         __syncthreads();
@@ -48,57 +53,66 @@ __device__ void plan_group(const PlanArgs& a, int g, uint32_t* bits, int* scan) 
     const int64_t t = N - 1;
     const int64_t n1 = Ntree / a.B;
     const int64_t words = (n1 + 31) / 32;
-    for (int h = 0; h < G; ++h)
-        for (int i = tid; i < static_cast<int>(words); i += kPlanThreads) bits[h * a.words + i] = 0u;
-    __syncthreads();
-    // every head's selected blocks into its bitmap: counts first, then all entries at once
-    __shared__ int s_cnt[8], s_off[9];
-    if (tid < G) {
-        const int64_t row = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + tid;
-        s_cnt[tid] = min(__ldcg(&a.sel_count[row]), a.sel_cap);
+    // every head's selected blocks into its bitmap: kPlanThreads / G threads per head load
+    // the head's count and their first kPlanSpec entries together (one round trip; entries
+    // past the count are dropped), while the bitmaps are cleared
+    const int tph = kPlanThreads / G, h = tid / tph, r = tid % tph;
+    const int64_t hrow = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + (h < G ? h : 0);
+    const int32_t* hsel = a.sel + hrow * a.sel_cap;
+    int32_t spec[kPlanSpec];
+#pragma unroll
+    for (int k = 0; k < kPlanSpec; ++k) {
+        const int j = r + k * tph;
+        spec[k] = (h < G && j < a.sel_cap) ? __ldcg(&hsel[j]) : -1;
     }
+    const int hcnt = h < G ? min(__ldcg(&a.sel_count[hrow]), a.sel_cap) : 0;
+    for (int hh = 0; hh < G; ++hh)
+        for (int i = tid; i < static_cast<int>(words); i += kPlanThreads) bits[hh * a.words + i] = 0u;
     __syncthreads();
-    if (tid == 0) {
-        s_off[0] = 0;
-        for (int h = 0; h < G; ++h) s_off[h + 1] = s_off[h] + s_cnt[h];
+    uint32_t* hb = bits + (h < G ? h : 0) * a.words;
+#pragma unroll
+    for (int k = 0; k < kPlanSpec; ++k) {
+        const int32_t blk = spec[k];
+        if (r + k * tph < hcnt && blk >= 0 && blk < n1) atomicOr(&hb[blk >> 5], 1u << (blk & 31));
     }
-    __syncthreads();
-    for (int j = tid; j < s_off[G]; j += kPlanThreads) {
-        int h = 0;
-        while (j >= s_off[h + 1]) ++h;
-        const int64_t row = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + h;
-        const int32_t blk = __ldcg(&a.sel[row * a.sel_cap + (j - s_off[h])]);
-        if (blk >= 0 && blk < n1) atomicOr(&bits[h * a.words + (blk >> 5)], 1u << (blk & 31));
+    for (int j = r + kPlanSpec * tph; j < hcnt; j += tph) {
+        const int32_t blk = __ldcg(&hsel[j]);
+        if (blk >= 0 && blk < n1) atomicOr(&hb[blk >> 5], 1u << (blk & 31));
     }
     const int64_t cb = min(t / a.B, n1);   // C_cur = [cb*B, t]
     if (tid < G && cb < n1) atomicOr(&bits[tid * a.words + (cb >> 5)], 1u << (cb & 31));
     __syncthreads();
-    // compaction of the union, ascending: thread owns words [w0, w1)
-    const int64_t per = (words + kPlanThreads - 1) / kPlanThreads;
-    const int64_t w0 = min(words, tid * per), w1 = min(words, w0 + per);
+    // compaction of the union, ascending, in rounds of kPlanThreads words (thread t holds word
+    // r * kPlanThreads + t): a block scan places each word's items, then each warp emits its 32
+    // words one at a time with one lane per bit (a word of a cluster has up to 32 blocks)
     const int nsplit = (a.B + kItemRowsMax - 1) / kItemRowsMax;   // items per block (B > 64)
-    int c = 0;
-    for (int64_t wd = w0; wd < w1; ++wd) {
-        uint32_t o = 0;
-        for (int h = 0; h < G; ++h) o |= bits[h * a.words + wd];
-        c += __popc(o) * nsplit;
-    }
-    int total;
-    int pos = block_exclusive_scan<kPlanThreads / 32>(c, scan, &total);
+    const int lane = tid & 31, wp = tid >> 5;
     int2* out = a.items + static_cast<int64_t>(g) * a.item_cap;
-    for (int64_t wd = w0; wd < w1; ++wd) {
+    int total = 0;
+    for (int64_t r0 = 0; r0 < words; r0 += kPlanThreads) {
+        const int64_t wd = r0 + tid;
         uint32_t o = 0;
-        for (int h = 0; h < G; ++h) o |= bits[h * a.words + wd];
-        while (o) {
-            const int bit = __ffs(o) - 1;
-            o &= o - 1;
-            uint32_t m = 0;
-            for (int h = 0; h < G; ++h) m |= ((bits[h * a.words + wd] >> bit) & 1u) << h;
-            if (nsplit == 1) {
-                out[pos++] = make_item((wd * 32 + bit) * a.B, a.B, m);
-            } else {
-                for (int st = 0; st < a.B; st += kItemRowsMax)
-                    out[pos++] = make_item((wd * 32 + bit) * a.B + st, min(kItemRowsMax, a.B - st), m);
+        if (wd < words)
+            for (int hh = 0; hh < G; ++hh) o |= bits[hh * a.words + wd];
+        int tot;
+        const int pos = total + block_exclusive_scan<kPlanThreads / 32>(__popc(o) * nsplit, scan, &tot);
+        total += tot;
+        for (int j = 0; j < 32; ++j) {
+            const uint32_t oj = __shfl_sync(0xffffffffu, o, j);
+            if (oj == 0u) continue;
+            const int pj = __shfl_sync(0xffffffffu, pos, j);
+            const int64_t wj = r0 + wp * 32 + j;
+            if ((oj >> lane) & 1u) {
+                uint32_t m = 0;
+                for (int hh = 0; hh < G; ++hh) m |= ((bits[hh * a.words + wj] >> lane) & 1u) << hh;
+                const int idx = pj + __popc(oj & ((1u << lane) - 1u)) * nsplit;
+                const int64_t k0 = (wj * 32 + lane) * a.B;
+                if (nsplit == 1) {
+                    out[idx] = make_item(k0, a.B, m);
+                } else {
+                    for (int st = 0, k = 0; st < a.B; st += kItemRowsMax, ++k)
+                        out[idx + k] = make_item(k0 + st, min(kItemRowsMax, a.B - st), m);
+                }
             }
         }
     }
