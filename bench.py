@@ -39,6 +39,7 @@ UNIT = "queries/s"
 FALLBACK_HBM_GBS = 6650.0
 POOL = 64                 # distinct (q, k_new, v_new) sets cycled through by the steps
 E2E_WARMUP = 3            # untimed end-to-end steps before the timed ones
+PHASE_STEPS = 200         # steps of the per-phase breakdown (after the timed one-graph steps)
 ATTEND_SOURCES = ["hierarchical_tree_indexed_b200/csrc/zha_attend.cuh",
                   "hierarchical_tree_indexed_b200/csrc/zha_attend_tc.cuh",
                   "hierarchical_tree_indexed_b200/csrc/zha_umma.cuh",
@@ -79,7 +80,7 @@ def config_dict(w, world: int) -> dict:
             "global_batch": w.batch * world, "seq_len": w.N, "parallelism": f"dp{world}",
             "kv_dtype": w.dtype,
             "l2": L2Flush.NOTE + f"; KV {w.batch * w.Hkv * w.N * w.d * 2 * (2 if w.dtype == 'bf16' else 4) / 2**30:.1f} GiB > L2",
-            "step": "append + route (plan fused) + attend, each phase one CUDA graph"}
+            "step": "append + route (plan fused) + attend as one CUDA graph (phases timed apart, each its own graph)"}
 
 
 class L2Flush:
@@ -271,6 +272,10 @@ class DecodeRun:
             with torch.cuda.graph(g, stream=s):
                 fn()
             self.graphs.append(g)
+        # the whole step as one graph: what a decode loop launches
+        self.g_step = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_step, stream=s):
+            self.append(); self.route(); self.attend()
         self.dense()
         torch.cuda.synchronize()
         self.g_dense = torch.cuda.CUDAGraph()
@@ -304,31 +309,41 @@ class DecodeRun:
             raise RuntimeError(f"device status after {what}: {self.zha.status_names(bits)}")
 
     def timed_steps(self, steps, flush, clocks=None):
-        """Device times of `steps` decode steps (append, route, attend), L2 flushed before each."""
+        """Device times of `steps` decode steps, each the one-graph step (append, route, attend)
+        after an L2 flush; then the phases (each its own graph) over min(steps, PHASE_STEPS) more
+        steps, for the breakdown."""
         import torch
         stream = torch.cuda.current_stream()
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
         rows_acc = torch.zeros((), dtype=torch.float64, device=self.dev)
         cand_acc = torch.zeros((), dtype=torch.float64, device=self.dev)
-        g_app, g_route, g_att = self.graphs
         for k in range(steps):
             self.load(self.step)
             self.step += 1
             flush()
-            e = ev[k]
-            e[0].record(stream)
-            g_app.replay()
-            e[1].record(stream)
-            g_route.replay()
-            e[2].record(stream)
-            g_att.replay()
-            e[3].record(stream)
+            ev[k][0].record(stream)
+            self.g_step.replay()
+            ev[k][1].record(stream)
             rows_acc += self.rows_v.sum()
             cand_acc += self.cand_v.sum()
         torch.cuda.synchronize()
         self.check_status("the timed steps")
-        t = [sum(e[i].elapsed_time(e[i + 1]) for e in ev) / 1e3 for i in range(3)]
-        return dict(t_app=t[0], t_route=t[1], t_att=t[2], t_step=sum(t),
+        t_step = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+        n_ph = min(steps, PHASE_STEPS)
+        pev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_ph)]
+        for k in range(n_ph):
+            self.load(self.step)
+            self.step += 1
+            flush()
+            e = pev[k]
+            e[0].record(stream)
+            for i, g in enumerate(self.graphs):
+                g.replay()
+                e[i + 1].record(stream)
+        torch.cuda.synchronize()
+        self.check_status("the phase steps")
+        t = [sum(e[i].elapsed_time(e[i + 1]) for e in pev) / 1e3 * steps / n_ph for i in range(3)]
+        return dict(t_app=t[0], t_route=t[1], t_att=t[2], t_step=t_step, t_phases=sum(t),
                     rows=rows_acc.item() / steps, cand=cand_acc.item() / steps)
 
     def dense_time(self, reps, flush):
@@ -369,7 +384,7 @@ def sweep(args, rank):
     points = []
     for n in [int(x) for x in args.sweep.split(",")]:
         w = dataclasses.replace(base, N=n, n_clusters=max(1, n // 2048), batch=args.batch or 1)
-        run = DecodeRun(w, dev, n + args.warmup + args.steps + 8, rank)
+        run = DecodeRun(w, dev, n + args.warmup + args.steps + min(args.steps, PHASE_STEPS) + 8, rank)
         for _ in range(args.warmup):
             run.load(run.step); run.step += 1
             for g in run.graphs:
@@ -651,7 +666,7 @@ def main():
     w = workload(args)
     K_steps, W_steps = args.steps, args.warmup
     e2e_steps = 0 if args.no_e2e else min(K_steps, 500)
-    N_cap = w.N + W_steps + K_steps + E2E_WARMUP + e2e_steps + 8
+    N_cap = w.N + W_steps + K_steps + min(K_steps, PHASE_STEPS) + E2E_WARMUP + e2e_steps + 8
     run = DecodeRun(w, dev, N_cap, rank)
     flush = L2Flush(dev)
     for _ in range(W_steps):
