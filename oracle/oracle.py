@@ -46,6 +46,12 @@ def lib():
         L.oracle_index_set.restype = I64
         L.oracle_attend.argtypes = [P, P, P, I32, I32, P, I64, D, P]
         L.oracle_attend.restype = None
+        L.oracle_build_v.argtypes = [P, P, I32, I64, I32, I32, I32, I32, I32, P, D, P, P, P]
+        L.oracle_build_v.restype = None
+        L.oracle_route2.argtypes = [P, I32, I32, I32, I32, I64, I32, P, P, D, P, P, P, P, P, P, P, P, P]
+        L.oracle_route2.restype = I64
+        L.oracle_attend_vsum.argtypes = [P, P, P, I32, I32, P, I64, D, P, P, I64, P]
+        L.oracle_attend_vsum.restype = None
         _lib = L
     return _lib
 
@@ -101,6 +107,7 @@ class Tree:
     khat: np.ndarray   # [total nodes][R][d] float64, level 1 first
     bhat: np.ndarray   # [total nodes][R]
     scale: float
+    vhat: np.ndarray | None = None   # [total nodes][R][d] value summaries, when built with V
 
     @property
     def L(self) -> int:
@@ -112,8 +119,9 @@ class Tree:
 
 
 def build_tree(K_slice, N: int, B: int, b: int, qref_slice, scale: float | None = None,
-               L_fixed: int = 0) -> Tree:
-    """K_slice: [>= N, d] keys of one (sequence, KV head); qref_slice: [>= L][R][d]."""
+               L_fixed: int = 0, V_slice=None) -> Tree:
+    """K_slice: [>= N, d] keys of one (sequence, KV head); qref_slice: [>= L][R][d].
+    With V_slice, the value summaries too (Tree.vhat)."""
     K, dt = _kv_array(K_slice)
     d = K.shape[-1]
     n = levels(N, B, b, L_fixed)
@@ -124,8 +132,15 @@ def build_tree(K_slice, N: int, B: int, b: int, qref_slice, scale: float | None 
     tot = sum(n)
     khat = np.zeros((max(tot, 1), R, d), dtype=np.float64)
     bhat = np.zeros((max(tot, 1), R), dtype=np.float64)
-    lib().oracle_build(_ptr(K), dt, N, d, B, b, R, len(n), _ptr(q), scale, _ptr(khat), _ptr(bhat))
-    return Tree(N, B, b, R, d, n, khat[:tot], bhat[:tot], scale)
+    if V_slice is None:
+        lib().oracle_build(_ptr(K), dt, N, d, B, b, R, len(n), _ptr(q), scale, _ptr(khat), _ptr(bhat))
+        return Tree(N, B, b, R, d, n, khat[:tot], bhat[:tot], scale)
+    V, dv = _kv_array(V_slice)
+    assert dv == dt
+    vhat = np.zeros_like(khat)
+    lib().oracle_build_v(_ptr(K), _ptr(V), dt, N, d, B, b, R, len(n), _ptr(q), scale, _ptr(khat), _ptr(bhat),
+                         _ptr(vhat))
+    return Tree(N, B, b, R, d, n, khat[:tot], bhat[:tot], scale, vhat[:tot])
 
 
 @dataclass
@@ -134,6 +149,9 @@ class Route:
     n_cand: np.ndarray   # per level (level 1 first)
     n_kept: np.ndarray
     margin: np.ndarray
+    pr_node: np.ndarray | None = None    # pruned nodes (global index, level 1 first), their planes
+    pr_plane: np.ndarray | None = None   # and scores, level by level from the top
+    pr_s: np.ndarray | None = None
 
     @property
     def min_margin(self) -> float:
@@ -151,9 +169,16 @@ def route(q, tree: Tree, p) -> Route:
     mg = np.zeros(L, dtype=np.float64)
     kh = tree.khat if tree.khat.size else np.zeros((1, tree.R, tree.d))
     bh = tree.bhat if tree.bhat.size else np.zeros((1, tree.R))
-    cnt = lib().oracle_route(_ptr(qd), tree.d, tree.R, tree.B, tree.b, tree.N, L, _ptr(kh), _ptr(bh),
-                             tree.scale, _ptr(pl), _ptr(sel), _ptr(nc), _ptr(nk), _ptr(mg))
-    return Route(sel[:cnt].copy(), nc, nk, mg)
+    tot = max(sum(tree.n), 1)
+    prn = np.zeros(tot, dtype=np.int64)
+    prp = np.zeros(tot, dtype=np.int32)
+    prs = np.zeros(tot, dtype=np.float64)
+    npr = np.zeros(1, dtype=np.int64)
+    cnt = lib().oracle_route2(_ptr(qd), tree.d, tree.R, tree.B, tree.b, tree.N, L, _ptr(kh), _ptr(bh),
+                              tree.scale, _ptr(pl), _ptr(sel), _ptr(nc), _ptr(nk), _ptr(mg),
+                              _ptr(prn), _ptr(prp), _ptr(prs), _ptr(npr))
+    k = int(npr[0])
+    return Route(sel[:cnt].copy(), nc, nk, mg, prn[:k].copy(), prp[:k].copy(), prs[:k].copy())
 
 
 def index_set(sel, t: int, B: int, n1: int) -> np.ndarray:
@@ -186,3 +211,28 @@ def decode_query(q, tree: Tree, K_slice, V_slice, t: int, p) -> tuple[Route, np.
     r = route(q, tree, p)
     idx = index_set(r.sel, t, tree.B, tree.n[0])
     return r, idx, attend(q, K_slice, V_slice, idx, tree.scale)
+
+
+def attend_vsum(q, K_slice, V_slice, idx, tree: Tree, rt: Route) -> np.ndarray:
+    """Attention over idx plus the pruned nodes of rt as pseudo-keys (score, value summary)."""
+    assert tree.vhat is not None, "the tree was built without V"
+    qd = _f64(q).reshape(-1)
+    K, dt = _kv_array(K_slice)
+    V, dt2 = _kv_array(V_slice)
+    assert dt == dt2
+    d = K.shape[-1]
+    ix = np.ascontiguousarray(np.asarray(idx, dtype=np.int64))
+    prv = np.ascontiguousarray(tree.vhat[rt.pr_node, rt.pr_plane].reshape(-1, d)) if len(rt.pr_node) \
+        else np.zeros((1, d))
+    prs = np.ascontiguousarray(rt.pr_s, dtype=np.float64) if len(rt.pr_s) else np.zeros(1)
+    o = np.zeros(d, dtype=np.float64)
+    lib().oracle_attend_vsum(_ptr(qd), _ptr(K), _ptr(V), dt, d, _ptr(ix), len(ix), tree.scale,
+                             _ptr(prs), _ptr(prv), len(rt.pr_node), _ptr(o))
+    return o
+
+
+def decode_query_vsum(q, tree: Tree, K_slice, V_slice, t: int, p) -> tuple[Route, np.ndarray, np.ndarray]:
+    """decode_query with the pruned subtrees' value summaries: (route, idx, o)."""
+    r = route(q, tree, p)
+    idx = index_set(r.sel, t, tree.B, tree.n[0])
+    return r, idx, attend_vsum(q, K_slice, V_slice, idx, tree, r)

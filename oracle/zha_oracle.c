@@ -91,8 +91,24 @@ int oracle_levels(int64_t N, int B, int b, int L_fixed, int64_t *n, int max_leve
  *   z_c = s_c(qhat), w = softmax(z), khat = sum_c w_c khat_{c,r*(c)}
  *   (r* = the plane attaining the max, lowest r' on ties), bhat = LSE(z) - scale qhat.khat.
  */
+void oracle_build_v(const void *K, const void *V, int dtype, int64_t N, int d, int B, int b, int R, int L,
+                    const double *qref, double scale, double *khat, double *bhat, double *vhat);
+
 void oracle_build(const void *K, int dtype, int64_t N, int d, int B, int b, int R, int L,
                   const double *qref, double scale, double *khat, double *bhat) {
+    oracle_build_v(K, NULL, dtype, N, d, B, b, R, L, qref, scale, khat, bhat, NULL);
+}
+
+/*
+ * The same build, and, when V and vhat are given, the value summaries ([HTI]
+ * Future Directions (4): pruned subtrees contribute coarse attention outputs).
+ * Reading: the value summary is pooled with the weights that pool the key
+ * summary -- vhat_r = Attn(qhat_r, K_C, V_C) = sum_i w_i v_i at a leaf; at an
+ * upper node, sum_c w_c vhat_{c,r*(c)} with the children's weights w_c and best
+ * planes r*(c) of khat.  vhat has the layout of khat: [node][R][d].
+ */
+void oracle_build_v(const void *K, const void *V, int dtype, int64_t N, int d, int B, int b, int R, int L,
+                    const double *qref, double scale, double *khat, double *bhat, double *vhat) {
     int64_t n[64];
     if (oracle_levels(N, B, b, L, n, 64) != L) return;
     double *z = (double *)malloc(sizeof(double) * (size_t)(B > b ? B : b));
@@ -109,6 +125,14 @@ void oracle_build(const void *K, int dtype, int64_t N, int d, int B, int b, int 
             for (int i = 0; i < B; ++i) {
                 double w = exp(z[i] - F);
                 for (int e = 0; e < d; ++e) kh[e] += w * elem(K, dtype, (j * B + i) * d + e);
+            }
+            if (vhat) {
+                double *vh = vhat + (j * R + r) * d;
+                for (int e = 0; e < d; ++e) vh[e] = 0.0;
+                for (int i = 0; i < B; ++i) {
+                    double w = exp(z[i] - F);
+                    for (int e = 0; e < d; ++e) vh[e] += w * elem(V, dtype, (j * B + i) * d + e);
+                }
             }
             bhat[j * R + r] = F - scale * dot(q, kh, d);
         }
@@ -146,6 +170,15 @@ void oracle_build(const void *K, int dtype, int64_t N, int d, int B, int b, int 
                     const double *kc = khat + ((off_child + c) * R + rs[c - c0]) * d;
                     for (int e = 0; e < d; ++e) kh[e] += w * kc[e];
                 }
+                if (vhat) {
+                    double *vh = vhat + ((off + i) * R + r) * d;
+                    for (int e = 0; e < d; ++e) vh[e] = 0.0;
+                    for (int64_t c = c0; c < c1; ++c) {
+                        double w = exp(z[c - c0] - F);
+                        const double *vc = vhat + ((off_child + c) * R + rs[c - c0]) * d;
+                        for (int e = 0; e < d; ++e) vh[e] += w * vc[e];
+                    }
+                }
                 bhat[(off + i) * R + r] = F - scale * dot(q, kh, d);
             }
         }
@@ -157,7 +190,7 @@ void oracle_build(const void *K, int dtype, int64_t N, int d, int B, int b, int 
 }
 
 /* ---- routing ---- */
-typedef struct { double s; int64_t id; } scored_t;
+typedef struct { double s; int64_t id; int plane; } scored_t;
 
 /* descending score; ties go to the lower node id */
 static int cmp_scored(const void *a, const void *b) {
@@ -189,9 +222,30 @@ static int cmp_i64(const void *a, const void *b) {
  * (absent terms = +inf).
  * Returns the count.
  */
+int64_t oracle_route2(const double *q, int d, int R, int B, int b, int64_t N, int L,
+                      const double *khat, const double *bhat, double scale, const double *p,
+                      int64_t *sel, int64_t *n_cand, int64_t *n_kept, double *margin,
+                      int64_t *pr_node, int *pr_plane, double *pr_s, int64_t *n_pr);
+
 int64_t oracle_route(const double *q, int d, int R, int B, int b, int64_t N, int L,
                      const double *khat, const double *bhat, double scale, const double *p,
                      int64_t *sel, int64_t *n_cand, int64_t *n_kept, double *margin) {
+    return oracle_route2(q, d, R, B, b, N, L, khat, bhat, scale, p, sel, n_cand, n_kept, margin,
+                         NULL, NULL, NULL, NULL);
+}
+
+/*
+ * The same routing, and, when pr_node is given, the pruned nodes: at every level
+ * the candidates the cut drops (their subtrees are not searched further), as
+ * global node indices (level 1 first, the layout of khat), each with its score
+ * s and the plane attaining it (lowest plane on ties).  Kept level-1 blocks and
+ * the leaves under pruned nodes partition the tree's blocks.  pr_* need room for
+ * every node of the tree; *n_pr gets the count.
+ */
+int64_t oracle_route2(const double *q, int d, int R, int B, int b, int64_t N, int L,
+                      const double *khat, const double *bhat, double scale, const double *p,
+                      int64_t *sel, int64_t *n_cand, int64_t *n_kept, double *margin,
+                      int64_t *pr_node, int *pr_plane, double *pr_s, int64_t *n_pr) {
     int64_t n[64];
     if (oracle_levels(N, B, b, L, n, 64) != L) return -1;
     int64_t off[64];
@@ -201,6 +255,7 @@ int64_t oracle_route(const double *q, int d, int R, int B, int b, int64_t N, int
 
     int64_t cap = n[0] > n[L - 1] ? n[0] : n[L - 1];
     if (cap < 1) cap = 1;
+    if (pr_node) *n_pr = 0;
     scored_t *cand = (scored_t *)malloc(sizeof(scored_t) * (size_t)cap);
     int64_t *kept = (int64_t *)malloc(sizeof(int64_t) * (size_t)cap);
     int64_t n_keep = 0;
@@ -217,11 +272,13 @@ int64_t oracle_route(const double *q, int d, int R, int B, int b, int64_t N, int
         for (int64_t i = 0; i < nc; ++i) {
             int64_t node = off[l - 1] + cand[i].id;
             double best = -INFINITY;
+            int br = 0;
             for (int r = 0; r < R; ++r) {
                 double t = scale * dot(q, khat + (node * R + r) * d, d) + bhat[node * R + r];
-                if (t > best) best = t;
+                if (t > best) { best = t; br = r; }
             }
             cand[i].s = best;
+            cand[i].plane = br;
         }
         qsort(cand, (size_t)nc, sizeof(scored_t), cmp_scored);
 
@@ -247,6 +304,13 @@ int64_t oracle_route(const double *q, int d, int R, int B, int b, int64_t N, int
         n_cand[l - 1] = nc;
         n_kept[l - 1] = m;
         margin[l - 1] = mg;
+        if (pr_node)
+            for (int64_t i = m; i < nc; ++i) {
+                pr_node[*n_pr] = off[l - 1] + cand[i].id;
+                pr_plane[*n_pr] = cand[i].plane;
+                pr_s[*n_pr] = cand[i].s;
+                ++*n_pr;
+            }
         for (int64_t i = 0; i < m; ++i) kept[i] = cand[i].id;
         qsort(kept, (size_t)m, sizeof(int64_t), cmp_i64);
         n_keep = m;
@@ -292,6 +356,37 @@ void oracle_attend(const double *q, const void *K, const void *V, int dtype, int
     for (int64_t i = 0; i < n_idx; ++i) {
         double w = exp(z[i] - F);
         for (int e = 0; e < d; ++e) o[e] += w * elem(V, dtype, idx[i] * d + e);
+    }
+    free(z);
+}
+
+/*
+ * Attention with the pruned subtrees' value summaries ([HTI] Future Directions
+ * (4)).  Reading: each pruned node n enters the softmax as one pseudo-key with
+ * log-mass s_n (its routing score, the tangent estimate of LSE over its keys) and
+ * value vhat_n (its plane r*): o = (sum_{i in I} e^{z_i} v_i + sum_n e^{s_n} vhat_n)
+ * / (sum_{i in I} e^{z_i} + sum_n e^{s_n}), z_i = scale q.k_i.  Keys of I(q) that
+ * also lie under a pruned node (the sink, a current chunk inside the tree) count in
+ * both terms, as the index set and the summaries define them.
+ * pr_vhat: n_pr rows of d doubles (each pruned node's vhat at its plane).
+ */
+void oracle_attend_vsum(const double *q, const void *K, const void *V, int dtype, int d,
+                        const int64_t *idx, int64_t n_idx, double scale,
+                        const double *pr_s, const double *pr_vhat, int64_t n_pr, double *o) {
+    for (int e = 0; e < d; ++e) o[e] = 0.0;
+    int64_t n = n_idx + n_pr;
+    if (n <= 0) return;
+    double *z = (double *)malloc(sizeof(double) * (size_t)n);
+    for (int64_t i = 0; i < n_idx; ++i) z[i] = scale * dot_slice(q, K, dtype, idx[i], d);
+    for (int64_t j = 0; j < n_pr; ++j) z[n_idx + j] = pr_s[j];
+    double F = lse(z, n);
+    for (int64_t i = 0; i < n_idx; ++i) {
+        double w = exp(z[i] - F);
+        for (int e = 0; e < d; ++e) o[e] += w * elem(V, dtype, idx[i] * d + e);
+    }
+    for (int64_t j = 0; j < n_pr; ++j) {
+        double w = exp(z[n_idx + j] - F);
+        for (int e = 0; e < d; ++e) o[e] += w * pr_vhat[j * d + e];
     }
     free(z);
 }

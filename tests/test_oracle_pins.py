@@ -383,3 +383,97 @@ def test_eq1_decomposition_holds_with_the_actual_mass(which):
     full = O.attend(x, K, V, np.arange(t + 1))
     split = pstar * O.attend(x, K, V, S) + (1 - pstar) * O.attend(x, K, V, Sbar)
     assert np.max(np.abs(full - split)) < 1e-12
+
+
+# ---------------------------------------------------------------- value summaries
+# [HTI] Future Directions (4): pruned subtrees contribute coarse attention outputs.
+# Reading: vhat pools the values with the weights that pool khat; a pruned node enters the
+# softmax as one pseudo-key of log-mass s (its routing score) and value vhat.
+
+def test_value_summary_of_a_uniform_block_is_its_mean_value():
+    """A leaf whose keys are all equal gives every key the same weight: vhat is the plain
+    mean of the block's values; a block of one key summarises to that key's value."""
+    d, B, b = 8, 4, 4
+    r = rng(900)
+    k = r.standard_normal(d).astype(np.float32)
+    K = np.tile(k, (B * 2, 1))
+    V = r.standard_normal((B * 2, d)).astype(np.float32)
+    tree = O.build_tree(K, B * 2, B, b, r.standard_normal((4, 1, d)), V_slice=V)
+    for j in range(2):
+        assert np.max(np.abs(tree.vhat[j, 0] - V[j * B:(j + 1) * B].astype(np.float64).mean(0))) < 1e-14
+    K1 = r.standard_normal((5, d)).astype(np.float32)
+    V1 = r.standard_normal((5, d)).astype(np.float32)
+    t1 = O.build_tree(K1, 5, 1, 2, r.standard_normal((8, 1, d)), V_slice=V1)
+    assert np.max(np.abs(t1.vhat[:5, 0] - V1.astype(np.float64))) == 0.0
+
+
+@pytest.mark.parametrize("seed,p", [(0, 0.5), (1, 0.8), (2, 0.95), (3, 0.3)])
+def test_kept_blocks_and_pruned_subtrees_partition_the_tree(seed, p):
+    d, B, b, N = 8, 4, 4, 4 * 4 * 4 * 5 + 2
+    r = rng(910 + seed)
+    K = (r.standard_normal((N, d)) * 2).astype(np.float32)
+    V = r.standard_normal((N, d)).astype(np.float32)
+    tree = O.build_tree(K, N, B, b, r.standard_normal((4, 1, d)), V_slice=V)
+    rt = O.route(r.standard_normal(d) * 2, tree, p)
+    offs = np.cumsum([0] + tree.n)
+    cover = np.zeros(tree.n[0], dtype=int)
+    cover[rt.sel] += 1
+    for node in rt.pr_node:
+        lvl = int(np.searchsorted(offs, node, side="right"))   # 1-based level
+        i = int(node - offs[lvl - 1])
+        span = b ** (lvl - 1)
+        cover[i * span:min((i + 1) * span, tree.n[0])] += 1
+    assert (cover == 1).all()
+
+
+@pytest.mark.parametrize("p", [0.3, 0.6, 0.9])
+def test_summaries_are_exact_when_every_top_node_holds_one_key(p):
+    """Keys equal under each top-level node make every tangent exact (a node's log-mass is
+    scale q.k + log(count), its vhat the mean of its values): attention over I(q) plus the
+    pruned nodes then equals dense causal attention for any p, while I(q) alone does not.
+    The query favours the sink's node, so key 0 is never also counted inside a pruned node."""
+    d, B, b = 8, 4, 4
+    r = rng(920)
+    n_top, per_top = 3, B * b * b           # three level-3 nodes of 64 keys
+    N = n_top * per_top + 3                 # C_cur = the last 3 keys, past the tree
+    tops = r.standard_normal((n_top, d))
+    K = np.concatenate([np.repeat(tops, per_top, axis=0), r.standard_normal((3, d))]).astype(np.float32)
+    V = r.standard_normal((N, d)).astype(np.float32)
+    tree = O.build_tree(K, N, B, b, r.standard_normal((4, 1, d)), V_slice=V)
+    assert tree.L == 3
+    q = 0.6 * tops[0] / np.linalg.norm(tops[0]) * math.sqrt(d) + 0.1 * r.standard_normal(d)
+    rt, idx, o = O.decode_query_vsum(q, tree, K, V, N - 1, p)
+    assert 0 in rt.sel and len(rt.pr_node) > 0
+    dense = O.attend(q, K, V, np.arange(N))
+    assert np.max(np.abs(o - dense)) < 1e-12
+    assert np.max(np.abs(O.attend(q, K, V, idx) - dense)) > 1e-4
+
+
+def test_summaries_vanish_at_p_one():
+    d, B, b, N = 8, 4, 4, 150
+    r = rng(930)
+    K = r.standard_normal((N, d)).astype(np.float32)
+    V = r.standard_normal((N, d)).astype(np.float32)
+    tree = O.build_tree(K, N, B, b, r.standard_normal((4, 1, d)), V_slice=V)
+    q = r.standard_normal(d)
+    rt, idx, o = O.decode_query_vsum(q, tree, K, V, N - 1, 1.0)
+    assert len(rt.pr_node) == 0
+    assert np.max(np.abs(o - O.attend(q, K, V, idx))) == 0.0
+
+
+@pytest.mark.parametrize("R", [1, 2])
+def test_value_summaries_pool_with_the_key_summaries_weights(R):
+    """With values a linear map of the keys (V = K M), pooling V with khat's weights (and the
+    children's best planes) gives vhat = khat M at every level and plane; any other weights
+    (uniform, another plane) break it."""
+    d, B, b, N = 8, 4, 4, 4 * 4 * 4 * 3 + 6
+    r = rng(940 + R)
+    K = (r.standard_normal((N, d)) * 1.5).astype(np.float64)
+    M = r.standard_normal((d, d))
+    tree = O.build_tree(K.astype(np.float32), N, B, b, r.standard_normal((4, R, d)),
+                        V_slice=(K.astype(np.float32).astype(np.float64) @ M).astype(np.float32))
+    # the oracle widens V from fp32: compare against khat of the same fp32 keys, mapped by M,
+    # to the rounding of V to fp32
+    Vf = (K.astype(np.float32).astype(np.float64) @ M).astype(np.float32).astype(np.float64)
+    err_v = np.abs(Vf - K.astype(np.float32).astype(np.float64) @ M).max()
+    assert np.max(np.abs(tree.vhat - tree.khat @ M)) < 4 * err_v + 1e-12
