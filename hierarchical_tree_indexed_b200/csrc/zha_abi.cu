@@ -52,15 +52,15 @@ int fail(int code, const char* fmt, ...) {
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct TreeLayout {
-    int Lcap, R;
+    int Lcap, R, vsum;
     int64_t ncap[kMaxLevels];
-    size_t off_ntree, off_qref, off_khat[kMaxLevels], off_bhat[kMaxLevels], total;
+    size_t off_ntree, off_qref, off_khat[kMaxLevels], off_bhat[kMaxLevels], off_vhat[kMaxLevels], total;
 };
 
 struct WsLayout {
     int64_t cand_cap, par_cap, kb_cap, sel_cap, item_cap, words;
     size_t off_scores, off_parents, off_sel, off_count, off_items, off_nitems, off_ml, off_acc, off_counters;
-    size_t off_rows, off_cand, off_ballot, off_grp;
+    size_t off_rows, off_cand, off_ballot, off_grp, off_pr_ml, off_pr_acc;
     size_t total;
 };
 
@@ -81,6 +81,8 @@ int validate(const zha_config* c) {
     if (c->batch < 1) return fail(ZHA_ERR_INVALID_ARG, "batch=%d", c->batch);
     if (c->N_cap < 1 || c->N_cap > (int64_t{1} << 31) - 128) return fail(ZHA_ERR_INVALID_ARG, "N_cap=%lld", (long long)c->N_cap);
     if (c->L_fixed < 0 || c->L_fixed > ZHA_MAX_LEVELS) return fail(ZHA_ERR_INVALID_ARG, "L_fixed=%d", c->L_fixed);
+    if (c->vsum != 0 && c->vsum != 1) return fail(ZHA_ERR_INVALID_ARG, "vsum=%d must be 0 or 1", c->vsum);
+    if (c->vsum && c->R != 1) return fail(ZHA_ERR_UNSUPPORTED, "vsum=1: value summaries take R = 1 (R=%d)", c->R);
     if (!(c->scale >= 0.f) || !std::isfinite(c->scale)) return fail(ZHA_ERR_INVALID_ARG, "scale must be finite and >= 0");
     int64_t n[kMaxLevels];
     const int L = tree_levels(c->N_cap, c->B, c->b, c->L_fixed, n);
@@ -97,6 +99,7 @@ int tree_layout(const zha_config* c, TreeLayout* t) {
     int64_t n[kMaxLevels];
     t->Lcap = tree_levels(c->N_cap, c->B, c->b, c->L_fixed, n);
     t->R = c->R;
+    t->vsum = c->vsum;
     const int64_t slices = static_cast<int64_t>(c->batch) * c->Hkv;
     size_t off = 0;
     t->off_ntree = off;
@@ -109,6 +112,8 @@ int tree_layout(const zha_config* c, TreeLayout* t) {
         off = align256(off + sizeof(float) * static_cast<size_t>(slices) * t->ncap[l] * c->R * c->d);
         t->off_bhat[l] = off;
         off = align256(off + sizeof(float) * static_cast<size_t>(slices) * t->ncap[l] * c->R);
+        t->off_vhat[l] = off;
+        if (c->vsum) off = align256(off + sizeof(float) * static_cast<size_t>(slices) * t->ncap[l] * c->d);
     }
     t->total = off;
     return ZHA_OK;
@@ -122,6 +127,7 @@ TreeDev tree_view(const TreeLayout& t, void* tree) {
     for (int l = 0; l < kMaxLevels; ++l) {
         v.khat[l] = reinterpret_cast<float*>(base + t.off_khat[l]);
         v.bhat[l] = reinterpret_cast<float*>(base + t.off_bhat[l]);
+        v.vhat[l] = t.vsum && t.ncap[l] > 0 ? reinterpret_cast<float*>(base + t.off_vhat[l]) : nullptr;
         v.ncap[l] = t.ncap[l];
     }
     v.Lcap = t.Lcap;
@@ -162,6 +168,8 @@ int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
     w->off_rows = off;     off = align256(off + sizeof(int32_t) * groups);
     w->off_cand = off;     off = align256(off + sizeof(int32_t) * ctas);
     w->off_ballot = off;   off = align256(off + sizeof(uint32_t) * ctas * 2 * w->kb_cap);
+    w->off_pr_ml = off;    off = align256(off + (c->vsum ? sizeof(float2) * ctas : 0));
+    w->off_pr_acc = off;   off = align256(off + (c->vsum ? sizeof(float) * ctas * c->d : 0));
     w->total = off;
     if (static_cast<size_t>(G) * w->words * 4 > 200 * 1024)
         return fail(ZHA_ERR_UNSUPPORTED, "N_cap too large for the on-chip union bitmap");
@@ -224,11 +232,12 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // ---------------------------------------------------------------- build / append
 template <typename T, int D>
-int run_build(const zha_config* c, const TreeLayout& lay, const void* K, const int32_t* N, void* tree,
+int run_build(const zha_config* c, const TreeLayout& lay, const void* K, const void* V, const int32_t* N, void* tree,
               cudaStream_t st) {
     BuildArgs a{};
     a.tree = tree_view(lay, tree);
     a.K = K;
+    a.V = V;
     a.N = N;
     a.batch = c->batch; a.Hkv = c->Hkv; a.B = c->B; a.b = c->b; a.L_fixed = c->L_fixed;
     a.N_cap = c->N_cap;
@@ -247,11 +256,12 @@ int run_build(const zha_config* c, const TreeLayout& lay, const void* K, const i
 
 // Extension: leaves and ancestors that change, then the new count (the kernels read the old one).
 template <typename T, int D>
-int run_extend(const zha_config* c, const TreeLayout& lay, const void* K, const int32_t* N, void* tree,
+int run_extend(const zha_config* c, const TreeLayout& lay, const void* K, const void* V, const int32_t* N, void* tree,
                cudaStream_t st) {
     BuildArgs a{};
     a.tree = tree_view(lay, tree);
     a.K = K;
+    a.V = V;
     a.N = N;
     a.batch = c->batch; a.Hkv = c->Hkv; a.B = c->B; a.b = c->b; a.L_fixed = c->L_fixed;
     a.incremental = 1;
@@ -288,7 +298,8 @@ bool plan_fits_route(const zha_config* c, const WsLayout& wl);
 
 template <typename T, int D, int NVR>
 int run_route_t(const RouteArgs& a, int ctas, cudaStream_t st) {
-    auto kern = a.tree.R > 1 ? route_decode_kernel<T, D, NVR, true> : route_decode_kernel<T, D, NVR, false>;
+    auto kern = a.tree.R > 1 ? route_decode_kernel<T, D, NVR, true>
+                : a.pr_ml ? route_decode_kernel<T, D, NVR, false, true> : route_decode_kernel<T, D, NVR, false>;
     ZHA_TRY(allow_smem(kern, sizeof(RouteSmem)));
     kern<<<ctas, kRouteThreads, sizeof(RouteSmem), st>>>(a);
     return check_launch("route");
@@ -311,6 +322,8 @@ int run_route(const zha_config* c, const TreeLayout& lay, const WsLayout& wl, co
     for (int l = 0; l < kMaxLevels; ++l) a.p[l] = c->p[l];
     a.plan = plan_args(c, wl, lay, tree, N, sel, cnt, sel_cap, ws);
     a.grp_done = at<uint32_t>(ws, wl.off_grp);
+    a.pr_ml = c->vsum ? at<float2>(ws, wl.off_pr_ml) : nullptr;
+    a.pr_acc = c->vsum ? at<float>(ws, wl.off_pr_acc) : nullptr;
     a.fuse_plan = fuse ? 1 : 0;
     const int ctas = c->batch * c->Hq;
     if (c->b <= 4) return run_route_t<T, D, 4>(a, ctas, st);
@@ -374,6 +387,8 @@ int run_attend(const zha_config* c, const WsLayout& wl, const void* K, const voi
     a.part_ml = at<float2>(ws, wl.off_ml);
     a.part_acc = at<float>(ws, wl.off_acc);
     a.counters = at<uint32_t>(ws, wl.off_counters);
+    a.pr_ml = c->vsum ? at<float2>(ws, wl.off_pr_ml) : nullptr;
+    a.pr_acc = c->vsum ? at<float>(ws, wl.off_pr_acc) : nullptr;
     a.item_cap = wl.item_cap; a.N_cap = c->N_cap;
     a.groups = c->batch * c->Hkv; a.Hq = c->Hq; a.Hkv = c->Hkv; a.n_q = 1;
     a.qscale = scale_of(c) * 1.4426950408889634f;
@@ -433,6 +448,7 @@ struct PfLayout {
 
 int pf_layout(const zha_config* c, int n_q, const TreeLayout& t, PfLayout* p) {
     if (n_q < 2) return fail(ZHA_ERR_INVALID_ARG, "n_q=%d", n_q);
+    if (c->vsum) return fail(ZHA_ERR_UNSUPPORTED, "n_q=%d: chunked prefill does not take value summaries (vsum = 1)", n_q);
     if (c->dtype != ZHA_BF16) return fail(ZHA_ERR_UNSUPPORTED, "n_q=%d: chunked prefill takes bf16 K, V and Q", n_q);
     if (c->B != 64) return fail(ZHA_ERR_UNSUPPORTED, "n_q=%d: chunked prefill needs leaf blocks of B = 64 keys", n_q);
     const int G = c->Hq / c->Hkv;
@@ -738,6 +754,16 @@ int zha_tree_level(const zha_config* cfg, int32_t level, size_t* khat_offset, si
     return ZHA_OK;
 }
 
+int zha_tree_level_v(const zha_config* cfg, int32_t level, size_t* vhat_offset) {
+    TreeLayout t;
+    ZHA_TRY(need(vhat_offset, "vhat_offset"));
+    ZHA_TRY(tree_layout(cfg, &t));
+    if (!cfg->vsum) return fail(ZHA_ERR_INVALID_ARG, "the tree holds no value summaries (vsum = 0)");
+    if (level < 1 || level > t.Lcap) return fail(ZHA_ERR_INVALID_ARG, "level=%d outside 1..%d", level, t.Lcap);
+    *vhat_offset = t.off_vhat[level - 1];
+    return ZHA_OK;
+}
+
 int zha_tree_count_offset(const zha_config* cfg, size_t* offset) {
     TreeLayout t;
     ZHA_TRY(need(offset, "offset"));
@@ -809,26 +835,29 @@ int zha_workspace_init(const zha_config* cfg, void* ws, size_t ws_bytes, zha_str
     return ZHA_OK;
 }
 
-int zha_build(const zha_config* cfg, const void* K, const float* Qref, const int32_t* N, void* tree,
+int zha_build(const zha_config* cfg, const void* K, const void* V, const float* Qref, const int32_t* N, void* tree,
               zha_stream_t stream) {
     TreeLayout t;
     ZHA_TRY(tree_layout(cfg, &t));
     ZHA_TRY(need(K, "K"));
+    if (cfg->vsum) ZHA_TRY(need(V, "V (vsum = 1)"));
     ZHA_TRY(need(Qref, "Qref"));
     ZHA_TRY(need(N, "N"));
     ZHA_TRY(need(tree, "tree"));
     const size_t qbytes = sizeof(float) * static_cast<size_t>(cfg->Hkv) * t.Lcap * cfg->R * cfg->d;
     ZHA_CUDA(cudaMemcpyAsync(static_cast<char*>(tree) + t.off_qref, Qref, qbytes, cudaMemcpyDeviceToDevice, stream));
-    return ZHA_DISPATCH(cfg, run_build, cfg, t, K, N, tree, stream);
+    return ZHA_DISPATCH(cfg, run_build, cfg, t, K, V, N, tree, stream);
 }
 
-int zha_extend(const zha_config* cfg, const void* K, const int32_t* N, void* tree, zha_stream_t stream) {
+int zha_extend(const zha_config* cfg, const void* K, const void* V, const int32_t* N, void* tree,
+               zha_stream_t stream) {
     TreeLayout t;
     ZHA_TRY(tree_layout(cfg, &t));
     ZHA_TRY(need(K, "K"));
+    if (cfg->vsum) ZHA_TRY(need(V, "V (vsum = 1)"));
     ZHA_TRY(need(N, "N"));
     ZHA_TRY(need(tree, "tree"));
-    return ZHA_DISPATCH(cfg, run_extend, cfg, t, K, N, tree, stream);
+    return ZHA_DISPATCH(cfg, run_extend, cfg, t, K, V, N, tree, stream);
 }
 
 int zha_append(const zha_config* cfg, void* K, void* V, const void* k_new, const void* v_new, int32_t* N,
@@ -913,6 +942,8 @@ int zha_attend(const zha_config* cfg, const void* K, const void* V, const void* 
 int zha_attend_noalloc(const zha_config* cfg, const void* K, const void* V, const void* tree, const void* Q,
                        int32_t n_q, const int32_t* N, const int32_t* sel, const int32_t* sel_count, int32_t sel_cap,
                        float* O, zha_stream_t stream) {
+    if (cfg && cfg->vsum)
+        return fail(ZHA_ERR_UNSUPPORTED, "zha_attend_noalloc: value summaries need the router's workspace (vsum = 1)");
     TreeLayout t;
     WsLayout w;
     ZHA_TRY(tree_layout(cfg, &t));

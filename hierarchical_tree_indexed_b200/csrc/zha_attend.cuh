@@ -60,6 +60,8 @@ struct AttendArgs {
     float2* part_ml;           // [groups][kSplitMax][G]  (max in log2 units, sum)
     float* part_acc;           // [groups][kSplitMax][G][d]
     uint32_t* counters;        // [groups] partials done, zero between calls
+    const float2* pr_ml;       // value summaries: per query row (log2 max, sum) and [d] value sum of
+    const float* pr_acc;       //   the nodes routing dropped, one more partial in the merge; else null
     int64_t item_cap, N_cap;
     int groups, Hq, Hkv, n_q;
     float qscale;              // scale * log2(e)
@@ -537,9 +539,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
                 }
                 consumer_sync();
                 if (w < G) {   // warp h: M_h, the weights, L_h
+                    // value summaries: the dropped nodes' partial of this head's query joins the merge
+                    const float2 pr = a.pr_ml ? a.pr_ml[(static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + w]
+                                              : make_float2(-INFINITY, 0.f);
                     float M = -INFINITY;
                     for (int k = lane; k < sp; k += 32) M = fmaxf(M, fw[k * G + w]);
-                    M = warp_max(M);
+                    M = fmaxf(warp_max(M), pr.x);
                     float Ls = 0.f;
                     for (int k = lane; k < sp; k += 32) {
                         const float f = M == -INFINITY ? 0.f : exp2f(fw[k * G + w] - M);
@@ -547,7 +552,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
                         Ls += f * fl[k * G + w];
                     }
                     Ls = warp_sum(Ls);
-                    if (lane == 0) sm.cl[0][w] = Ls;
+                    const float fpr = (M == -INFINITY || pr.x == -INFINITY) ? 0.f : exp2f(pr.x - M);
+                    if (lane == 0) {
+                        sm.cl[0][w] = fmaf(fpr, pr.y, Ls);
+                        sm.cm[0][w] = fpr;
+                    }
                 }
                 consumer_sync();
                 for (int x = ct; x < G * D; x += kAttConsumers * 32) {
@@ -569,6 +578,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
                     for (; k < sp; ++k) o0 = fmaf(fw[k * G + h], __ldcg(at_k(k)), o0);
                     const float Ls = sm.cl[0][h];
                     const int64_t orow = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + h;
+                    if (a.pr_acc) o0 = fmaf(sm.cm[0][h], a.pr_acc[orow * D + e], o0);
                     a.O[orow * D + e] = Ls > 0.f ? ((o0 + o1) + (o2 + o3)) / Ls : 0.f;
                 }
                 if (ct == 0) a.counters[g] = 0u;

@@ -76,6 +76,7 @@ struct TcCtl {
     int red[2][4][4];              // [pair parity][warp][head] order-mapped maxima
     float lsum[4][4];              // [warp][head] softmax sums
     float mL[4];                   // [head] a merge's total sum
+    float mPr[4];                  // [head] a merge's weight of the dropped nodes' partial (value summaries)
     int prefix[1];                 // [groups + 1] first global item of each group; then the merge's
                                    // (max, sum) -> (weight, sum) of every partial, float2 [grid][4]
 };
@@ -527,9 +528,12 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                     twait(&ctl->mg[0], nm & 1u, ctl);
                     if (warp < G) {
                         const int h = warp;
+                        // value summaries: the dropped nodes' partial of this head's query joins the merge
+                        const float2 pr = a.pr_ml ? a.pr_ml[(static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + h]
+                                                  : make_float2(-INFINITY, 0.f);
                         float M = -INFINITY;
                         for (int k = lane; k < sp; k += 32) M = fmaxf(M, mbuf[k * 4 + h].x);
-                        M = warp_max(M);
+                        M = fmaxf(warp_max(M), pr.x);
                         float Ls = 0.f;
                         for (int k = lane; k < sp; k += 32) {
                             const float2 ml = mbuf[k * 4 + h];
@@ -538,7 +542,11 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                             Ls = fmaf(f, ml.y, Ls);
                         }
                         Ls = warp_sum(Ls);
-                        if (lane == 0) ctl->mL[h] = Ls;
+                        const float fpr = (M == -INFINITY || pr.x == -INFINITY) ? 0.f : exp2f(pr.x - M);
+                        if (lane == 0) {
+                            ctl->mL[h] = fmaf(fpr, pr.y, Ls);
+                            ctl->mPr[h] = fpr;
+                        }
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&ctl->mg[1]);
@@ -558,6 +566,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                     for (int h = 0; h < G; ++h) {
                         const float Ls = ctl->mL[h];
                         const int64_t orow = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + h;
+                        if (a.pr_acc) o[h] = fmaf(ctl->mPr[h], a.pr_acc[orow * D + i], o[h]);
                         a.O[orow * D + i] = Ls > 0.f ? o[h] / Ls : 0.f;
                     }
                     if (i == 0) a.counters[grp] = 0u;

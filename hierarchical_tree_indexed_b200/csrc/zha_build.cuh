@@ -23,11 +23,13 @@
 namespace zha {
 
 // One warp: summary of `count` rows (row stride D elements of T, 16-byte aligned),
-// optional per-row bias (nullptr = 0), reference query q (fp32 [D]).
-template <typename T, int D>
+// optional per-row bias (nullptr = 0), reference query q (fp32 [D]).  WV: the value
+// rows vrows (same layout) are pooled with the same weights into vhat_out.
+template <typename T, int D, bool WV = false>
 __device__ void summarize_rows(const T* __restrict__ rows, const float* __restrict__ bias, int count,
                                const float* __restrict__ q, float scale, float* __restrict__ khat_out,
-                               float* __restrict__ bhat_out) {
+                               float* __restrict__ bhat_out, const T* __restrict__ vrows = nullptr,
+                               float* __restrict__ vhat_out = nullptr) {
     constexpr int VEC = Elem<T>::kVec;   // elements per 16-byte load
     constexpr int LPR = D / VEC;         // lanes per row
     constexpr int RPW = 32 / LPR;        // rows per warp-wide load
@@ -40,20 +42,27 @@ __device__ void summarize_rows(const T* __restrict__ rows, const float* __restri
 #pragma unroll
     for (int e = 0; e < VEC; ++e) qv[e] = q[li * VEC + e] * scale;
 
-    float m = -INFINITY, l = 0.f, acc[VEC];
+    float m = -INFINITY, l = 0.f, acc[VEC], accv[WV ? VEC : 1];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int e = 0; e < (WV ? VEC : 1); ++e) accv[e] = 0.f;
 
     for (int base = 0; base < count; base += RPW * U) {
-        float x[U][VEC], z[U];
+        float x[U][VEC], xv[U][WV ? VEC : 1], z[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int row = base + u * RPW + sub;
             if (row < count) {
                 Elem<T>::load16(rows + static_cast<int64_t>(row) * D + li * VEC, x[u]);
+                if constexpr (WV) Elem<T>::load16(vrows + static_cast<int64_t>(row) * D + li * VEC, xv[u]);
             } else {
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) x[u][e] = 0.f;
+                if constexpr (WV) {
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) xv[u][e] = 0.f;
+                }
             }
         }
 #pragma unroll
@@ -94,6 +103,15 @@ __device__ void summarize_rows(const T* __restrict__ rows, const float* __restri
             for (int u = 0; u < U; ++u) a = fmaf(w[u], x[u][e], a);
             acc[e] = a;
         }
+        if constexpr (WV) {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                float a = accv[e] * alpha;
+#pragma unroll
+                for (int u = 0; u < U; ++u) a = fmaf(w[u], xv[u][e], a);
+                accv[e] = a;
+            }
+        }
         m = mn;
     }
 #pragma unroll
@@ -101,6 +119,18 @@ __device__ void summarize_rows(const T* __restrict__ rows, const float* __restri
 #pragma unroll
         for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
     const float inv = 1.f / l;
+    if constexpr (WV) {
+#pragma unroll
+        for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) accv[e] += __shfl_xor_sync(0xffffffffu, accv[e], o);
+        if (sub == 0) {
+#pragma unroll
+            for (int e = 0; e < VEC; e += 4)
+                *reinterpret_cast<float4*>(vhat_out + li * VEC + e) =
+                    make_float4(accv[e] * inv, accv[e + 1] * inv, accv[e + 2] * inv, accv[e + 3] * inv);
+        }
+    }
     float pd = 0.f;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
@@ -170,6 +200,7 @@ __device__ void summarize_children_planes(const float* __restrict__ kh, const fl
 struct BuildArgs {
     TreeDev tree;
     const void* K;      // [batch][Hkv][N_cap][d]
+    const void* V;      // the same layout; read when the tree holds value summaries
     const int32_t* N;   // [batch]
     int batch, Hkv, B, b, L_fixed;
     int incremental;    // 1: the tree already indexes tree.n_tree[s] keys; summarise only what changes
@@ -214,7 +245,13 @@ __global__ void __launch_bounds__(256) build_leaf_kernel(BuildArgs a) {
     const float* q = a.tree.qref + (static_cast<int64_t>(h) * a.tree.Lcap * R + pl) * D;
     float* kh = a.tree.khat[0] + ((slice * n1cap + j) * R + pl) * D;
     float* bh = a.tree.bhat[0] + (slice * n1cap + j) * R + pl;
-    summarize_rows<T, D>(rows, nullptr, a.B, q, a.scale, kh, bh);
+    if (a.tree.vhat[0]) {   // value summaries: R = 1
+        const T* vrows = static_cast<const T*>(a.V) + (slice * a.N_cap + j * a.B) * D;
+        summarize_rows<T, D, true>(rows, nullptr, a.B, q, a.scale, kh, bh, vrows,
+                                   a.tree.vhat[0] + (slice * n1cap + j) * D);
+    } else {
+        summarize_rows<T, D>(rows, nullptr, a.B, q, a.scale, kh, bh);
+    }
 }
 
 // Level l >= 2: one warp per (sequence, KV head, node) over its children at l-1.
@@ -230,7 +267,10 @@ __device__ __forceinline__ void summarize_node(const TreeDev& t, int64_t slice, 
     const float* q = t.qref + ((static_cast<int64_t>(h) * t.Lcap + (l - 1)) * R + pl) * D;
     float* kh = t.khat[l - 1] + ((slice * t.ncap[l - 1] + i) * R + pl) * D;
     float* bh = t.bhat[l - 1] + (slice * t.ncap[l - 1] + i) * R + pl;
-    if (R == 1) summarize_rows<float, D>(rows, bias, cnt, q, scale, kh, bh);
+    if (R == 1 && t.vhat[l - 1])
+        summarize_rows<float, D, true>(rows, bias, cnt, q, scale, kh, bh, t.vhat[l - 2] + (slice * cc + c0) * D,
+                                       t.vhat[l - 1] + (slice * t.ncap[l - 1] + i) * D);
+    else if (R == 1) summarize_rows<float, D>(rows, bias, cnt, q, scale, kh, bh);
     else summarize_children_planes<D>(rows, bias, cnt, R, q, scale, kh, bh);
 }
 
@@ -318,9 +358,14 @@ __global__ void append_kernel(AppendArgs a) {
             const T* rows = static_cast<const T*>(a.K) + (slice * a.N_cap + j * a.B) * D;
             for (int pl = 0; pl < R; ++pl) {
                 const float* q = a.tree.qref + (static_cast<int64_t>(h) * a.tree.Lcap * R + pl) * D;
-                summarize_rows<T, D>(rows, nullptr, a.B, q, a.scale,
-                                     a.tree.khat[0] + ((slice * a.tree.ncap[0] + j) * R + pl) * D,
-                                     a.tree.bhat[0] + (slice * a.tree.ncap[0] + j) * R + pl);
+                float* kh = a.tree.khat[0] + ((slice * a.tree.ncap[0] + j) * R + pl) * D;
+                float* bh = a.tree.bhat[0] + (slice * a.tree.ncap[0] + j) * R + pl;
+                if (a.tree.vhat[0])   // value summaries: R = 1
+                    summarize_rows<T, D, true>(rows, nullptr, a.B, q, a.scale, kh, bh,
+                                               static_cast<const T*>(a.V) + (slice * a.N_cap + j * a.B) * D,
+                                               a.tree.vhat[0] + (slice * a.tree.ncap[0] + j) * D);
+                else
+                    summarize_rows<T, D>(rows, nullptr, a.B, q, a.scale, kh, bh);
             }
             int64_t n0[kMaxLevels], n1[kMaxLevels];
             const int L0 = tree_levels(N, a.B, a.b, a.L_fixed, n0);

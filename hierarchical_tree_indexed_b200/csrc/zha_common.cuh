@@ -42,6 +42,7 @@ struct TreeDev {
     float* qref;                // [Hkv][Lcap][R][d]
     float* khat[kMaxLevels];    // level l-1: [batch][Hkv][ncap][R][d]
     float* bhat[kMaxLevels];    // level l-1: [batch][Hkv][ncap][R]
+    float* vhat[kMaxLevels];    // level l-1: [batch][Hkv][ncap][d] value summaries (R = 1), or null
     int64_t ncap[kMaxLevels];
     int Lcap;
     int R;                      // reference queries (planes) per node

@@ -45,6 +45,8 @@ struct RouteArgs {
     int64_t cand_cap, par_cap, kb_cap, N_cap;
     PlanArgs plan;          // the gather plan, built here by the group's last CTA when fuse_plan
     uint32_t* grp_done;     // [batch*Hkv] query heads routed, zero between calls
+    float2* pr_ml;          // value summaries (tree.vhat set): [batch*n_q*Hq] (max in log2 units, sum)
+    float* pr_acc;          //   and [batch*n_q*Hq][d] of the nodes the cut dropped; else null
     int fuse_plan;
     int sel_cap, batch, Hq, Hkv, B, b, L_fixed, n_q;
     float scale;
@@ -61,6 +63,9 @@ struct RouteSmem {
     int32_t keep_prefix[kScoresSmem / 32];
     int32_t tie_slot[kTieMax];
     float q[128];
+    float pr_acc[128];                 // the dropped nodes' running value sum (value summaries)
+    float pr_m, pr_l;                  //   its max (nats) and mass
+    float pr_lw[kRouteWarps];          //   per-warp masses of one level
     int scan[kRouteWarps + 1];
     float redf[kRouteWarps];
     int redi[kRouteWarps];
@@ -423,14 +428,104 @@ __device__ __forceinline__ void scan_children2(const float* __restrict__ kh0, co
     }
 }
 
+// Value summaries: the candidates of one level that the cut dropped (valid, not in the
+// ascending kept list) join the running partial (sm.pr_m, sm.pr_l, sm.pr_acc) as pseudo-keys
+// of log-mass s and value vhat.  Slots are parent-major (b per parent, as the scan wrote
+// them); one warp per parent, lane r decides child r, the kept rows are skipped.
+template <int D, int NVR>
+__device__ void add_dropped(const float* sc, const int32_t* par, int np_par, int b, int64_t nl,
+                            const int32_t* kept, int n_kept, const float* vh, RouteSmem& sm) {
+    constexpr int VF = D / 32;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    auto is_kept = [&](int32_t node) {
+        int lo = 0, hi = n_kept;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (kept[mid] < node) lo = mid + 1;
+            else hi = mid;
+        }
+        return lo < n_kept && kept[lo] == node;
+    };
+    // the level's largest dropped score
+    float mx = -INFINITY;
+    for (int i = tid; i < np_par * b; i += kRouteThreads) {
+        const float s = sc[i];
+        if (s != -INFINITY && !is_kept(par[i / b] * b + i % b)) mx = fmaxf(mx, s);
+    }
+    mx = warp_max(mx);
+    if (lane == 0) sm.redf[w] = mx;
+    __syncthreads();
+    mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kRouteWarps; ++i) mx = fmaxf(mx, sm.redf[i]);
+    if (mx == -INFINITY) return;   // uniform: nothing dropped at this level
+    const float m_old = sm.pr_m, m_new = fmaxf(m_old, mx);
+    float acc[VF], lw = 0.f;
+#pragma unroll
+    for (int e = 0; e < VF; ++e) acc[e] = 0.f;
+    for (int pi = w; pi < np_par; pi += kRouteWarps) {
+        const int64_t c0 = static_cast<int64_t>(par[pi]) * b;
+        const int cnt = static_cast<int>(min(static_cast<int64_t>(b), nl - c0));
+        float wr = 0.f;
+        if (lane < cnt) {
+            const float s = sc[pi * b + lane];
+            if (s != -INFINITY && !is_kept(static_cast<int32_t>(c0 + lane))) wr = expf(s - m_new);
+        }
+        lw += wr;
+        const uint32_t mask = __ballot_sync(0xffffffffu, wr > 0.f);
+        for (int r0 = 0; r0 < NVR; r0 += 4) {   // four rows' loads in flight at a time
+            if (((mask >> r0) & 0xfu) == 0u) continue;
+            float x[4][VF];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                if ((mask >> (r0 + r)) & 1u) load_n<float, VF>(vh + (c0 + r0 + r) * D + lane * VF, x[r]);
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                if ((mask >> (r0 + r)) & 1u) {
+                    const float e = __shfl_sync(0xffffffffu, wr, r0 + r);
+#pragma unroll
+                    for (int f = 0; f < VF; ++f) acc[f] = fmaf(e, x[r][f], acc[f]);
+                }
+        }
+    }
+    lw = warp_sum(lw);
+    // cross-warp sum: [warp][D] values through the (idle) block-cut bins, masses in pr_lw
+    static_assert(kRouteWarps * 128 * sizeof(float) <= sizeof(RouteSmem::bin_mass), "scratch fits the bins");
+    float* red = reinterpret_cast<float*>(sm.bin_mass);
+#pragma unroll
+    for (int f = 0; f < VF; ++f) red[w * D + lane * VF + f] = acc[f];
+    if (lane == 0) sm.pr_lw[w] = lw;
+    __syncthreads();
+    const float alpha = m_old == -INFINITY ? 0.f : expf(m_old - m_new);
+    if (tid < D) {
+        float t = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < kRouteWarps; ++ww) t += red[ww * D + tid];
+        sm.pr_acc[tid] = sm.pr_acc[tid] * alpha + t;
+    }
+    if (tid == 0) {
+        float t = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < kRouteWarps; ++ww) t += sm.pr_lw[ww];
+        sm.pr_l = sm.pr_l * alpha + t;
+        sm.pr_m = m_new;
+    }
+    __syncthreads();
+}
+
 // The top-down walk of one decode query (the body of route_decode_kernel).
-template <typename T, int D, int NVR, bool MP>
+template <typename T, int D, int NVR, bool MP, bool VS>
 __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, int cta, int64_t row, int64_t slice,
                                            int64_t N, int64_t Ntree) {
     constexpr int VF = D / 32;   // fp32 summary elements per lane
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     (void)N;
     if (tid < D) sm.q[tid] = to_f32(static_cast<const T*>(a.Q)[row * D + tid]) * a.scale;
+    constexpr bool vsum = VS && !MP;   // value summaries (R = 1)
+    if constexpr (vsum) {
+        if (tid < D) sm.pr_acc[tid] = 0.f;
+        if (tid == 0) { sm.pr_m = -INFINITY; sm.pr_l = 0.f; }
+    }
     int64_t n[kMaxLevels];
     const int L = tree_levels(Ntree, a.B, a.b, a.L_fixed, n);
     float qv[VF];
@@ -494,6 +589,7 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
         }
         __syncthreads();
         // ---- top-p cut and compaction of the kept node ids
+        const int np_par = np;
         const int nxt = nc <= kParentsSmem ? (cur == 0 ? 1 : 0) : (cur == 2 ? 3 : 2);
         auto node_of = [par, b](int i) { return static_cast<int32_t>(par[i / b] * b + i % b); };
         if (nc <= 64) {
@@ -508,6 +604,8 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
             np = top_p_select(sc, nc, a.p[l - 1], bufs[nxt], sm, big ? ws_kb : sm.keep_ballot,
                               big ? reinterpret_cast<int32_t*>(ws_kb) + a.kb_cap : sm.keep_prefix, node_of);
         }
+        if constexpr (vsum)
+            add_dropped<D, NVR>(sc, par, np_par, b, nl, bufs[nxt], np, a.tree.vhat[l - 1] + slice * ncap * D, sm);
         cur = nxt;
     }
     // ---- level-1 selection -> sel
@@ -520,14 +618,19 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
         a.cand[row] = static_cast<int32_t>(scored);
         if (np > a.sel_cap) raise_status(ZHA_ERR_CAPACITY);
     }
+    if constexpr (vsum) {   // the dropped nodes' partial, max in log2 units as the attention's partials
+        if (tid < D) a.pr_acc[row * D + tid] = sm.pr_acc[tid];
+        if (tid == 0) a.pr_ml[row] = make_float2(sm.pr_m * 1.4426950408889634f, sm.pr_l);
+    }
 }
 
 
 // One CTA per (sequence, query head): the whole top-down walk of one decode query.
 // NVR = b rounded up to a power of two (4, 8, 16 or 32).
 // MP: nodes carry several reference-query planes (R > 1); R = 1 compiles the
-// single-plane scan alone.
-template <typename T, int D, int NVR, bool MP>
+// single-plane scan alone.  VS: the tree holds value summaries (R = 1): the nodes the
+// cut drops are summed into a per-query partial.
+template <typename T, int D, int NVR, bool MP, bool VS = false>
 __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     RouteSmem& sm = *reinterpret_cast<RouteSmem*>(smem_raw);
@@ -543,7 +646,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
     if (!valid) {
         if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.sel_count[row] = 0; a.cand[row] = 0; }
     } else {
-        route_walk<T, D, NVR, MP>(a, sm, cta, row, slice, N, Ntree);
+        route_walk<T, D, NVR, MP, VS>(a, sm, cta, row, slice, N, Ntree);
     }
     if (a.fuse_plan) {
         // the last of the group's G query-head CTAs builds the group's gather plan; the

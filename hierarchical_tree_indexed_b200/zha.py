@@ -35,10 +35,10 @@ class ZhaConfig(ctypes.Structure):
                 ("B", ctypes.c_int32), ("b", ctypes.c_int32), ("R", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("batch", ctypes.c_int32), ("N_cap", ctypes.c_int64),
                 ("L_fixed", ctypes.c_int32), ("scale", ctypes.c_float),
-                ("p", ctypes.c_float * MAX_LEVELS)]
+                ("p", ctypes.c_float * MAX_LEVELS), ("vsum", ctypes.c_int32)]
 
 
-EXPORTS = ["zha_levels_cap", "zha_tree_bytes", "zha_tree_level", "zha_tree_count_offset", "zha_workspace_bytes", "zha_workspace_init", "zha_workspace_stats", "zha_attend_kernel", "zha_build",
+EXPORTS = ["zha_levels_cap", "zha_tree_bytes", "zha_tree_level", "zha_tree_level_v", "zha_tree_count_offset", "zha_workspace_bytes", "zha_workspace_init", "zha_workspace_stats", "zha_attend_kernel", "zha_build",
            "zha_extend", "zha_append", "zha_route", "zha_attend", "zha_attend_noalloc", "zha_decode", "zha_dense", "zha_get_status",
            "zha_last_error"]
 
@@ -58,13 +58,14 @@ def lib():
         "zha_levels_cap": [C, P],
         "zha_tree_bytes": [C, P],
         "zha_tree_level": [C, I32, P, P, P],
+        "zha_tree_level_v": [C, I32, P],
         "zha_tree_count_offset": [C, P],
         "zha_workspace_bytes": [C, I32, P],
         "zha_workspace_init": [C, P, SZ, P],
         "zha_workspace_stats": [C, I32, P, P],
         "zha_attend_kernel": [C, I32, P],
-        "zha_build": [C, P, P, P, P, P],
-        "zha_extend": [C, P, P, P, P],
+        "zha_build": [C, P, P, P, P, P, P],
+        "zha_extend": [C, P, P, P, P, P],
         "zha_append": [C, P, P, P, P, P, P, P],
         "zha_route": [C, P, P, I32, P, P, P, I32, P, SZ, P],
         "zha_attend": [C, P, P, P, P, I32, P, P, P, I32, P, P, SZ, P],
@@ -119,12 +120,14 @@ class Config:
     R: int = 1
     L_fixed: int = 0
     scale: float = 0.0
+    vsum: int = 0
 
     def c(self) -> ZhaConfig:
         cfg = ZhaConfig()
         cfg.d, cfg.Hq, cfg.Hkv, cfg.B, cfg.b, cfg.R = self.d, self.Hq, self.Hkv, self.B, self.b, self.R
         cfg.dtype = {"f32": F32, "bf16": BF16}[self.dtype]
         cfg.batch, cfg.N_cap, cfg.L_fixed, cfg.scale = self.batch, self.N_cap, self.L_fixed, self.scale
+        cfg.vsum = self.vsum
         ps = [self.p] * MAX_LEVELS if isinstance(self.p, (int, float)) else list(self.p)
         ps = ps + [ps[-1]] * (MAX_LEVELS - len(ps))
         for i in range(MAX_LEVELS):
@@ -164,6 +167,16 @@ def tree_level_view(cfg: Config, tree: torch.Tensor, level: int) -> tuple[torch.
     kh = tree[ko.value:ko.value + 4 * cfg.batch * cfg.Hkv * n * cfg.R * cfg.d].view(torch.float32)
     bh = tree[bo.value:bo.value + 4 * cfg.batch * cfg.Hkv * n * cfg.R].view(torch.float32)
     return kh.view(cfg.batch, cfg.Hkv, n, cfg.R, cfg.d), bh.view(cfg.batch, cfg.Hkv, n, cfg.R)
+
+
+def tree_vhat_view(cfg: Config, tree: torch.Tensor, level: int) -> torch.Tensor:
+    """vhat [batch][Hkv][nodes_cap][d] fp32 view of one level (cfg.vsum = 1)."""
+    vo, ko, bo, nc = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_int64()
+    _check(lib().zha_tree_level(ctypes.byref(cfg.c()), level, ctypes.byref(ko), ctypes.byref(bo), ctypes.byref(nc)))
+    _check(lib().zha_tree_level_v(ctypes.byref(cfg.c()), level, ctypes.byref(vo)))
+    n = nc.value
+    vh = tree[vo.value:vo.value + 4 * cfg.batch * cfg.Hkv * n * cfg.d].view(torch.float32)
+    return vh.view(cfg.batch, cfg.Hkv, n, cfg.d)
 
 
 def tree_count_view(cfg: Config, tree: torch.Tensor) -> torch.Tensor:
@@ -206,17 +219,18 @@ def alloc_workspace(cfg: Config, n_q: int = 1, device="cuda", stream=None) -> to
     return ws
 
 
-def build(cfg: Config, K, qref, N, tree, stream=None):
-    """qref: [Hkv][>= levels_cap][R][d] fp32 (sliced to levels_cap here)."""
+def build(cfg: Config, K, qref, N, tree, stream=None, V=None):
+    """qref: [Hkv][>= levels_cap][R][d] fp32 (sliced to levels_cap here).  V: the value cache
+    (read with cfg.vsum = 1)."""
     Lc = levels_cap(cfg)
     q = qref[:, :Lc].contiguous()
-    _check(lib().zha_build(ctypes.byref(cfg.c()), _ptr(K), _ptr(q), _ptr(N), _ptr(tree), _stream(stream)))
+    _check(lib().zha_build(ctypes.byref(cfg.c()), _ptr(K), _ptr(V), _ptr(q), _ptr(N), _ptr(tree), _stream(stream)))
     return q   # keep alive until the copy has run
 
 
-def extend(cfg: Config, K, N, tree, stream=None):
+def extend(cfg: Config, K, N, tree, stream=None, V=None):
     """Grows the tree to index keys [0, N[s]) already written into K (see include/zha.h)."""
-    _check(lib().zha_extend(ctypes.byref(cfg.c()), _ptr(K), _ptr(N), _ptr(tree), _stream(stream)))
+    _check(lib().zha_extend(ctypes.byref(cfg.c()), _ptr(K), _ptr(V), _ptr(N), _ptr(tree), _stream(stream)))
 
 
 def append(cfg: Config, K, V, k_new, v_new, N, tree, stream=None):

@@ -83,7 +83,20 @@ typedef struct zha_config {
     int32_t L_fixed;  /* 0 = depth rule, else the fixed number of levels      */
     float scale;      /* softmax scale; 0 = 1/sqrt(d)                         */
     float p[ZHA_MAX_LEVELS];
+    int32_t vsum;     /* 1: value summaries (decode, R = 1), see below        */
 } zha_config;
+
+/*
+ * Value summaries (vsum = 1; [HTI] Future Directions (4): pruned subtrees
+ * contribute coarse attention outputs).  Every node also stores vhat, the
+ * values pooled with the weights that pool its khat (a leaf: softmax(scale
+ * qhat.K) V; above: the children's vhat with the children's weights), and
+ * decoding adds every node the top-p cut drops as one pseudo-key: log-mass =
+ * its routing score s, value = its vhat.  Keys of I(q) that also lie under a
+ * dropped node (the sink, a current chunk inside the tree) count in both
+ * terms.  zha_build and zha_extend then need V; R must be 1; chunked prefill
+ * (n_q > 1) is refused.  vsum = 0 leaves every call as without it.
+ */
 
 /* Levels the tree can reach for any N <= N_cap (Qref must hold this many). */
 int zha_levels_cap(const zha_config *cfg, int32_t *levels);
@@ -97,6 +110,9 @@ int zha_tree_bytes(const zha_config *cfg, size_t *bytes);
  * [batch][Hkv][nodes_cap][R] fp32 arrays, and nodes_cap.  For inspection. */
 int zha_tree_level(const zha_config *cfg, int32_t level, size_t *khat_offset, size_t *bhat_offset,
                    int64_t *nodes_cap);
+/* With vsum = 1: byte offset of level `level`'s vhat [batch][Hkv][nodes_cap][d] fp32.
+ * ZHA_ERR_INVALID_ARG when vsum = 0. */
+int zha_tree_level_v(const zha_config *cfg, int32_t level, size_t *vhat_offset);
 
 /* Byte offset of the per-sequence count of indexed keys, int32 [batch]. */
 int zha_tree_count_offset(const zha_config *cfg, size_t *offset);
@@ -133,9 +149,10 @@ int zha_attend_kernel(const zha_config *cfg, int32_t n_q, int32_t *kind);
  * Upper levels are "constructed recursively from their children's
  * summaries": each child is a pseudo-key of log-mass scale q.khat_c + bhat_c,
  * and the node is the tangent of their LSE at the level's reference query.
- * Qref is copied into the tree.  N is read on the device.
+ * Qref is copied into the tree.  N is read on the device.  V (the value cache,
+ * laid out as K) is read only with vsum = 1, and may then not be NULL.
  */
-int zha_build(const zha_config *cfg, const void *K, const float *Qref, const int32_t *N,
+int zha_build(const zha_config *cfg, const void *K, const void *V, const float *Qref, const int32_t *N,
               void *tree, zha_stream_t stream);
 
 /*
@@ -145,9 +162,10 @@ int zha_build(const zha_config *cfg, const void *K, const float *Qref, const int
  * level ([EoQ] "the tree is built on the fly as the context grows").  The
  * result is bitwise equal to zha_build at N.  N[s] below the tree's current
  * count, or above N_cap, sets ZHA_ERR_INVALID_ARG on the device and leaves
- * that sequence's count unchanged.
+ * that sequence's count unchanged.  V as for zha_build.
  */
-int zha_extend(const zha_config *cfg, const void *K, const int32_t *N, void *tree, zha_stream_t stream);
+int zha_extend(const zha_config *cfg, const void *K, const void *V, const int32_t *N, void *tree,
+               zha_stream_t stream);
 
 /*
  * zha_append -- decode-time growth ([EoQ] "the tree is built on the fly as the

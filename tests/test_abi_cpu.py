@@ -32,9 +32,10 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_struct_layout_matches_header():
-    # int32 x 8, int64, int32, float, float[16] -> 8*4 + 8 + 4 + 4 + 64 = 112 bytes
-    assert ctypes.sizeof(zha.ZhaConfig) == 112
-    assert zha.ZhaConfig.N_cap.offset == 32 and zha.ZhaConfig.p.offset == 48
+    # int32 x 8, int64, int32, float, float[16], int32 -> 8*4 + 8 + 4 + 4 + 64 + 4 = 116 bytes,
+    # padded to the int64's alignment: 120
+    assert ctypes.sizeof(zha.ZhaConfig) == 120
+    assert zha.ZhaConfig.N_cap.offset == 32 and zha.ZhaConfig.p.offset == 48 and zha.ZhaConfig.vsum.offset == 112
 
 
 def cfg(**kw):
@@ -58,6 +59,7 @@ def test_sizes_and_levels(lib):
     (dict(d=96), 2), (dict(R=17), 2), (dict(Hq=30), 1), (dict(Hq=64), 2), (dict(B=0), 1),
     (dict(B=512), 2), (dict(b=1), 1), (dict(b=64), 2), (dict(batch=0), 1), (dict(N_cap=0), 1),
     (dict(p=0.0), 1), (dict(p=float("nan")), 1), (dict(L_fixed=17), 1), (dict(scale=-1.0), 1),
+    (dict(vsum=2), 1), (dict(vsum=1, R=2), 2),
 ])
 def test_config_validation(lib, kw, code):
     with pytest.raises(zha.ZhaError) as e:
@@ -69,7 +71,10 @@ def test_config_validation(lib, kw, code):
 def test_null_pointers_and_small_workspace_are_refused_on_the_host(lib):
     c = cfg(batch=1, N_cap=4096)
     cc = ctypes.byref(c.c())
-    assert lib.zha_build(cc, None, None, None, None, None) == 1
+    assert lib.zha_build(cc, None, None, None, None, None, None) == 1
+    assert lib.zha_extend(cc, None, None, None, None, None) == 1
+    cv = ctypes.byref(cfg(batch=1, N_cap=4096, vsum=1).c())                # value summaries need V
+    assert lib.zha_build(cv, 1, None, 1, 1, 1, None) == 1
     assert lib.zha_append(cc, None, None, None, None, None, None, None) == 1
     need = zha.workspace_bytes(c)
     assert lib.zha_route(cc, 1, 1, 1, 1, 1, 1, 16, 256, need - 1, None) == 6

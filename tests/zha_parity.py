@@ -124,7 +124,7 @@ class Decoder:
         self.O = torch.zeros((cfg.batch, 1, cfg.Hq, cfg.d), dtype=torch.float32, device="cuda")
 
     def build(self):
-        self._q = zha.build(self.cfg, self.K, self.qref, self.N, self.tree)
+        self._q = zha.build(self.cfg, self.K, self.qref, self.N, self.tree, V=self.V)
 
     def route_attend(self, Q: torch.Tensor):
         zha.route(self.cfg, self.tree, Q, self.N, self.sel, self.cnt, self.ws)
