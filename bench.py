@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling cases)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's N (profiling cases)")
     ap.add_argument("--sweep", default="", help="comma-separated context lengths: tree path vs dense baseline")
+    ap.add_argument("--vsum", action="store_true",
+                    help="decode with value summaries of the dropped subtrees, and report their error against dense")
     return ap.parse_args()
 
 
@@ -235,7 +237,7 @@ def reference_arm(args, rank):
 class DecodeRun:
     """Device buffers of one decode workload and its three captured phases."""
 
-    def __init__(self, w, dev, N_cap, rank):
+    def __init__(self, w, dev, N_cap, rank, vsum=False):
         import torch
 
         from hierarchical_tree_indexed_b200 import workloads as W
@@ -245,7 +247,8 @@ class DecodeRun:
         data = W.planted(w, device=dev, N_cap=N_cap, n_queries=POOL, seq_base=rank.rank * w.batch)
         self.K, self.V, self.Qp, self.knp, self.vnp = data["K"], data["V"], data["Q"], data["k_new"], data["v_new"]
         self.cfg = zha.Config(d=w.d, Hq=w.Hq, Hkv=w.Hkv, B=w.B, b=w.b, batch=w.batch, N_cap=N_cap,
-                              dtype=w.dtype, p=w.p)
+                              dtype=w.dtype, p=w.p, vsum=1 if vsum else 0)
+        self.qref = data["qref"]
         cfg = self.cfg
         self.N = torch.full((w.batch,), w.N, dtype=torch.int32, device=dev)
         self.tree = zha.alloc_tree(cfg, dev)
@@ -258,7 +261,7 @@ class DecodeRun:
         self.v_in = torch.empty_like(self.k_in)
         self.rows_v, self.cand_v = zha.workspace_stats_view(cfg, self.ws)
         zha.get_status(clear=True)
-        self.qref_dev = zha.build(cfg, self.K, data["qref"], self.N, self.tree)
+        self.qref_dev = zha.build(cfg, self.K, data["qref"], self.N, self.tree, V=self.V)
         del data
         torch.cuda.synchronize()
         self.load(0)
@@ -645,6 +648,44 @@ def prefill_main(args, rank, w):
     return 0
 
 
+def value_summary_report(run, args, queries=8, ps=(None, 0.8, 0.5)):
+    """Relative L2 error against dense attention of the decode outputs with and without the
+    dropped subtrees' value summaries, on the same queries and the same cache, for a few p
+    (None = the workload's).  The tree without summaries is built apart (its layout differs)."""
+    import dataclasses
+
+    import torch
+
+    zha, w = run.zha, run.w
+    cfg_v = run.cfg
+    cfg_0 = dataclasses.replace(cfg_v, vsum=0)
+    tree_0 = zha.alloc_tree(cfg_0, run.dev)
+    q_keep = zha.build(cfg_0, run.K, run.qref, run.N, tree_0)
+    ws_0 = zha.alloc_workspace(cfg_0, device=run.dev)
+    out = {}
+    for p in ps:
+        pv = w.p if p is None else p
+        cv, c0 = dataclasses.replace(cfg_v, p=pv), dataclasses.replace(cfg_0, p=pv)
+        ev, e0 = [], []
+        for j in range(queries):
+            q = run.Qp[j].reshape(w.batch, 1, w.Hq, w.d).contiguous()
+            ov, o0, od = (torch.zeros_like(run.O) for _ in range(3))
+            zha.route(cv, run.tree, q, run.N, run.sel, run.cnt, run.ws)
+            zha.attend(cv, run.K, run.V, run.tree, q, run.N, None, None, ov, run.ws)
+            zha.route(c0, tree_0, q, run.N, run.sel, run.cnt, ws_0)
+            zha.attend(c0, run.K, run.V, tree_0, q, run.N, None, None, o0, ws_0)
+            zha.dense(c0, run.K, run.V, q, run.N, od, ws_0)
+            nd = od.norm(dim=-1)
+            ev.append(((ov - od).norm(dim=-1) / nd).mean().item())
+            e0.append(((o0 - od).norm(dim=-1) / nd).mean().item())
+        out[str(pv)] = {"with": sum(ev) / len(ev), "without": sum(e0) / len(e0)}
+    torch.cuda.synchronize()
+    run.check_status("the value-summary report")
+    del q_keep
+    return {"error_vs_dense": out, "queries": queries * w.batch * w.Hq,
+            "note": "mean over (query, head) of |o - o_dense| / |o_dense|, decode queries of the workload"}
+
+
 def main():
     args = parse()
     from hierarchical_tree_indexed_b200 import dist as D
@@ -667,7 +708,7 @@ def main():
     K_steps, W_steps = args.steps, args.warmup
     e2e_steps = 0 if args.no_e2e else min(K_steps, 500)
     N_cap = w.N + W_steps + K_steps + min(K_steps, PHASE_STEPS) + E2E_WARMUP + e2e_steps + 8
-    run = DecodeRun(w, dev, N_cap, rank)
+    run = DecodeRun(w, dev, N_cap, rank, vsum=args.vsum)
     flush = L2Flush(dev)
     for _ in range(W_steps):
         run.load(run.step)
@@ -701,6 +742,8 @@ def main():
     t_dense = run.dense_time(8, flush)
     es = 2 if w.dtype == "bf16" else 4
     dense_gbs = (w.batch * w.Hkv * int(run.N[0].item()) * w.d * es * 2) / t_dense / 1e9
+
+    vsum_report = value_summary_report(run, args) if args.vsum else None
 
     # ---- end to end through the public C-ABI call with host buffers
     e2e = None
@@ -745,7 +788,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": rank.world, "steps": K_steps,
             "warmup": W_steps, "ms_per_step": t_max / K_steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": config_dict(w, rank.world),
+            "config": {**config_dict(w, rank.world), **({"value_summaries": True} if args.vsum else {})},
             "hbm_gbs": step_gbs, "hbm_frac_of_peak": step_gbs / peak,
             "roofline": {"bound": "hbm", "kernel": run.zha.attend_kernel(run.cfg), "achieved": att_gbs, "peak": peak,
                          "unit": "GB/s", "frac": att_gbs / peak, "traffic": traffic,
@@ -755,6 +798,7 @@ def main():
                           "attend": r["t_att"] / K_steps * 1e3},
             "bytes_per_step": {"attend": attend_bytes, "route": route_bytes, "append": append_bytes},
             "read_fraction": read_fraction,
+            "value_summaries": vsum_report,
             "dense_baseline": {"ms_per_step": t_dense * 1e3, "hbm_gbs": dense_gbs,
                                "queries_per_s": w.batch / t_dense, "speedup_of_tree": t_dense / (t_max / K_steps)},
             "gpu_launches": 3 * K_steps,
