@@ -10,6 +10,14 @@ K/V, N = 1,048,576 keys per sequence, leaf block 64, branching 16, p = 0.95,
 planted-cluster synthetic keys and queries.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference]
+                    [--workload decode1m|decode128k|decode8m|prefill256k] [--vsum] [--sweep N1,N2,...]
+
+The step runs as one CUDA graph (append, route with the plan fused, attend); the
+phases are timed apart in a second pass.  --workload prefill256k times a chunked
+prefill (a 4096-query chunk over a 256K prefix) instead; --vsum decodes with the
+dropped subtrees' value summaries and reports their error against dense
+attention; --sweep compares the decode step with the dense baseline over context
+lengths.
 
 Prints one JSON line on rank 0.  Times are CUDA-event device times on the
 launching stream (max over ranks); L2 is flushed (256 MiB write, then a 256 MiB read) before every

@@ -16,8 +16,11 @@
  *
  * Parity: leaf summary, upper-level summary, routing, index set and
  * attention are each pinned by tests (closed forms, brute force, the p = 1
- * dense limit, tangent exactness).  The margin of S8 (a test-side construct
- * the pages do not define) and the generators are "parity unpinned".
+ * dense limit, tangent exactness); so are the value summaries (uniform
+ * blocks, a linear map V = K M, the partition of the tree by kept blocks and
+ * dropped nodes, exactness when every top node holds one key).  The routing
+ * margin (how far a cut lies from p; a test-side construct the pages do not
+ * define) and the generators are "parity unpinned".
  */
 #include <math.h>
 #include <stdint.h>

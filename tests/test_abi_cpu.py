@@ -75,6 +75,13 @@ def test_null_pointers_and_small_workspace_are_refused_on_the_host(lib):
     assert lib.zha_extend(cc, None, None, None, None, None) == 1
     cv = ctypes.byref(cfg(batch=1, N_cap=4096, vsum=1).c())                # value summaries need V
     assert lib.zha_build(cv, 1, None, 1, 1, 1, None) == 1
+    with pytest.raises(zha.ZhaError) as e:                                  # no chunked prefill with them
+        zha.workspace_bytes(cfg(batch=1, N_cap=4096, vsum=1), 64)
+    assert e.value.code == 2
+    assert lib.zha_attend_noalloc(cv, 1, 1, 1, 1, 1, 1, 1, 1, 16, 1, None) == 2   # nor the no-alloc call
+    off = ctypes.c_size_t()
+    assert lib.zha_tree_level_v(cc, 1, ctypes.byref(off)) == 1             # vsum = 0: no vhat
+    assert lib.zha_tree_level_v(cv, 1, ctypes.byref(off)) == 0
     assert lib.zha_append(cc, None, None, None, None, None, None, None) == 1
     need = zha.workspace_bytes(c)
     assert lib.zha_route(cc, 1, 1, 1, 1, 1, 1, 16, 256, need - 1, None) == 6
