@@ -10,6 +10,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -203,22 +204,28 @@ int dev_info(DevInfo* info) {
 template <typename Kern>
 int allow_smem(Kern kernel, size_t need) {
     static std::mutex mu;
-    static std::set<std::pair<const void*, int>> done;
-    DevInfo di;
-    ZHA_TRY(dev_info(&di));
-    cudaFuncAttributes fa;
-    ZHA_CUDA(cudaFuncGetAttributes(&fa, kernel));
-    const size_t dyn_max = static_cast<size_t>(di.smem_optin) - fa.sharedSizeBytes;
-    if (need > dyn_max)
-        return fail(ZHA_ERR_UNSUPPORTED, "kernel needs %zu B of dynamic shared memory (device max %zu)", need, dyn_max);
+    static std::map<std::pair<const void*, int>, size_t> done;   // (kernel, device) -> dynamic shared memory allowed
     int dev = 0;
     ZHA_CUDA(cudaGetDevice(&dev));
-    std::lock_guard<std::mutex> lk(mu);
-    auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
-    if (!done.count(key)) {
-        ZHA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn_max)));
-        done.insert(key);
+    const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+    size_t dyn_max = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto it = done.find(key);
+        if (it != done.end()) dyn_max = it->second;
     }
+    if (dyn_max == 0) {   // first launch of this kernel on this device
+        DevInfo di;
+        ZHA_TRY(dev_info(&di));
+        cudaFuncAttributes fa;
+        ZHA_CUDA(cudaFuncGetAttributes(&fa, kernel));
+        dyn_max = static_cast<size_t>(di.smem_optin) - fa.sharedSizeBytes;
+        ZHA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dyn_max)));
+        std::lock_guard<std::mutex> lk(mu);
+        done[key] = dyn_max;
+    }
+    if (need > dyn_max)
+        return fail(ZHA_ERR_UNSUPPORTED, "kernel needs %zu B of dynamic shared memory (device max %zu)", need, dyn_max);
     return ZHA_OK;
 }
 
