@@ -45,6 +45,7 @@ PREFILL_METRIC = "ZHA chunked prefill queries/s at 256K ctx (4096-query chunk, t
 FALLBACK_BF16_TFLOPS = 1590.0
 UNIT = "queries/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # the B200 spec-sheet HBM3e bandwidth, for a second fraction beside the measured copy
 POOL = 64                 # distinct (q, k_new, v_new) sets cycled through by the steps
 E2E_WARMUP = 3            # untimed end-to-end steps before the timed ones
 PHASE_STEPS = 200         # steps of the per-phase breakdown (after the timed one-graph steps)
@@ -182,11 +183,48 @@ class Clocks:
 
 # ------------------------------------------------------------------ CPU oracle arm
 
-def oracle_sample(w, seconds: float, warmup: int = 1, steps: int | None = None):
-    """Times the oracle's route + attend of single query heads on one (sequence, KV head)
-    slice of the workload (tree built once, not timed).  Decode: the query of the token
-    appended at N.  Chunked prefill: queries of the chunk at t = N + i over a tree on the
-    first N keys.  Returns (seconds per head-query, head-queries timed, setup seconds)."""
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def time_oracle(calls, seconds: float, threads: int, steps: int | None = None):
+    """Runs the oracle calls (closures, cycled) on `threads` host threads for about `seconds` of
+    wall time (or exactly `steps` calls); the oracle is C behind ctypes, which releases the
+    GIL, so the threads run in parallel.  Returns (seconds per call, calls made)."""
+    import concurrent.futures as cf
+    import threading
+
+    lock = threading.Lock()
+    state = {"i": 0, "done": 0}
+    t_end = time.perf_counter() + seconds
+
+    def worker():
+        while True:
+            with lock:
+                if (steps is None and time.perf_counter() >= t_end) or (steps is not None and state["i"] >= steps):
+                    return
+                k = state["i"]
+                state["i"] += 1
+            calls[k % len(calls)]()
+            with lock:
+                state["done"] += 1
+
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        for f in [ex.submit(worker) for _ in range(threads)]:
+            f.result()
+    spent = time.perf_counter() - t0
+    return spent / max(state["done"], 1), state["done"]
+
+
+def oracle_sample(w, seconds: float, warmup: int = 1, steps: int | None = None, threads: int = 1):
+    """Times the oracle's route + attend of single query heads on one (sequence, KV head) slice of
+    the workload drawn on the host (tree built once, not timed).  Decode: the query of the token
+    appended at N.  Chunked prefill: queries of the chunk at t = N + i over a tree on the first N
+    keys.  Returns (seconds per head-query, head-queries timed, setup seconds)."""
     import torch
 
     from hierarchical_tree_indexed_b200 import workloads as W
@@ -206,27 +244,91 @@ def oracle_sample(w, seconds: float, warmup: int = 1, steps: int | None = None):
     qs = qs.to(torch.bfloat16).float().reshape(-1, w.d)
     pos = [w.N + ((k // w.G) * 61) % extra if w.prefill else w.N for k in range(len(qs))]
     setup = time.perf_counter() - t0
-    done, spent, i = 0, 0.0, 0
     for _ in range(warmup):
         O.decode_query(qs[0], tree, K, V, pos[0], w.p)
-    while (steps is None and spent < seconds) or (steps is not None and done < steps):
-        k = i % len(qs)
-        i += 1
-        t = time.perf_counter()
-        O.decode_query(qs[k], tree, K, V, pos[k], w.p)
-        spent += time.perf_counter() - t
-        done += 1
-    return spent / done, done, setup
+    calls = [lambda k=k: O.decode_query(qs[k], tree, K, V, pos[k], w.p) for k in range(len(qs))]
+    per, done = time_oracle(calls, seconds, threads, steps)
+    return per, done, setup
+
+
+MARGIN = 1e-4   # index sets must be bit-exact where the oracle's cut margin exceeds this
+
+
+def oracle_leg(run, w, seconds: float, slices, n_queries: int = 8):
+    """The CPU-oracle leg, after the timed region, on the GPU run's own data: for each sampled
+    (sequence, KV head) slice the host copies its keys and values, the oracle builds its tree
+    (untimed), and then
+      * parity: the GPU routes n_queries pool queries at the current N and its index sets are
+        compared with the oracle's (bit-exact required where the cut margin exceeds 1e-4; the
+        mismatch rate below it is reported);
+      * timing: the oracle's route + attend of single query heads over the slices' pool
+        queries, on one host core and on every core this process may use."""
+    import numpy as np
+    import torch
+
+    from oracle import oracle as O
+    zha, dev = run.zha, run.dev
+    t0 = time.perf_counter()
+    torch.cuda.synchronize()
+    N = run.N.cpu()
+    host, trees = {}, {}
+    for (s, h) in slices:
+        n = int(N[s])
+        host[(s, h)] = (run.K[s, h, :n].cpu(), run.V[s, h, :n].cpu())
+        trees[(s, h)] = O.build_tree(host[(s, h)][0], n, w.B, w.b, run.qref[h].cpu())
+    setup = time.perf_counter() - t0
+    rep = {"queries": 0, "exact_required": 0, "mismatches_required": 0, "low_margin": 0,
+           "mismatches_low_margin": 0}
+    calls = []
+    for j in range(n_queries):
+        q = run.Qp[j].reshape(w.batch, 1, w.Hq, w.d).contiguous()
+        zha.route(run.cfg, run.tree, q, run.N, run.sel, run.cnt, run.ws)
+        torch.cuda.synchronize()
+        sel, cnt, qh = run.sel.cpu(), run.cnt.cpu(), q.cpu().float()
+        for (s, h) in slices:
+            n = int(N[s])
+            for hq in range(h * w.G, (h + 1) * w.G):
+                rt = O.route(qh[s, 0, hq], trees[(s, h)], w.p)
+                g = sel[s, 0, hq, :int(cnt[s, 0, hq])].numpy().astype(np.int64)
+                same = len(g) == len(rt.sel) and bool(np.array_equal(g, rt.sel))
+                rep["queries"] += 1
+                if rt.min_margin > MARGIN:
+                    rep["exact_required"] += 1
+                    rep["mismatches_required"] += 0 if same else 1
+                else:
+                    rep["low_margin"] += 1
+                    rep["mismatches_low_margin"] += 0 if same else 1
+                K_h, V_h = host[(s, h)]
+                calls.append(lambda q_=qh[s, 0, hq], t_=trees[(s, h)], K_=K_h, V_=V_h, n_=n:
+                             O.decode_query(q_, t_, K_, V_, n_ - 1, w.p))
+    run.check_status("the parity sample")
+    rep["slices"] = [list(x) for x in slices]
+    rep["note"] = (f"{n_queries} pool queries routed on the GPU at the current N, each query head of the sampled "
+                   f"slices checked against the fp64 oracle on the same keys; index sets must be bit-exact where the "
+                   f"oracle's cut margin exceeds {MARGIN:g}")
+    calls[0]()   # warm-up
+    per1, done1 = time_oracle(calls, seconds / 2, 1)
+    cores = host_cores()
+    perN, doneN = time_oracle(calls, seconds / 2, cores)
+    cpu = {"value": 1.0 / (perN * w.Hq), "unit": UNIT, "cores": cores, "kind": "oracle",
+           "single_core_value": 1.0 / (per1 * w.Hq),
+           "sample": f"fp64 C oracle route + attend of single query heads on {len(slices)} (sequence, KV head) slices "
+                     f"of {w.name} (the GPU run's keys at N={int(N[slices[0][0]])}, trees built in {setup:.1f}s "
+                     f"untimed): {done1} calls on 1 core, {doneN} calls on {cores} threads, scaled to decode "
+                     f"queries of all {w.Hq} heads"}
+    return cpu, rep
 
 
 def reference_arm(args, rank):
     if rank.rank != 0:
         return 0
     w = workload(args)
-    per_head, done, setup = oracle_sample(w, 0.0, warmup=args.warmup, steps=args.steps)
+    cores = host_cores()
+    # each step is a bounded sample: one call per host thread
+    per_head, done, setup = oracle_sample(w, 0.0, warmup=args.warmup, steps=args.steps * cores, threads=cores)
     value = 1.0 / (per_head * w.Hq)
-    sample = (f"{done} single-head route+attend calls of the fp64 C oracle on one (sequence, KV head) "
-              f"slice of {w.name} (N={w.N}, tree built once in {setup:.1f}s untimed), scaled to "
+    sample = (f"{done} single-head route+attend calls of the fp64 C oracle on {cores} host threads, on one "
+              f"(sequence, KV head) slice of {w.name} (N={w.N}, tree built once in {setup:.1f}s untimed), scaled to "
               f"{'chunk' if w.prefill else 'decode'} queries of all {w.Hq} heads")
     line = {"metric": PREFILL_METRIC if w.prefill else METRIC, "value": value, "unit": UNIT, "impl": "reference",
             "n_gpus": args.gpus,
@@ -234,7 +336,7 @@ def reference_arm(args, rank):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": dict(config_dict(w, args.gpus), step="one query head's route + attend in the fp64 oracle"),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -267,7 +369,7 @@ class DecodeRun:
         self.q_in = torch.empty((w.batch, 1, w.Hq, w.d), dtype=self.K.dtype, device=dev)
         self.k_in = torch.empty((w.batch, w.Hkv, w.d), dtype=self.K.dtype, device=dev)
         self.v_in = torch.empty_like(self.k_in)
-        self.rows_v, self.cand_v = zha.workspace_stats_view(cfg, self.ws)
+        self.rows_v, self.cand_v, self.scan_v = zha.workspace_stats_view(cfg, self.ws)
         zha.get_status(clear=True)
         self.qref_dev = zha.build(cfg, self.K, data["qref"], self.N, self.tree, V=self.V)
         del data
@@ -328,6 +430,7 @@ class DecodeRun:
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
         rows_acc = torch.zeros((), dtype=torch.float64, device=self.dev)
         cand_acc = torch.zeros((), dtype=torch.float64, device=self.dev)
+        scan_acc = torch.zeros((), dtype=torch.float64, device=self.dev)
         for k in range(steps):
             self.load(self.step)
             self.step += 1
@@ -337,6 +440,7 @@ class DecodeRun:
             ev[k][1].record(stream)
             rows_acc += self.rows_v.sum()
             cand_acc += self.cand_v.sum()
+            scan_acc += self.scan_v.sum()
         torch.cuda.synchronize()
         self.check_status("the timed steps")
         t_step = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
@@ -355,7 +459,7 @@ class DecodeRun:
         self.check_status("the phase steps")
         t = [sum(e[i].elapsed_time(e[i + 1]) for e in pev) / 1e3 * steps / n_ph for i in range(3)]
         return dict(t_app=t[0], t_route=t[1], t_att=t[2], t_step=t_step, t_phases=sum(t),
-                    rows=rows_acc.item() / steps, cand=cand_acc.item() / steps)
+                    rows=rows_acc.item() / steps, cand=cand_acc.item() / steps, scanned=scan_acc.item() / steps)
 
     def dense_time(self, reps, flush):
         import torch
@@ -370,11 +474,15 @@ class DecodeRun:
         self.check_status("the dense baseline")
         return sum(a.elapsed_time(b) for a, b in evs[2:]) / reps / 1e3
 
-    def bytes_per_step(self, rows, cand):
+    def bytes_per_step(self, rows, scanned):
+        """Algorithmic bytes of one step: the attention's K and V rows gathered (the union over a
+        KV head's query heads) plus q read and O written; the route's tree nodes read (the
+        distinct nodes per KV head, 4d + 4 bytes each) plus q; the append's token and its share
+        of a leaf block's summary."""
         w = self.w
         es = 2 if w.dtype == "bf16" else 4
         attend = rows * w.d * es * 2 + w.batch * w.Hq * w.d * (es + 4)
-        route = cand * (4 * w.d + 4) + w.batch * w.Hq * w.d * es
+        route = scanned * (4 * w.d + 4) + w.batch * w.Hq * w.d * es
         append = w.batch * w.Hkv * (2 * w.d * es + (w.B * w.d * es + (w.d + 1) * 4 * 4) / w.B)
         return attend, route, append
 
@@ -456,7 +564,7 @@ def prefill_main(args, rank, w):
     cnt = torch.zeros((w.batch, n_q, w.Hq), dtype=torch.int32, device=dev)
     O = torch.zeros((w.batch, n_q, w.Hq, w.d), dtype=torch.float32, device=dev)
     Od = torch.zeros_like(O)
-    steps_v, cand_v = zha.workspace_stats_view(cfg, ws, n_q)
+    steps_v, cand_v, _ = zha.workspace_stats_view(cfg, ws, n_q)
     zha.get_status(clear=True)
     zha.build(cfg, K, qref, torch.full((w.batch,), Np, dtype=torch.int32, device=dev), tree)
 
@@ -617,11 +725,14 @@ def prefill_main(args, rank, w):
                "note": "zha_route + zha_attend per chunk (not graphed) after 3 untimed chunks, pinned host Q, chunk K/V and O"}
     cpu = None
     if rank.leader and rank.world == 1 and not args.no_cpu_baseline:
-        per_head, done, setup = oracle_sample(w, args.cpu_seconds)
-        cpu = {"value": 1.0 / (per_head * w.Hq), "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{done} single-head route+attend calls of the fp64 C oracle for chunk queries of one "
-                         f"(sequence, KV head) slice of {w.name} (tree built once, {setup:.1f}s untimed), scaled "
-                         f"to chunk queries of all {w.Hq} heads"}
+        per1, done1, setup = oracle_sample(w, args.cpu_seconds / 2)
+        cores = host_cores()
+        perN, doneN, _ = oracle_sample(w, args.cpu_seconds / 2, threads=cores)
+        cpu = {"value": 1.0 / (perN * w.Hq), "unit": UNIT, "cores": cores, "kind": "oracle",
+               "single_core_value": 1.0 / (per1 * w.Hq),
+               "sample": f"single-head route+attend calls of the fp64 C oracle for chunk queries of one (sequence, KV "
+                         f"head) slice of {w.name} drawn on the host (tree built once, {setup:.1f}s untimed): {done1} "
+                         f"calls on 1 core, {doneN} on {cores} threads, scaled to chunk queries of all {w.Hq} heads"}
     if rank.leader:
         line = {
             "metric": PREFILL_METRIC, "value": value, "unit": UNIT, "n_gpus": rank.world, "steps": K_steps,
@@ -737,11 +848,12 @@ def main():
     queries = w.batch * K_steps * rank.world
     value = queries / t_max
 
-    attend_bytes, route_bytes, append_bytes = run.bytes_per_step(r["rows"], r["cand"])
+    attend_bytes, route_bytes, append_bytes = run.bytes_per_step(r["rows"], r["scanned"])
     step_bytes = attend_bytes + route_bytes + append_bytes
     peak, peak_src = measured_peaks()
     att_gbs = attend_bytes / (r["t_att"] / K_steps) / 1e9
     step_gbs = step_bytes / (r["t_step"] / K_steps) / 1e9
+    ra_gbs = (attend_bytes + route_bytes) / ((r["t_route"] + r["t_att"]) / K_steps) / 1e9
     read_fraction = r["rows"] / (w.batch * w.Hkv * w.N)
     khash = source_hash(ATTEND_SOURCES)
     tr = profiled_traffic(khash)
@@ -788,13 +900,9 @@ def main():
                        "host row copied in once, O copied out; L2 not flushed"}
         run.check_status("the e2e steps")
 
-    cpu = None
+    cpu, parity = None, None
     if rank.leader and rank.world == 1 and not args.no_cpu_baseline:
-        per_head, done, setup = oracle_sample(w, args.cpu_seconds)
-        cpu = {"value": 1.0 / (per_head * w.Hq), "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{done} single-head route+attend calls of the fp64 C oracle on one (sequence, KV head) "
-                         f"slice of {w.name} (tree built once, {setup:.1f}s untimed), scaled to decode queries "
-                         f"of all {w.Hq} heads"}
+        cpu, parity = oracle_leg(run, w, args.cpu_seconds, [(0, 0), (w.batch - 1, w.Hkv - 1)])
 
     if rank.leader:
         line = {
@@ -802,14 +910,21 @@ def main():
             "warmup": W_steps, "ms_per_step": t_max / K_steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {**config_dict(w, rank.world), **({"value_summaries": True} if args.vsum else {})},
-            "hbm_gbs": step_gbs, "hbm_frac_of_peak": step_gbs / peak,
+            "hbm_gbs": step_gbs, "hbm_frac_of_peak": step_gbs / peak, "hbm_frac_of_nominal": step_gbs / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "kernel": run.zha.attend_kernel(run.cfg), "achieved": att_gbs, "peak": peak,
                          "unit": "GB/s", "frac": att_gbs / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} copy bandwidth", "algorithmic_bytes_per_launch": attend_bytes,
+                         "frac_of_nominal": att_gbs / NOMINAL_HBM_GBS, "frac_of_dense_kernel": att_gbs / dense_gbs,
                          "kernel_source_sha256_16": khash},
+            "route_attend": {"gbs": ra_gbs, "frac_of_peak": ra_gbs / peak, "frac_of_nominal": ra_gbs / NOMINAL_HBM_GBS,
+                             "frac_of_dense_kernel": ra_gbs / dense_gbs, "bytes": attend_bytes + route_bytes,
+                             "ms": (r["t_route"] + r["t_att"]) / K_steps * 1e3,
+                             "note": "route (plan fused) and attend phases, each its own CUDA graph, over the "
+                                     "algorithmic bytes: distinct tree nodes read, K and V rows gathered, q and O"},
             "phases_ms": {"append": r["t_app"] / K_steps * 1e3, "route": r["t_route"] / K_steps * 1e3,
                           "attend": r["t_att"] / K_steps * 1e3},
             "bytes_per_step": {"attend": attend_bytes, "route": route_bytes, "append": append_bytes},
+            "route_nodes": {"distinct_per_step": r["scanned"], "per_head_sum_per_step": r["cand"]},
             "read_fraction": read_fraction,
             "value_summaries": vsum_report,
             "dense_baseline": {"ms_per_step": t_dense * 1e3, "hbm_gbs": dense_gbs,
@@ -818,6 +933,7 @@ def main():
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "parity": parity,
         }
         print(json.dumps(line), flush=True)
     del run

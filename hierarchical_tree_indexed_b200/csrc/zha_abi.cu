@@ -4,12 +4,14 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <set>
@@ -29,6 +31,19 @@ using namespace zha;
 namespace {
 
 thread_local char g_err[512] = "";
+
+// An NVTX range around one C-ABI call, so that a profiler's timeline names the call
+// each kernel belongs to (free when no tool is attached).
+struct Range {
+    explicit Range(const char* name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range&) = delete;
+    Range& operator=(const Range&) = delete;
+};
+
+// Bound of the tensor-core decode attention's waits on another warp's progress
+// (zha_set_wait_limit); waits on the kernel's own copies and MMAs keep kWaitLongNs.
+std::atomic<uint64_t> g_wait_ns{kWaitLongNs};
 
 int fail(int code, const char* fmt, ...) {
     va_list ap;
@@ -61,7 +76,7 @@ struct TreeLayout {
 struct WsLayout {
     int64_t cand_cap, par_cap, kb_cap, sel_cap, item_cap, words;
     size_t off_scores, off_parents, off_sel, off_count, off_items, off_nitems, off_ml, off_acc, off_counters;
-    size_t off_rows, off_cand, off_ballot, off_grp, off_pr_ml, off_pr_acc;
+    size_t off_rows, off_cand, off_ballot, off_scanned, off_pr_ml, off_pr_acc;
     size_t total;
 };
 
@@ -136,12 +151,12 @@ TreeDev tree_view(const TreeLayout& t, void* tree) {
     return v;
 }
 
-// The decode kernels clear their own per-group counters when they finish, so these
-// must hold zero between calls.  They sit at the front of every workspace layout,
+// The decode attention clears its own per-group merge counters when it finishes, so
+// these must hold zero between calls.  They sit at the front of every workspace layout,
 // decode and prefill alike, and no prefill call writes there: a workspace moves
 // between decode and chunks of any length without being zeroed again.
 size_t ws_counter_bytes(const zha_config* c) {
-    return 2 * align256(sizeof(uint32_t) * static_cast<size_t>(c->batch) * c->Hkv);
+    return align256(sizeof(uint32_t) * static_cast<size_t>(c->batch) * c->Hkv);
 }
 
 int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
@@ -157,7 +172,6 @@ int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
     w->words = (t.ncap[0] + 31) / 32;
     size_t off = 0;
     w->off_counters = off; off = align256(off + sizeof(uint32_t) * groups);
-    w->off_grp = off;      off = align256(off + sizeof(uint32_t) * groups);
     w->off_scores = off;   off = align256(off + sizeof(float) * ctas * w->cand_cap);
     w->off_parents = off;  off = align256(off + sizeof(int32_t) * ctas * 2 * w->par_cap);
     w->off_sel = off;      off = align256(off + sizeof(int32_t) * ctas * w->sel_cap);
@@ -168,6 +182,7 @@ int ws_layout(const zha_config* c, int n_q, const TreeLayout& t, WsLayout* w) {
     w->off_acc = off;      off = align256(off + sizeof(float) * groups * kSplitMax * G * c->d);
     w->off_rows = off;     off = align256(off + sizeof(int32_t) * groups);
     w->off_cand = off;     off = align256(off + sizeof(int32_t) * ctas);
+    w->off_scanned = off;  off = align256(off + sizeof(int32_t) * groups);
     w->off_ballot = off;   off = align256(off + sizeof(uint32_t) * ctas * 2 * w->kb_cap);
     w->off_pr_ml = off;    off = align256(off + (c->vsum ? sizeof(float2) * ctas : 0));
     w->off_pr_acc = off;   off = align256(off + (c->vsum ? sizeof(float) * ctas * c->d : 0));
@@ -200,14 +215,41 @@ int dev_info(DevInfo* info) {
     return ZHA_OK;
 }
 
-// Lets `kernel` use the device's opt-in shared memory (once per kernel and device).
+// The calling thread's current CUDA context (the driver entry point is looked up once
+// through the runtime, so the library needs no link against the driver library).
+int current_context(CUcontext* out) {
+    using GetCtx = CUresult (*)(CUcontext*);
+    static std::mutex mu;
+    static GetCtx fn = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!fn) {
+            void* p = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            ZHA_CUDA(cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q));
+            if (q != cudaDriverEntryPointSuccess || !p) return fail(ZHA_ERR_CUDA, "cuCtxGetCurrent is not available");
+            fn = reinterpret_cast<GetCtx>(p);
+        }
+    }
+    if (fn(out) == CUDA_SUCCESS && *out) return ZHA_OK;
+    int dev = 0;   // no context yet: binding the current device initialises its primary context
+    ZHA_CUDA(cudaGetDevice(&dev));
+    ZHA_CUDA(cudaSetDevice(dev));
+    if (fn(out) != CUDA_SUCCESS || !*out) return fail(ZHA_ERR_CUDA, "no current CUDA context");
+    return ZHA_OK;
+}
+
+// Lets `kernel` use the device's opt-in shared memory (once per kernel, device and
+// context: a device reset creates a new context, which starts with the defaults).
 template <typename Kern>
 int allow_smem(Kern kernel, size_t need) {
     static std::mutex mu;
-    static std::map<std::pair<const void*, int>, size_t> done;   // (kernel, device) -> dynamic shared memory allowed
+    static std::map<std::pair<const void*, std::pair<int, CUcontext>>, size_t> done;   // -> dynamic smem allowed
     int dev = 0;
     ZHA_CUDA(cudaGetDevice(&dev));
-    const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+    CUcontext ctx = nullptr;
+    ZHA_TRY(current_context(&ctx));
+    const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), std::make_pair(dev, ctx));
     size_t dyn_max = 0;
     {
         std::lock_guard<std::mutex> lk(mu);
@@ -301,14 +343,50 @@ int run_append(const zha_config* c, const TreeLayout& lay, void* K, void* V, con
 // ---------------------------------------------------------------- route
 PlanArgs plan_args(const zha_config* c, const WsLayout& wl, const TreeLayout& lay, const void* tree,
                    const int32_t* N, const int32_t* sel, const int32_t* cnt, int32_t sel_cap, void* ws);
-bool plan_fits_route(const zha_config* c, const WsLayout& wl);
+
+// The plan region of the fused route: the G plan bitmaps (wl.words words each), then the
+// bitmap of kept nodes of every level l >= 2 (for the count of distinct nodes read).
+// Returns its words and fills the level offsets.
+int route_region_words(const zha_config* c, const TreeLayout& lay, const WsLayout& wl, int* lvl_off) {
+    const int G = c->Hq / c->Hkv;
+    int64_t words = static_cast<int64_t>(G) * std::max<int64_t>(wl.words, 1);
+    for (int l = 0; l < kMaxLevels; ++l) lvl_off[l] = 0;
+    for (int l = 2; l <= lay.Lcap; ++l) {
+        lvl_off[l - 1] = static_cast<int>(words);
+        words += (lay.ncap[l - 1] + 31) / 32;
+    }
+    return static_cast<int>(std::min<int64_t>(words, int64_t{1} << 30));
+}
+
+// The route kernel builds the plan itself (clusters of G CTAs) when its plan region fits
+// next to the router's shared memory on this device.
+bool plan_fits_route(const zha_config* c, const TreeLayout& lay, const WsLayout& wl) {
+    DevInfo di;
+    if (dev_info(&di) != ZHA_OK) return false;
+    int lvl_off[kMaxLevels];
+    const size_t need = sizeof(RouteSmem) + 4 * static_cast<size_t>(route_region_words(c, lay, wl, lvl_off));
+    return need + 1024 <= static_cast<size_t>(di.smem_optin);
+}
 
 template <typename T, int D, int NVR>
-int run_route_t(const RouteArgs& a, int ctas, cudaStream_t st) {
+int run_route_t(const RouteArgs& a, int ctas, int G, cudaStream_t st) {
     auto kern = a.tree.R > 1 ? route_decode_kernel<T, D, NVR, true>
                 : a.pr_ml ? route_decode_kernel<T, D, NVR, false, true> : route_decode_kernel<T, D, NVR, false>;
-    ZHA_TRY(allow_smem(kern, sizeof(RouteSmem)));
-    kern<<<ctas, kRouteThreads, sizeof(RouteSmem), st>>>(a);
+    const size_t smem = sizeof(RouteSmem) + (a.fuse_plan ? 4 * static_cast<size_t>(a.region_words) : 0);
+    ZHA_TRY(allow_smem(kern, smem));
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(static_cast<unsigned>(ctas));
+    lc.blockDim = dim3(kRouteThreads);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = a.fuse_plan ? static_cast<unsigned>(G) : 1u;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    ZHA_CUDA(cudaLaunchKernelEx(&lc, kern, a));
     return check_launch("route");
 }
 
@@ -328,15 +406,17 @@ int run_route(const zha_config* c, const TreeLayout& lay, const WsLayout& wl, co
     a.scale = scale_of(c);
     for (int l = 0; l < kMaxLevels; ++l) a.p[l] = c->p[l];
     a.plan = plan_args(c, wl, lay, tree, N, sel, cnt, sel_cap, ws);
-    a.grp_done = at<uint32_t>(ws, wl.off_grp);
+    a.scanned = at<int32_t>(ws, wl.off_scanned);
+    a.region_words = route_region_words(c, lay, wl, a.lvl_off);
     a.pr_ml = c->vsum ? at<float2>(ws, wl.off_pr_ml) : nullptr;
     a.pr_acc = c->vsum ? at<float>(ws, wl.off_pr_acc) : nullptr;
     a.fuse_plan = fuse ? 1 : 0;
     const int ctas = c->batch * c->Hq;
-    if (c->b <= 4) return run_route_t<T, D, 4>(a, ctas, st);
-    if (c->b <= 8) return run_route_t<T, D, 8>(a, ctas, st);
-    if (c->b <= 16) return run_route_t<T, D, 16>(a, ctas, st);
-    return run_route_t<T, D, 32>(a, ctas, st);
+    const int G = c->Hq / c->Hkv;
+    if (c->b <= 4) return run_route_t<T, D, 4>(a, ctas, G, st);
+    if (c->b <= 8) return run_route_t<T, D, 8>(a, ctas, G, st);
+    if (c->b <= 16) return run_route_t<T, D, 16>(a, ctas, G, st);
+    return run_route_t<T, D, 32>(a, ctas, G, st);
 }
 
 // ---------------------------------------------------------------- attend
@@ -399,9 +479,11 @@ int run_attend(const zha_config* c, const WsLayout& wl, const void* K, const voi
     a.item_cap = wl.item_cap; a.N_cap = c->N_cap;
     a.groups = c->batch * c->Hkv; a.Hq = c->Hq; a.Hkv = c->Hkv; a.n_q = 1;
     a.qscale = scale_of(c) * 1.4426950408889634f;
+    a.wait_ns = kWaitLongNs;
     DevInfo di;
     ZHA_TRY(dev_info(&di));
     if (attend_tc_fits(c, di)) {
+        a.wait_ns = g_wait_ns.load();
         switch (c->Hq / c->Hkv) {
             case 1: return run_attend_tc<1>(c, a, st);
             case 2: return run_attend_tc<2>(c, a, st);
@@ -429,10 +511,6 @@ PlanArgs plan_args(const zha_config* c, const WsLayout& wl, const TreeLayout& la
     return a;
 }
 
-// The route kernel builds the plan itself when the group's bitmap fits its score buffer.
-bool plan_fits_route(const zha_config* c, const WsLayout& wl) {
-    return static_cast<int64_t>(c->Hq / c->Hkv) * std::max<int64_t>(wl.words, 1) <= kScoresSmem;
-}
 
 int run_plan(const zha_config* c, const WsLayout& wl, const TreeLayout& lay, const void* tree, const int32_t* N,
              const int32_t* sel, const int32_t* cnt, int32_t sel_cap, void* ws, cudaStream_t st) {
@@ -706,23 +784,29 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 
-// Device address of g_noalloc_scratch on the current device, looked up once per
-// device (the symbol's host-side name is not a device address).
+// Device address of g_noalloc_scratch in the current device's current context,
+// looked up once per (device, context) with that device current (the symbol's
+// host-side name is not a device address).  Keying on the context as well means a
+// device reset, which gives the device a new primary context and reloads the
+// library's module there, never leaves a stale address behind.
 int noalloc_scratch_ptr(void** out) {
     static std::mutex mu;
-    static void* ptrs[64] = {};
+    static std::map<std::pair<int, CUcontext>, void*> ptrs;
     int dev = 0;
     ZHA_CUDA(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= 64) return fail(ZHA_ERR_UNSUPPORTED, "device %d", dev);
+    CUcontext ctx = nullptr;
+    ZHA_TRY(current_context(&ctx));
     std::lock_guard<std::mutex> lk(mu);
-    if (!ptrs[dev]) {
+    const auto key = std::make_pair(dev, ctx);
+    auto it = ptrs.find(key);
+    if (it == ptrs.end()) {
         void* p = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || !p)
             return fail(ZHA_ERR_CUDA, "cudaGetSymbolAddress(g_noalloc_scratch): %s", cudaGetErrorString(e));
-        ptrs[dev] = p;
+        it = ptrs.emplace(key, p).first;
     }
-    *out = ptrs[dev];
+    *out = it->second;
     return ZHA_OK;
 }
 
@@ -795,22 +879,26 @@ int zha_workspace_bytes(const zha_config* cfg, int32_t n_q, size_t* bytes) {
     return ZHA_OK;
 }
 
-int zha_workspace_stats(const zha_config* cfg, int32_t n_q, size_t* rows_offset, size_t* cand_offset) {
+int zha_workspace_stats(const zha_config* cfg, int32_t n_q, size_t* rows_offset, size_t* cand_offset,
+                        size_t* scanned_offset) {
     TreeLayout t;
     WsLayout w;
     ZHA_TRY(need(rows_offset, "rows_offset"));
     ZHA_TRY(need(cand_offset, "cand_offset"));
+    ZHA_TRY(need(scanned_offset, "scanned_offset"));
     ZHA_TRY(tree_layout(cfg, &t));
     if (n_q > 1) {
         PfLayout p;
         ZHA_TRY(pf_layout(cfg, n_q, t, &p));
         *rows_offset = p.off_steps;
         *cand_offset = p.off_cand;
+        *scanned_offset = p.off_cand;
         return ZHA_OK;
     }
     ZHA_TRY(ws_layout(cfg, n_q, t, &w));
     *rows_offset = w.off_rows;
     *cand_offset = w.off_cand;
+    *scanned_offset = w.off_scanned;
     return ZHA_OK;
 }
 
@@ -844,6 +932,7 @@ int zha_workspace_init(const zha_config* cfg, void* ws, size_t ws_bytes, zha_str
 
 int zha_build(const zha_config* cfg, const void* K, const void* V, const float* Qref, const int32_t* N, void* tree,
               zha_stream_t stream) {
+    Range nvtx_range("zha_build");
     TreeLayout t;
     ZHA_TRY(tree_layout(cfg, &t));
     ZHA_TRY(need(K, "K"));
@@ -858,6 +947,7 @@ int zha_build(const zha_config* cfg, const void* K, const void* V, const float* 
 
 int zha_extend(const zha_config* cfg, const void* K, const void* V, const int32_t* N, void* tree,
                zha_stream_t stream) {
+    Range nvtx_range("zha_extend");
     TreeLayout t;
     ZHA_TRY(tree_layout(cfg, &t));
     ZHA_TRY(need(K, "K"));
@@ -869,6 +959,7 @@ int zha_extend(const zha_config* cfg, const void* K, const void* V, const int32_
 
 int zha_append(const zha_config* cfg, void* K, void* V, const void* k_new, const void* v_new, int32_t* N,
                void* tree, zha_stream_t stream) {
+    Range nvtx_range("zha_append");
     TreeLayout t;
     ZHA_TRY(tree_layout(cfg, &t));
     ZHA_TRY(need(K, "K"));
@@ -882,6 +973,7 @@ int zha_append(const zha_config* cfg, void* K, void* V, const void* k_new, const
 
 int zha_route(const zha_config* cfg, const void* tree, const void* Q, int32_t n_q, const int32_t* N, int32_t* sel,
               int32_t* sel_count, int32_t sel_cap, void* ws, size_t ws_bytes, zha_stream_t stream) {
+    Range nvtx_range("zha_route");
     TreeLayout t;
     WsLayout w;
     if (n_q > 1) {
@@ -905,7 +997,8 @@ int zha_route(const zha_config* cfg, const void* tree, const void* Q, int32_t n_
     ZHA_TRY(need(sel, "sel"));
     ZHA_TRY(need(sel_count, "sel_count"));
     if (sel_cap < 1) return fail(ZHA_ERR_INVALID_ARG, "sel_cap=%d", sel_cap);
-    const bool fuse = plan_fits_route(cfg, w);
+    const bool fuse = plan_fits_route(cfg, t, w);
+    if (!fuse) ZHA_CUDA(cudaMemsetAsync(at<int32_t>(ws, w.off_scanned), 0, sizeof(int32_t) * cfg->batch * cfg->Hkv, stream));
     ZHA_TRY(ZHA_DISPATCH(cfg, run_route, cfg, t, w, tree, Q, N, sel, sel_count, sel_cap, ws, fuse, stream));
     return fuse ? ZHA_OK : run_plan(cfg, w, t, tree, N, sel, sel_count, sel_cap, ws, stream);
 }
@@ -913,6 +1006,7 @@ int zha_route(const zha_config* cfg, const void* tree, const void* Q, int32_t n_
 int zha_attend(const zha_config* cfg, const void* K, const void* V, const void* tree, const void* Q, int32_t n_q,
                const int32_t* N, const int32_t* sel, const int32_t* sel_count, int32_t sel_cap, float* O, void* ws,
                size_t ws_bytes, zha_stream_t stream) {
+    Range nvtx_range("zha_attend");
     TreeLayout t;
     WsLayout w;
     if (n_q > 1) {
@@ -949,6 +1043,10 @@ int zha_attend(const zha_config* cfg, const void* K, const void* V, const void* 
 int zha_attend_noalloc(const zha_config* cfg, const void* K, const void* V, const void* tree, const void* Q,
                        int32_t n_q, const int32_t* N, const int32_t* sel, const int32_t* sel_count, int32_t sel_cap,
                        float* O, zha_stream_t stream) {
+    Range nvtx_range("zha_attend_noalloc");
+    if (n_q != 1)
+        return fail(ZHA_ERR_UNSUPPORTED, "zha_attend_noalloc: decode only (n_q = 1, got %d); a chunked prefill "
+                    "needs zha_attend with a workspace", n_q);
     if (cfg && cfg->vsum)
         return fail(ZHA_ERR_UNSUPPORTED, "zha_attend_noalloc: value summaries need the router's workspace (vsum = 1)");
     TreeLayout t;
@@ -979,6 +1077,7 @@ int zha_attend_noalloc(const zha_config* cfg, const void* K, const void* V, cons
 
 int zha_decode(const zha_config* cfg, void* K, void* V, void* tree, const void* q, const void* k_new,
                const void* v_new, int32_t* N, float* O, void* ws, size_t ws_bytes, zha_stream_t stream) {
+    Range nvtx_range("zha_decode");
     TreeLayout t;
     WsLayout w;
     ZHA_TRY(tree_layout(cfg, &t));
@@ -990,7 +1089,8 @@ int zha_decode(const zha_config* cfg, void* K, void* V, void* tree, const void* 
     int32_t* sel = at<int32_t>(ws, w.off_sel);
     int32_t* cnt = at<int32_t>(ws, w.off_count);
     const int32_t sel_cap = static_cast<int32_t>(w.sel_cap);
-    const bool fuse = plan_fits_route(cfg, w);
+    const bool fuse = plan_fits_route(cfg, t, w);
+    if (!fuse) ZHA_CUDA(cudaMemsetAsync(at<int32_t>(ws, w.off_scanned), 0, sizeof(int32_t) * cfg->batch * cfg->Hkv, stream));
     ZHA_TRY(ZHA_DISPATCH(cfg, run_route, cfg, t, w, tree, q, N, sel, cnt, sel_cap, ws, fuse, stream));
     if (!fuse) ZHA_TRY(run_plan(cfg, w, t, tree, N, sel, cnt, sel_cap, ws, stream));
     return ZHA_DISPATCH(cfg, run_attend, cfg, w, K, V, q, O, ws, stream);
@@ -998,6 +1098,7 @@ int zha_decode(const zha_config* cfg, void* K, void* V, void* tree, const void* 
 
 int zha_dense(const zha_config* cfg, const void* K, const void* V, const void* Q, int32_t n_q, const int32_t* N,
               float* O, void* ws, size_t ws_bytes, zha_stream_t stream) {
+    Range nvtx_range("zha_dense");
     TreeLayout t;
     WsLayout w;
     if (n_q > 1) {
@@ -1037,6 +1138,12 @@ int zha_get_status(int32_t* status_bits, int32_t clear, zha_stream_t stream) {
         ZHA_CUDA(cudaMemcpyToSymbol(g_status, &z, sizeof z));
     }
     *status_bits = v;
+    return ZHA_OK;
+}
+
+int zha_set_wait_limit(uint64_t ns, uint64_t* previous) {
+    const uint64_t old = g_wait_ns.exchange(ns);
+    if (previous) *previous = old;
     return ZHA_OK;
 }
 

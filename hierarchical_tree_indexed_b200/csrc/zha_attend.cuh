@@ -65,6 +65,7 @@ struct AttendArgs {
     int64_t item_cap, N_cap;
     int groups, Hq, Hkv, n_q;
     float qscale;              // scale * log2(e)
+    uint64_t wait_ns;          // bound of a wait on another warp's progress (then ZHA_ERR_TIMEOUT)
 };
 
 constexpr int kAttConsumers = 8;                       // consumer warps
@@ -165,7 +166,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
         auto acquire_slot = [&](int slot) {   // wait until the consumers released this slot
             if (fills >= kAttStages && ok) {
                 bool got = true;
-                if (lane == 0) got = mbar_wait_bounded(&sm.empty[slot], ((fills / kAttStages) - 1) & 1);
+                if (lane == 0) got = mbar_wait_bounded(&sm.empty[slot], ((fills / kAttStages) - 1) & 1, a.wait_ns);
                 ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
                 if (!ok && lane == 0) raise_status(ZHA_ERR_TIMEOUT);
             }
@@ -273,10 +274,18 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
             x = seg_end;
           }
         }
-        // sentinel: tells the consumers that no stage follows
+        // the bulk copies of the last stages have landed before this warp leaves (on an abort
+        // the consumers may have stopped reading them, and the CTA must not exit with copies
+        // in flight); no stage is re-armed before this, so each wait is on its own data phase
+        if (lane == 0)
+            for (int f = fills > kAttStages ? fills - kAttStages : 0; f < fills; ++f)
+                mbar_wait_bounded(&sm.full[f % kAttStages], (f / kAttStages) & 1, kWaitLongNs);
+        __syncwarp();
+        // sentinel: tells the consumers that no stage follows (not after an abort: a slot still
+        // waiting on the consumers must not be re-armed; they give up on their own bound)
         const int slot = fills % kAttStages;
         acquire_slot(slot);
-        if (lane == 0) {
+        if (ok && lane == 0) {
             sm.desc[slot].n_rows = -1;
             mbar_arrive(&sm.full[slot]);
         }
@@ -295,7 +304,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
     bool stop = false;
     while (!stop) {
         const int slotA = it % kAttStages;
-        if (!mbar_wait_bounded(&sm.full[slotA], (it / kAttStages) & 1)) {
+        if (!mbar_wait_bounded(&sm.full[slotA], (it / kAttStages) & 1, a.wait_ns)) {
             if (lane == 0) raise_status(ZHA_ERR_TIMEOUT);
             break;
         }
@@ -308,7 +317,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
         int slotB = slotA, nB = 0, nst = 1;
         if (!(flags & 1)) {   // not the run's last stage: the next stage belongs to the same run
             slotB = (it + 1) % kAttStages;
-            if (!mbar_wait_bounded(&sm.full[slotB], ((it + 1) / kAttStages) & 1)) {
+            if (!mbar_wait_bounded(&sm.full[slotB], ((it + 1) / kAttStages) & 1, a.wait_ns)) {
                 if (lane == 0) raise_status(ZHA_ERR_TIMEOUT);
                 break;
             }

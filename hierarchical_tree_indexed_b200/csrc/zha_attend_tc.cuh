@@ -73,6 +73,7 @@ struct TcCtl {
     uint32_t tmem;
     int abort;
     int last_flag, sp;
+    uint64_t wait_ns;              // bound of a wait on another warp's progress
     int red[2][4][4];              // [pair parity][warp][head] order-mapped maxima
     float lsum[4][4];              // [warp][head] softmax sums
     float mL[4];                   // [head] a merge's total sum
@@ -91,7 +92,7 @@ __host__ __device__ constexpr size_t tc_smem_bytes(int groups, int grid) {
 // Bounded wait; a timeout is recorded once and later waits of the CTA return at once.
 __device__ __forceinline__ bool twait(uint64_t* bar, uint32_t parity, TcCtl* ctl) {
     if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
-    if (mbar_wait_bounded(bar, parity)) return true;
+    if (mbar_wait_bounded(bar, parity, ctl->wait_ns)) return true;
     *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
     raise_status(ZHA_ERR_TIMEOUT);
     return false;
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         mbar_init(&ctl->fin, 1);
         fence_mbar_init();
         ctl->abort = 0;
+        ctl->wait_ns = a.wait_ns;
         umma::prefetch_tensormap(&tmK);
         umma::prefetch_tensormap(&tmV);
         umma::prefetch_tensormap(&tmQ);
@@ -279,9 +281,10 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                 mbar_arrive(&ctl->kv_full[fills % kTCStages]);
                 ++fills;
             }
-            // the loads of the last pairs have landed before the CTA may exit
+            // the loads of the last pairs have landed before the CTA may exit (the slot the
+            // sentinel re-armed held a pair the MMAs had consumed, so its data was in)
             for (int f = fills > kTCStages ? fills - kTCStages : 0; f < fills; ++f)
-                mbar_wait_bounded(&ctl->kv_full[f % kTCStages], (f / kTCStages) & 1);
+                mbar_wait_bounded(&ctl->kv_full[f % kTCStages], (f / kTCStages) & 1, kWaitLongNs);
         }
     } else if (warp == 5) {
         // ================= MMA issue (one lane): S^T and P V of the pairs in order
@@ -345,7 +348,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                     t_last = global_timer_ns();
                 } else if ((++idle & 1023u) == 0) {
                     if (tc_aborted(ctl)) break;
-                    if (global_timer_ns() - t_last > 2000000000ull) {
+                    if (global_timer_ns() - t_last > ctl->wait_ns) {
                         *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
                         raise_status(ZHA_ERR_TIMEOUT);
                         break;
@@ -353,7 +356,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                 }
             }
             umma::commit(&ctl->fin);
-            mbar_wait_bounded(&ctl->fin, 0);
+            mbar_wait_bounded(&ctl->fin, 0, kWaitLongNs);   // every MMA issued has completed
         }
     } else {
         // ================= softmax warps 0-3

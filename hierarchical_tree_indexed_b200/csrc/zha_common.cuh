@@ -208,15 +208,43 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
     return t;
 }
-// Waits for the phase with the given parity; gives up after ~2 s and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+// The bound of a wait on something that cannot fail to come: a copy this CTA issued
+// itself, or the tensor cores' completion of its own MMAs (~2 s).
+constexpr uint64_t kWaitLongNs = 2000000000ull;
+
+// Waits for the phase with the given parity; gives up after limit_ns of %globaltimer and
+// returns false.  limit_ns = 0 gives up at once unless the phase has already completed.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLongNs) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if (limit_ns == 0) return false;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0 && global_timer_ns() - t0 > 2000000000ull) return false;
+        if ((i & 15u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
     }
 }
+// ---------------------------------------------------------------- thread-block clusters
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Split cluster barrier: every thread of every CTA of the cluster arrives (release), then
+// waits (acquire) for all of them; shared-memory writes before the arrival, local or
+// remote, are visible to every CTA of the cluster after the wait.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// The shared::cluster address of `p` (this CTA's shared memory) in the CTA of the given rank.
+__device__ __forceinline__ uint32_t cluster_map(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+// Atomic OR into a word of a cluster CTA's shared memory (no return value).
+__device__ __forceinline__ void dsmem_or(uint32_t addr, uint32_t v) {
+    asm volatile("red.relaxed.cluster.shared::cluster.or.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

@@ -34,23 +34,109 @@ struct PlanArgs {
     int64_t words;             // bitmap words per head: ceil(n1cap / 32)
 };
 
-// The gather plan of group g (one (sequence, KV head)), computed by one block of
-// kPlanThreads threads.  bits: shared memory for G * a.words words; scan: kPlanThreads/32+1 ints.
-// N, Ntree: the sequence's key count and tree count when the caller has them (else < 0).
-__device__ void plan_group(const PlanArgs& a, int g, uint32_t* bits, int* scan, int64_t N = -1, int64_t Ntree = -1) {
-    const int s = g / a.Hkv, kv = g % a.Hkv, tid = threadIdx.x;
+// The gather plan of group g from the per-head bitmaps of its selected blocks, by one
+// block of kPlanThreads threads.  bits: G bitmaps of a.words words in shared memory, word
+// w of head h at bits[h * a.words + w], holding every selected block below n_1 = Ntree / B
+// (bits at and beyond n_1 clear); the current chunk's block is added here.  scan:
+// kPlanThreads/32+1 ints.  N, Ntree: the sequence's key count and tree count, valid
+// (1 <= N <= N_cap, Ntree <= N).
+__device__ void plan_emit(const PlanArgs& a, int g, uint32_t* bits, int* scan, int64_t N, int64_t Ntree) {
+    const int tid = threadIdx.x;
     const int G = a.G;
     const uint32_t all = (1u << G) - 1u;
-    if (N < 0) {
-        N = a.N[s];
-        Ntree = a.n_tree[s];
+    const int64_t t = N - 1;
+    const int64_t n1 = Ntree / a.B;
+    const int64_t words = (n1 + 31) / 32;
+    const int64_t cb = min(t / a.B, n1);   // C_cur = [cb*B, t]
+    if (tid < G && cb < n1) atomicOr(&bits[tid * a.words + (cb >> 5)], 1u << (cb & 31));
+    __syncthreads();
+    // compaction of the union, ascending.  Warp w takes the words [w*per, (w+1)*per), per a
+    // multiple of 32: its lanes load 32 words at a time and count their blocks; one block scan
+    // places the warps' runs; then each warp walks its non-empty words one at a time, a lane per
+    // block (a word of a cluster often holds 32 blocks).
+    const int nsplit = (a.B + kItemRowsMax - 1) / kItemRowsMax;   // items per block (B > 64)
+    constexpr int NWP = kPlanThreads / 32;
+    const int lane = tid & 31, wp = tid >> 5;
+    int2* out = a.items + static_cast<int64_t>(g) * a.item_cap;
+    const int64_t per = ((words + NWP - 1) / NWP + 31) / 32 * 32;
+    const int64_t w0 = min(words, wp * per), w1 = min(words, w0 + per);
+    auto word_union = [&](int64_t wd) {
+        uint32_t o = 0;
+        if (wd < w1)
+            for (int hh = 0; hh < G; ++hh) o |= bits[hh * a.words + wd];
+        return o;
+    };
+    int mine = 0;
+    for (int64_t c = w0; c < w1; c += 32) mine += __popc(word_union(c + lane));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+    int total;
+    int pos = block_exclusive_scan<NWP>(lane == 0 ? mine * nsplit : 0, scan, &total);
+    pos = __shfl_sync(0xffffffffu, pos, 0);
+    for (int64_t c = w0; c < w1; c += 32) {
+        const uint32_t u = word_union(c + lane);
+        const int cntw = __popc(u) * nsplit;
+        int incl = cntw;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        uint32_t nz = __ballot_sync(0xffffffffu, u != 0u);
+        while (nz) {
+            const int j = __ffs(nz) - 1;
+            nz &= nz - 1u;
+            const uint32_t oj = __shfl_sync(0xffffffffu, u, j);
+            const int pj = pos + __shfl_sync(0xffffffffu, incl - cntw, j);
+            const int64_t wj = c + j;
+            if ((oj >> lane) & 1u) {
+                uint32_t m = 0;
+                for (int hh = 0; hh < G; ++hh) m |= ((bits[hh * a.words + wj] >> lane) & 1u) << hh;
+                const int idx = pj + __popc(oj & ((1u << lane) - 1u)) * nsplit;
+                const int64_t k0 = (wj * 32 + lane) * a.B;
+                if (nsplit == 1) {
+                    out[idx] = make_item(k0, a.B, m);
+                } else {
+                    for (int st = 0, k = 0; st < a.B; st += kItemRowsMax, ++k)
+                        out[idx + k] = make_item(k0 + st, min(kItemRowsMax, a.B - st), m);
+                }
+            }
+        }
+        pos += __shfl_sync(0xffffffffu, incl, 31);
     }
+    if (tid == 0) {
+        int n = total;
+        int64_t rows = static_cast<int64_t>(nsplit == 1 ? total : total / nsplit) * a.B;
+        if (n1 >= 1) {   // sink: key 0 for the heads whose block 0 is not in the union
+            uint32_t m0 = 0;
+            for (int h = 0; h < G; ++h) m0 |= (bits[h * a.words] & 1u) << h;
+            if ((m0 & all) != all) { out[n++] = make_item(0, 1, all & ~m0); rows += 1; }
+        }
+        if (cb == n1)   // C_cur past the last leaf block: the keys [n1*B, t], 64 at a time
+            for (int64_t st = cb * a.B; st <= t && n < a.item_cap; st += kItemRowsMax) {
+                const int c = static_cast<int>(t - st + 1 < kItemRowsMax ? t - st + 1 : kItemRowsMax);
+                out[n++] = make_item(st, c, all);
+                rows += c;
+            }
+        a.n_items[g] = n;
+        a.rows[g] = static_cast<int32_t>(rows);
+    }
+    __syncthreads();
+}
+
+// The gather plan of group g (one (sequence, KV head)) from the selection lists in global
+// memory, computed by one block of kPlanThreads threads.  bits: shared memory for
+// G * a.words words; scan: kPlanThreads/32+1 ints.
+__device__ void plan_group(const PlanArgs& a, int g, uint32_t* bits, int* scan) {
+    const int s = g / a.Hkv, kv = g % a.Hkv, tid = threadIdx.x;
+    const int G = a.G;
+    const int64_t N = a.N[s];
+    const int64_t Ntree = a.n_tree[s];
     if (N < 1 || N > a.N_cap || Ntree > N) {
         if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.n_items[g] = 0; a.rows[g] = 0; }
         __syncthreads();
         return;
     }
-    const int64_t t = N - 1;
     const int64_t n1 = Ntree / a.B;
     const int64_t words = (n1 + 31) / 32;
     // every head's selected blocks into its bitmap: kPlanThreads / G threads per head load
@@ -79,61 +165,8 @@ __device__ void plan_group(const PlanArgs& a, int g, uint32_t* bits, int* scan, 
         const int32_t blk = __ldcg(&hsel[j]);
         if (blk >= 0 && blk < n1) atomicOr(&hb[blk >> 5], 1u << (blk & 31));
     }
-    const int64_t cb = min(t / a.B, n1);   // C_cur = [cb*B, t]
-    if (tid < G && cb < n1) atomicOr(&bits[tid * a.words + (cb >> 5)], 1u << (cb & 31));
     __syncthreads();
-    // compaction of the union, ascending, in rounds of kPlanThreads words (thread t holds word
-    // r * kPlanThreads + t): a block scan places each word's items, then each warp emits its 32
-    // words one at a time with one lane per bit (a word of a cluster has up to 32 blocks)
-    const int nsplit = (a.B + kItemRowsMax - 1) / kItemRowsMax;   // items per block (B > 64)
-    const int lane = tid & 31, wp = tid >> 5;
-    int2* out = a.items + static_cast<int64_t>(g) * a.item_cap;
-    int total = 0;
-    for (int64_t r0 = 0; r0 < words; r0 += kPlanThreads) {
-        const int64_t wd = r0 + tid;
-        uint32_t o = 0;
-        if (wd < words)
-            for (int hh = 0; hh < G; ++hh) o |= bits[hh * a.words + wd];
-        int tot;
-        const int pos = total + block_exclusive_scan<kPlanThreads / 32>(__popc(o) * nsplit, scan, &tot);
-        total += tot;
-        for (int j = 0; j < 32; ++j) {
-            const uint32_t oj = __shfl_sync(0xffffffffu, o, j);
-            if (oj == 0u) continue;
-            const int pj = __shfl_sync(0xffffffffu, pos, j);
-            const int64_t wj = r0 + wp * 32 + j;
-            if ((oj >> lane) & 1u) {
-                uint32_t m = 0;
-                for (int hh = 0; hh < G; ++hh) m |= ((bits[hh * a.words + wj] >> lane) & 1u) << hh;
-                const int idx = pj + __popc(oj & ((1u << lane) - 1u)) * nsplit;
-                const int64_t k0 = (wj * 32 + lane) * a.B;
-                if (nsplit == 1) {
-                    out[idx] = make_item(k0, a.B, m);
-                } else {
-                    for (int st = 0, k = 0; st < a.B; st += kItemRowsMax, ++k)
-                        out[idx + k] = make_item(k0 + st, min(kItemRowsMax, a.B - st), m);
-                }
-            }
-        }
-    }
-    if (tid == 0) {
-        int n = total;
-        int64_t rows = static_cast<int64_t>(nsplit == 1 ? total : total / nsplit) * a.B;
-        if (n1 >= 1) {   // sink: key 0 for the heads whose block 0 is not in the union
-            uint32_t m0 = 0;
-            for (int h = 0; h < G; ++h) m0 |= (bits[h * a.words] & 1u) << h;
-            if ((m0 & all) != all) { out[n++] = make_item(0, 1, all & ~m0); rows += 1; }
-        }
-        if (cb == n1)   // C_cur past the last leaf block: the keys [n1*B, t], 64 at a time
-            for (int64_t st = cb * a.B; st <= t && n < a.item_cap; st += kItemRowsMax) {
-                const int c = static_cast<int>(t - st + 1 < kItemRowsMax ? t - st + 1 : kItemRowsMax);
-                out[n++] = make_item(st, c, all);
-                rows += c;
-            }
-        a.n_items[g] = n;
-        a.rows[g] = static_cast<int32_t>(rows);
-    }
-    __syncthreads();
+    plan_emit(a, g, bits, scan, N, Ntree);
 }
 
 // One CTA per (sequence, KV head).

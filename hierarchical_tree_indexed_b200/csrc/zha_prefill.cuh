@@ -135,7 +135,8 @@ __global__ void __launch_bounds__(kPRThreads, 2) route_prefill_kernel(PRouteArgs
                         const int64_t c1 = static_cast<int64_t>(par[pi + 1]) * b;
                         const int cnt1 = static_cast<int>(min(static_cast<int64_t>(b), nl - c1));
                         scan_children2<D, NVR>(kh + c0 * D, bh + c0, cnt0, kh + c1 * D, bh + c1, cnt1, b, qv,
-                                               sc + static_cast<int64_t>(pi) * b, sc + static_cast<int64_t>(pi + 1) * b);
+                                               sc + static_cast<int64_t>(pi) * b, sc + static_cast<int64_t>(pi + 1) * b,
+                                               nullptr, nullptr);
                     } else {
                         scan_children<D, NVR>(kh + c0 * D, bh + c0, cnt0, b, qv, sc + static_cast<int64_t>(pi) * b);
                     }

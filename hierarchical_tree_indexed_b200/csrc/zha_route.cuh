@@ -14,11 +14,15 @@
 //             transpose-reduce over the warp;
 //   top-p  -- exact and deterministic: masses exp(s - s_max) become 64-bit
 //             fixed-point integers (2^-40 units), so sums are order-free; equal
-//             scores are taken in ascending id order (ties to the lower id).  Up
-//             to 64 candidates one warp sorts them; above that the whole block
-//             bins them by score and ranks the crossing bin only (a single warp
-//             doing the same takes ~18 ns per candidate: 12 us at 650).  Kept ids
-//             stay ascending because children of ascending parents are ascending.
+//             scores are taken in ascending id order (ties to the lower id).  The
+//             masses are binned by score below the level's max (which the scan
+//             already found), one warp finds the bin where the cumulative mass
+//             crosses p, and only that bin's members are ranked exactly (a dense
+//             bin is split into sub-bins first).  Kept ids stay ascending
+//             because children of ascending parents are ascending.
+// The G query heads of one (sequence, KV head) run as one thread-block cluster:
+// each head ORs its kept nodes into the shared memory of the cluster's CTA 0,
+// which then builds the group's gather plan on chip.
 #pragma once
 
 #include "zha_common.cuh"
@@ -41,60 +45,59 @@ struct RouteArgs {
     int32_t* cand;          // [batch][n_q][Hq] candidates scored over all levels (accounting)
     float* ws_scores;       // [batch*Hq][cand_cap]
     int32_t* ws_parents;    // [batch*Hq][2][par_cap]
-    uint32_t* ws_ballot;    // [batch*Hq][2][kb_cap]
+    uint32_t* ws_ballot;    // [batch*Hq][2][kb_cap] the cut's ballot words when they exceed shared memory
     int64_t cand_cap, par_cap, kb_cap, N_cap;
-    PlanArgs plan;          // the gather plan, built here by the group's last CTA when fuse_plan
-    uint32_t* grp_done;     // [batch*Hkv] query heads routed, zero between calls
+    PlanArgs plan;          // the gather plan, built here by the cluster's CTA 0 when fuse_plan
+    int32_t* scanned;       // [batch*Hkv] distinct tree nodes the group's route read (fuse_plan)
+    int lvl_off[kMaxLevels];// fuse_plan: word offset, in CTA 0's plan region, of level l's bitmap of
+                            // kept nodes (index l-1, l >= 2); the G plan bitmaps start at word 0
+    int region_words;       // words of the plan region (dynamic shared memory after RouteSmem)
     float2* pr_ml;          // value summaries (tree.vhat set): [batch*n_q*Hq] (max in log2 units, sum)
     float* pr_acc;          //   and [batch*n_q*Hq][d] of the nodes the cut dropped; else null
-    int fuse_plan;
+    int fuse_plan;          // the G CTAs of a group run as one cluster and build its plan
     int sel_cap, batch, Hq, Hkv, B, b, L_fixed, n_q;
     float scale;
     float p[kMaxLevels];
 };
 
-constexpr int kTieMax = 4096;   // crossing-bin members listed in shared memory (more: found by a scan)
+constexpr int kSpecMax = 256;   // the level below the top is scored with the top level when it has at most this many nodes
+constexpr int kCutBins = 256;      // mass bins of 1/8 nat below the level's max score (a crossing bin
+                                   // with too many members is split again into 256 sub-bins)
+constexpr int kCutMembers = 256;   // crossing-bin members ranked pairwise in shared memory
+
+struct CutSmem {
+    unsigned long long bins[kCutBins];     // zero between cuts
+    unsigned long long mkey[kCutMembers];  // crossing-bin members: order key and mass
+    unsigned long long mmass[kCutMembers];
+    unsigned long long above, target;      // mass ordered before the crossing (sub-)bin; the target
+    int nm, cbin, sbin;                    // members; crossing bin; crossing sub-bin (-1: not split)
+};
 
 struct RouteSmem {
     float scores[kScoresSmem];
     int32_t parents[2][kParentsSmem];
-    unsigned long long bin_mass[1024];
-    uint32_t keep_ballot[kScoresSmem / 32];
-    int32_t keep_prefix[kScoresSmem / 32];
-    int32_t tie_slot[kTieMax];
+    float spec[kSpecMax + 32];         // scores of the level below the top, read with the top level
+    CutSmem cut;
+    uint32_t keep_ballot[kScoresSmem / 32];   // the cut's kept slots, a word per 32
+    int32_t keep_prefix[kScoresSmem / 32];    // and the kept ids before each word
+    float vred[kRouteWarps * 128];     // value summaries: per-warp value sums of one level
     float q[128];
     float pr_acc[128];                 // the dropped nodes' running value sum (value summaries)
     float pr_m, pr_l;                  //   its max (nats) and mass
     float pr_lw[kRouteWarps];          //   per-warp masses of one level
+    int mxkey[2];                      // a level's max score (order-mapped), by level parity
     int scan[kRouteWarps + 1];
     float redf[kRouteWarps];
     int redi[kRouteWarps];
-    int plan_last;
-    int tie_n, cut_bin;
-    unsigned long long cut_above, cut_target;
 };
 
-// Top-p over sc[0..nc) (invalid slots hold -inf).  Writes the kept node ids,
-// ascending, to out and returns their count.  node_of(i) maps a slot to its id.
-constexpr int kBins = 1024;          // score bins of 1/32 nat below the level's max score
-constexpr float kBinsPerNat = 32.0f;
-
-__device__ __forceinline__ int score_bin(float s, float smax) {
-    const float x = (smax - s) * kBinsPerNat;   // >= 0, weakly decreasing in s
-    return x >= static_cast<float>(kBins - 1) ? kBins - 1 : static_cast<int>(x);
+// Order-preserving map of a float (no NaN) to int, and back: the max of scores as an int max.
+__device__ __forceinline__ int ord_key(float x) {
+    const int i = __float_as_int(x);
+    return i >= 0 ? i : i ^ 0x7fffffff;
 }
+__device__ __forceinline__ float key_ord(int k) { return __int_as_float(k >= 0 ? k : k ^ 0x7fffffff); }
 
-// Top-p cut over sc[0..nc) (invalid slots hold -inf): keeps the smallest prefix,
-// in descending score order with ties to the lower slot (= lower node id), whose
-// fixed-point mass reaches ceil(p * total).  Writes the kept node ids, ascending,
-// to out; returns their count.  node_of(i) maps a slot to its node id.
-//
-// One pass bins the candidates by score (bins are monotone in the score, so the
-// bin order is the sorted order up to the order inside a bin) and sums their
-// masses per bin; one warp finds the bin where the cumulative mass crosses the
-// target; only the candidates of that bin are ranked exactly (by score, then
-// slot) against each other.  Candidate i is kept iff the mass of everything
-// ordered before it is below the target.
 // The same cut for nc <= 64, by warp 0 alone: the (score, slot) pairs are sorted by a
 // bitonic network (descending score, ascending slot; two elements per lane), the
 // fixed-point masses are prefix-summed in that order, and candidate e is kept iff the
@@ -162,146 +165,208 @@ __device__ int top_p_small(const float* sc, int nc, float p, int32_t* out, NodeO
     return __popcll(set);
 }
 
-// kball/kpre: ceil(nc/32) words each (shared memory, or the workspace for large nc).
-template <typename NodeOf>
-__device__ int top_p_select(const float* sc, int nc, float p, int32_t* out, RouteSmem& sm, uint32_t* kball,
-                            int32_t* kpre, NodeOf node_of) {
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    // 1. max score; clear the bins
-    float mx = -INFINITY;
-    for (int i = tid; i < nc; i += kRouteThreads) mx = fmaxf(mx, sc[i]);
-    mx = warp_max(mx);
-    if (lane == 0) sm.redf[w] = mx;
-    for (int k = tid; k < kBins; k += kRouteThreads) sm.bin_mass[k] = 0;
-    if (tid == 0) { sm.tie_n = 0; sm.cut_above = 0; sm.cut_target = 0; }
-    __syncthreads();
-    mx = -INFINITY;
+__device__ __forceinline__ int cut_bin(float s, float smax) {
+    const float x = (smax - s) * 8.0f;   // >= 0, weakly decreasing in s
+    return x >= static_cast<float>(kCutBins - 1) ? kCutBins - 1 : static_cast<int>(x);
+}
+// Sub-bin of s inside its bin `bin` (256 per bin; monotone in s within the bin).
+__device__ __forceinline__ int cut_sub(float s, float smax, int bin) {
+    const float f = ((smax - s) * 8.0f - static_cast<float>(bin)) * 256.0f;
+    return f >= 255.0f ? 255 : static_cast<int>(f);
+}
+// Order of the candidates: by score, then the lower slot first.
+__device__ __forceinline__ unsigned long long cut_key(float s, int i) {
+    return (static_cast<unsigned long long>(score_key(s)) << 32) | (0xffffffffu - static_cast<uint32_t>(i));
+}
+
+template <int NW>
+__device__ __forceinline__ void cut_sync() {
+    if constexpr (NW == 1) __syncwarp();
+    else __syncthreads();
+}
+
+// Warp 0: the bin where base + the cumulative mass of bins[0..] reaches target (bins are 8
+// rows of 32, lane j holding bins j + 32k, scanned as 8 independent warp scans); writes
+// the bin to *bin_out and base + the mass of the bins before it to *above_out, and leaves
+// the bins zero.  With target = 0 it first sets target = ceil(p * total), clamped to
+// [1, total], and writes it to *target_io.
+__device__ __forceinline__ void cut_locate(unsigned long long* bins, unsigned long long base, float p,
+                                           unsigned long long* target_io, int* bin_out,
+                                           unsigned long long* above_out) {
+    const int lane = threadIdx.x & 31;
+    unsigned long long v[8], in[8];
 #pragma unroll
-    for (int i = 0; i < kRouteWarps; ++i) mx = fmaxf(mx, sm.redf[i]);
-    if (mx == -INFINITY) return 0;   // no candidates (uniform: every thread read the same partials)
+    for (int k = 0; k < 8; ++k) {
+        v[k] = bins[lane + 32 * k];
+        bins[lane + 32 * k] = 0ull;
+        in[k] = v[k];
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const unsigned long long y = __shfl_up_sync(0xffffffffu, in[k], o);
+            if (lane >= o) in[k] += y;
+        }
+    unsigned long long rt[8], rp[8], tot = 0;   // row totals, exclusive prefix of the rows
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        rt[k] = __shfl_sync(0xffffffffu, in[k], 31);
+        rp[k] = tot;
+        tot += rt[k];
+    }
+    unsigned long long target = *target_io;
+    if (target == 0ull) {
+        target = static_cast<unsigned long long>(ceil(static_cast<double>(p) * static_cast<double>(tot)));
+        if (target < 1) target = 1;
+        if (target > tot) target = tot;
+    }
+    int kc = 7;
+#pragma unroll
+    for (int k = 7; k >= 0; --k)
+        if (base + rp[k] + rt[k] >= target) kc = k;
+    unsigned long long inc = 0, val = 0, rpc = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        if (k == kc) { inc = in[k]; val = v[k]; rpc = rp[k]; }
+    const uint32_t bal = __ballot_sync(0xffffffffu, base + rpc + inc >= target);
+    const int lc = bal ? __ffs(bal) - 1 : 31;
+    if (lane == lc) {
+        *bin_out = 32 * kc + lc;
+        *above_out = base + rpc + inc - val;
+        *target_io = target;
+    }
+}
+
+// Top-p cut over sc[0..nc) (invalid slots hold -inf) by the whole CTA: keeps the smallest
+// prefix, in descending score order with ties to the lower slot (= lower node id), whose
+// fixed-point mass reaches ceil(p * total); p >= 1 keeps every valid candidate.  mx is the
+// max valid score (-inf: none).  Writes the kept node ids, ascending, to out and returns their
+// count (in every thread).  cs.bins must be zero; they are left so.  kball, kpre: ceil(nc/32)
+// words each (shared memory, or the workspace for large nc); scan: kRouteWarps + 1 ints.
+//   1. every candidate's mass goes to its bin (1/8 nat below mx; masses below 2^-40 of the
+//      max's are 0 and skipped);
+//   2. warp 0 finds the bin where the cumulative mass reaches the target;
+//   3. the candidates of earlier bins are kept (one ballot word per 32 slots) and the crossing
+//      bin's members listed; when they are too many, their masses are binned again into 256
+//      sub-bins, the crossing sub-bin found, and its members listed instead;
+//   4. member k is kept iff the mass of the members ordered before it, plus the mass ordered
+//      before its (sub-)bin, is below the target (its bit joins the ballot words);
+//   5. a scan of the ballot words' counts places every word's kept ids, in slot order.
+template <typename NodeOf>
+__device__ int block_cut(const float* sc, int nc, float p, float mx, int32_t* out, CutSmem& cs, uint32_t* kball,
+                         int32_t* kpre, int* scan, NodeOf node_of) {
+    constexpr int NT = kRouteThreads;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    if (mx == -INFINITY || nc <= 0) return 0;   // uniform
     const bool keep_all = p >= 1.0f;
-    int cbin = kBins;                 // keep_all: every valid candidate is "before the crossing bin"
+    const int ngrp = (nc + 31) / 32;
+    int cbin = kCutBins, sbin = -1;
     if (!keep_all) {
-        // 2. mass per bin
-        for (int i = tid; i < nc; i += kRouteThreads) {
+        for (int i = t; i < nc; i += NT) {
             const float s = sc[i];
             if (s == -INFINITY) continue;
-            atomicAdd(&sm.bin_mass[score_bin(s, mx)], score_mass(s, mx));
+            const unsigned long long m = score_mass(s, mx);
+            if (m) atomicAdd(&cs.bins[cut_bin(s, mx)], m);
         }
+        if (t == 0) { cs.nm = 0; cs.target = 0; cs.sbin = -1; }
         __syncthreads();
-        // 3. one warp: total, target, the crossing bin and the mass of the bins before it.
-        //    Lane j first sums bins [32j, 32j+32) (independent partial sums), then the
-        //    crossing lane's 32 bins are scanned one per lane.
-        if (w == 0) {
-            const ulonglong2* bm = reinterpret_cast<const ulonglong2*>(sm.bin_mass + lane * 32);
-            unsigned long long p0 = 0, p1 = 0, p2 = 0, p3 = 0;
-#pragma unroll
-            for (int k = 0; k < 16; k += 2) {
-                const ulonglong2 x = bm[k], y = bm[k + 1];
-                p0 += x.x; p1 += x.y; p2 += y.x; p3 += y.y;
-            }
-            const unsigned long long ls = (p0 + p1) + (p2 + p3);
-            unsigned long long incl = ls;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            const unsigned long long tot = __shfl_sync(0xffffffffu, incl, 31);
-            unsigned long long target =
-                static_cast<unsigned long long>(ceil(static_cast<double>(p) * static_cast<double>(tot)));
-            if (target < 1) target = 1;
-            if (target > tot) target = tot;
-            const int J = __ffs(__ballot_sync(0xffffffffu, incl >= target)) - 1;
-            const unsigned long long base = __shfl_sync(0xffffffffu, incl - ls, J);   // bins before lane J's
-            const unsigned long long mb = sm.bin_mass[J * 32 + lane];
-            unsigned long long run = mb;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned long long y = __shfl_up_sync(0xffffffffu, run, o);
-                if (lane >= o) run += y;
-            }
-            const int k = __ffs(__ballot_sync(0xffffffffu, base + run >= target)) - 1;
-            if (lane == k) {
-                sm.cut_bin = J * 32 + k;
-                sm.cut_above = base + run - mb;
-                sm.cut_target = target;
-            }
-        }
+        if (w == 0) cut_locate(cs.bins, 0ull, p, &cs.target, &cs.cbin, &cs.above);
         __syncthreads();
-        cbin = sm.cut_bin;
-        // 4. gather the crossing bin's candidates
-        for (int i = tid; i < nc; i += kRouteThreads) {
-            const float s = sc[i];
-            if (s != -INFINITY && score_bin(s, mx) == cbin) {
-                const int t = atomicAdd(&sm.tie_n, 1);
-                if (t < kTieMax) sm.tie_slot[t] = i;
-            }
-        }
-        __syncthreads();
+        cbin = cs.cbin;
     }
-    const unsigned long long above = sm.cut_above, target = sm.cut_target;
-    const int nt = sm.tie_n;
-    // exact order inside the crossing bin: slot i of the bin is kept iff the mass of
-    // the bin's members ordered before it (higher score, or equal score and lower
-    // slot) plus the mass of the earlier bins stays below the target
-    auto before_in_bin = [&](int i, float si) -> unsigned long long {
-        unsigned long long bsum = 0;
-        if (nt <= kTieMax) {
-            for (int u = 0; u < nt; ++u) {
-                const int j = sm.tie_slot[u];
-                const float sj = sc[j];
-                if (sj > si || (sj == si && j < i)) bsum += score_mass(sj, mx);
-            }
-        } else {   // more members than the list holds: scan every slot
-            for (int j = 0; j < nc; ++j) {
-                const float sj = sc[j];
-                if (sj != -INFINITY && score_bin(sj, mx) == cbin && (sj > si || (sj == si && j < i)))
-                    bsum += score_mass(sj, mx);
-            }
-        }
-        return bsum;
-    };
-    auto kept = [&](int i) -> bool {
-        const float s = sc[i];
-        if (s == -INFINITY) return false;
-        if (keep_all) return true;
-        const int bn = score_bin(s, mx);
-        return bn < cbin || (bn == cbin && above + before_in_bin(i, s) < target);
-    };
-    // 5. compaction in slot order: one ballot per 32-slot group (warp w takes groups
-    //    w, w + 16, ...), an in-order prefix of the groups' counts by one warp, then writes
-    const int ngrp = (nc + 31) / 32;
+    // earlier bins as ballot words; the crossing bin's members listed
     for (int gi = w; gi < ngrp; gi += kRouteWarps) {
         const int i = gi * 32 + lane;
-        const uint32_t bal = __ballot_sync(0xffffffffu, i < nc && kept(i));
+        const float s = i < nc ? sc[i] : -INFINITY;
+        const int bn = s == -INFINITY ? kCutBins + 1 : (keep_all ? 0 : cut_bin(s, mx));
+        const uint32_t bal = __ballot_sync(0xffffffffu, bn < cbin);
         if (lane == 0) kball[gi] = bal;
-    }
-    __syncthreads();
-    if (w == 0) {
-        int run = 0;
-        for (int gi = 0; gi < ngrp; gi += 32) {
-            const int g2 = gi + lane;
-            const int c = g2 < ngrp ? __popc(kball[g2]) : 0;
-            int incl = c;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
+        if (bn == cbin) {
+            const int k = atomicAdd(&cs.nm, 1);
+            if (k < kCutMembers) {
+                cs.mkey[k] = cut_key(s, i);
+                cs.mmass[k] = score_mass(s, mx);
             }
-            if (g2 < ngrp) kpre[g2] = run + incl - c;
-            run += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) sm.redi[0] = run;
+    }
+    if (!keep_all) {
+        __syncthreads();
+        if (cs.nm > kCutMembers) {   // uniform: split the crossing bin
+            for (int i = t; i < nc; i += NT) {
+                const float s = sc[i];
+                if (s != -INFINITY && cut_bin(s, mx) == cbin) {
+                    const unsigned long long m = score_mass(s, mx);
+                    if (m) atomicAdd(&cs.bins[cut_sub(s, mx, cbin)], m);
+                }
+            }
+            __syncthreads();
+            if (t == 0) cs.nm = 0;
+            if (w == 0) cut_locate(cs.bins, cs.above, p, &cs.target, &cs.sbin, &cs.above);
+            __syncthreads();
+            sbin = cs.sbin;
+            for (int gi = w; gi < ngrp; gi += kRouteWarps) {   // earlier sub-bins join the ballots
+                const int i = gi * 32 + lane;
+                const float s = i < nc ? sc[i] : -INFINITY;
+                const bool in_bin = s != -INFINITY && cut_bin(s, mx) == cbin;
+                const int sb = in_bin ? cut_sub(s, mx, cbin) : 256;
+                const uint32_t bal = __ballot_sync(0xffffffffu, sb < sbin);
+                if (lane == 0 && bal) kball[gi] |= bal;
+                if (in_bin && sb == sbin) {
+                    const int k = atomicAdd(&cs.nm, 1);
+                    if (k < kCutMembers) {
+                        cs.mkey[k] = cut_key(s, i);
+                        cs.mmass[k] = score_mass(s, mx);
+                    }
+                }
+            }
+            __syncthreads();
+        }
+        // the members: thread k ranks member k against the others
+        const int nm = cs.nm;
+        const unsigned long long above = cs.above, target = cs.target;
+        if (nm <= kCutMembers) {
+            for (int k = t; k < nm; k += NT) {
+                const unsigned long long myk = cs.mkey[k];
+                unsigned long long before = 0;
+                for (int j = 0; j < nm; ++j)
+                    if (cs.mkey[j] > myk) before += cs.mmass[j];
+                if (above + before < target) {
+                    const int i = static_cast<int>(0xffffffffu - static_cast<uint32_t>(myk));
+                    atomicOr(&kball[i >> 5], 1u << (i & 31));
+                }
+            }
+        } else {   // more members than the list holds even after the split: scan every slot
+            for (int i = t; i < nc; i += NT) {
+                const float s = sc[i];
+                if (s == -INFINITY || cut_bin(s, mx) != cbin || (sbin >= 0 && cut_sub(s, mx, cbin) != sbin)) continue;
+                const unsigned long long myk = cut_key(s, i);
+                unsigned long long before = 0;
+                for (int j = 0; j < nc; ++j) {
+                    const float sj = sc[j];
+                    if (sj != -INFINITY && cut_bin(sj, mx) == cbin && (sbin < 0 || cut_sub(sj, mx, cbin) == sbin) &&
+                        cut_key(sj, j) > myk)
+                        before += score_mass(sj, mx);
+                }
+                if (above + before < target) atomicOr(&kball[i >> 5], 1u << (i & 31));
+            }
+        }
     }
     __syncthreads();
-    const int total = sm.redi[0];
+    // ballot words -> positions (a thread per word, in rounds of NT words) -> ids in slot order
+    int total = 0;
+    for (int g0 = 0; g0 < ngrp; g0 += NT) {
+        const int gi = g0 + t;
+        int tot;
+        const int x = block_exclusive_scan<kRouteWarps>(gi < ngrp ? __popc(kball[gi]) : 0, scan, &tot);
+        if (gi < ngrp) kpre[gi] = total + x;
+        total += tot;
+    }
+    __syncthreads();
     for (int gi = w; gi < ngrp; gi += kRouteWarps) {
         const uint32_t bal = kball[gi];
-        const int i = gi * 32 + lane;
-        if ((bal >> lane) & 1u) out[kpre[gi] + __popc(bal & ((1u << lane) - 1u))] = node_of(i);
+        if ((bal >> lane) & 1u) out[kpre[gi] + __popc(bal & ((1u << lane) - 1u))] = node_of(gi * 32 + lane);
     }
-    __syncthreads();
     return total;
 }
 
@@ -311,10 +376,12 @@ __device__ int top_p_select(const float* sc, int nc, float p, int32_t* out, Rout
 // With R planes per node, child r's plane p sits at kh[(r * R + p) * D]: the caller
 // passes the plane's first row, rs = R * D and bs = R, and calls once per plane with
 // first = (p == 0); later planes keep the max (the node's score is the max over planes).
+// With mxk, the max of the scores written goes into *mxk (order-mapped, atomicMax): pass it
+// on a candidate's last plane only.
 template <int D, int NVR>
 __device__ __forceinline__ void scan_children(const float* __restrict__ kh, const float* __restrict__ bh,
                                               int cnt, int b, const float* qv, float* __restrict__ out,
-                                              int rs = D, int bs = 1, bool first = true) {
+                                              int rs = D, int bs = 1, bool first = true, int* mxk = nullptr) {
     constexpr int VF = D / 32;
     const int lane = threadIdx.x & 31;
     float v[NVR];
@@ -352,12 +419,19 @@ __device__ __forceinline__ void scan_children(const float* __restrict__ kh, cons
         }
     }
     constexpr int low = 5 - H;
+    int mk = ord_key(-INFINITY);
     if ((lane & ((1 << low) - 1)) == 0) {
         const int r = (lane >> low) & (NVR - 1);
         if (r < b) {
             const float t = r < cnt ? v[0] + bh[static_cast<int64_t>(r) * bs] : -INFINITY;
-            out[r] = first ? t : fmaxf(out[r], t);
+            const float val = first ? t : fmaxf(out[r], t);
+            out[r] = val;
+            mk = ord_key(val);
         }
+    }
+    if (mxk) {
+        mk = __reduce_max_sync(0xffffffffu, mk);
+        if (lane == 0) atomicMax(mxk, mk);
     }
 }
 
@@ -367,8 +441,9 @@ template <int D, int NVR>
 __device__ __forceinline__ void scan_children2(const float* __restrict__ kh0, const float* __restrict__ bh0, int cnt0,
                                                const float* __restrict__ kh1, const float* __restrict__ bh1, int cnt1,
                                                int b, const float* qv, float* __restrict__ out0,
-                                               float* __restrict__ out1, int rs = D, int bs = 1,
-                                               bool first = true) {
+                                               float* __restrict__ out1, int* mxk0, int* mxk1) {
+    constexpr int rs = D, bs = 1;
+    constexpr bool first = true;
     constexpr int VF = D / 32;
     const int lane = threadIdx.x & 31;
     float x0[NVR][VF], x1[NVR][VF];
@@ -417,6 +492,7 @@ __device__ __forceinline__ void scan_children2(const float* __restrict__ kh0, co
         }
     }
     constexpr int low = 5 - H;
+    int mk0 = ord_key(-INFINITY), mk1 = ord_key(-INFINITY);
     if ((lane & ((1 << low) - 1)) == 0) {
         const int r = (lane >> low) & (NVR - 1);
         if (r < b) {
@@ -424,7 +500,17 @@ __device__ __forceinline__ void scan_children2(const float* __restrict__ kh0, co
             const float t1 = r < cnt1 ? v1[0] + bh1[static_cast<int64_t>(r) * bs] : -INFINITY;
             out0[r] = first ? t0 : fmaxf(out0[r], t0);
             out1[r] = first ? t1 : fmaxf(out1[r], t1);
+            mk0 = ord_key(t0);
+            mk1 = ord_key(t1);
         }
+    }
+    if (mxk0) {
+        mk0 = __reduce_max_sync(0xffffffffu, mk0);
+        if (lane == 0) atomicMax(mxk0, mk0);
+    }
+    if (mxk1) {
+        mk1 = __reduce_max_sync(0xffffffffu, mk1);
+        if (lane == 0) atomicMax(mxk1, mk1);
     }
 }
 
@@ -489,9 +575,8 @@ __device__ void add_dropped(const float* sc, const int32_t* par, int np_par, int
         }
     }
     lw = warp_sum(lw);
-    // cross-warp sum: [warp][D] values through the (idle) block-cut bins, masses in pr_lw
-    static_assert(kRouteWarps * 128 * sizeof(float) <= sizeof(RouteSmem::bin_mass), "scratch fits the bins");
-    float* red = reinterpret_cast<float*>(sm.bin_mass);
+    // cross-warp sum: [warp][D] values through vred, masses in pr_lw
+    float* red = sm.vred;
 #pragma unroll
     for (int f = 0; f < VF; ++f) red[w * D + lane * VF + f] = acc[f];
     if (lane == 0) sm.pr_lw[w] = lw;
@@ -513,14 +598,21 @@ __device__ void add_dropped(const float* sc, const int32_t* par, int np_par, int
     __syncthreads();
 }
 
-// The top-down walk of one decode query (the body of route_decode_kernel).
+// The top-down walk of one decode query (the body of route_decode_kernel).  With
+// `region` != 0 (fuse_plan) the kept nodes of every level are OR'd into the bitmaps of
+// the cluster's CTA 0 (shared::cluster address of its plan region): level 1 into head
+// `head`'s plan bitmap, level l >= 2 into the level's bitmap of kept nodes.  The walk
+// then waits on the cluster barrier that CTA 0 arrived on after clearing the region,
+// once, right after the top level's cut (before its first remote write).
 template <typename T, int D, int NVR, bool MP, bool VS>
 __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, int cta, int64_t row, int64_t slice,
-                                           int64_t N, int64_t Ntree) {
+                                           int64_t N, int64_t Ntree, uint32_t region, int head, float q_in) {
     constexpr int VF = D / 32;   // fp32 summary elements per lane
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     (void)N;
-    if (tid < D) sm.q[tid] = to_f32(static_cast<const T*>(a.Q)[row * D + tid]) * a.scale;
+    if (tid < D) sm.q[tid] = q_in * a.scale;   // q_in: element tid of the query (loaded by the caller)
+    if (tid < 2) sm.mxkey[tid] = ord_key(-INFINITY);
+    for (int i = tid; i < kCutBins; i += kRouteThreads) sm.cut.bins[i] = 0ull;
     constexpr bool vsum = VS && !MP;   // value summaries (R = 1)
     if constexpr (vsum) {
         if (tid < D) sm.pr_acc[tid] = 0.f;
@@ -544,6 +636,11 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
     int np = static_cast<int>((n[L - 1] + b - 1) / b);
     if (np > kParentsSmem) cur = 2;
     for (int i = tid; i < np; i += kRouteThreads) bufs[cur][i] = i;
+    // the level below the top, when small, is scored in the same pass as the top level (its
+    // candidates are children of top nodes, known before the top level's cut): one round trip
+    // to memory less; its scores wait in sm.spec for the cut to pick the kept parents' children
+    const bool spec = L >= 2 && n[L - 2] <= kSpecMax;
+    const int nspec = spec ? static_cast<int>(n[L - 1]) : 0;   // parents of the level below the top
     __syncthreads();
 
     int64_t scored = 0;
@@ -560,49 +657,89 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
         const int R = MP ? a.tree.R : 1;
         const float* kh = a.tree.khat[l - 1] + slice * ncap * R * D;
         const float* bh = a.tree.bhat[l - 1] + slice * ncap * R;
-        // ---- scan: one warp per kept parent, its b child rows of D fp32 (per plane, max over planes)
-        for (int pi = w; pi < np; pi += 2 * kRouteWarps) {
-            const int pj = pi + kRouteWarps;   // a second parent in the same round, if any
-            const int64_t c0 = static_cast<int64_t>(par[pi]) * b;
-            const int cnt0 = static_cast<int>(min(static_cast<int64_t>(b), nl - c0));
-            if constexpr (!MP) {
-                if (pj < np) {
-                    const int64_t c1 = static_cast<int64_t>(par[pj]) * b;
-                    const int cnt1 = static_cast<int>(min(static_cast<int64_t>(b), nl - c1));
-                    scan_children2<D, NVR>(kh + c0 * D, bh + c0, cnt0, kh + c1 * D, bh + c1, cnt1, b, qv,
-                                           sc + static_cast<int64_t>(pi) * b, sc + static_cast<int64_t>(pj) * b);
+        int* mxk = &sm.mxkey[l & 1];   // this level's max score, found by the scan
+        // the other slot is the next level's: its last reader, the cut one level up, is done
+        if (tid == 0) sm.mxkey[(l + 1) & 1] = ord_key(-INFINITY);
+        if (spec && l == L - 1) {
+            // ---- the scores were read with the top level: the kept parents' children
+            int mk = ord_key(-INFINITY);
+            for (int i = tid; i < nc; i += kRouteThreads) {
+                const int64_t c = static_cast<int64_t>(par[i / b]) * b + i % b;
+                const float v = c < nl ? sm.spec[c] : -INFINITY;
+                sc[i] = v;
+                mk = max(mk, ord_key(v));
+            }
+            mk = __reduce_max_sync(0xffffffffu, mk);
+            if (lane == 0) atomicMax(mxk, mk);
+        } else {
+            // ---- scan: one warp per parent (a job), its b child rows of D fp32 (per plane, max over
+            //      planes); at the top level, jobs past the top's parents are the spec level's parents
+            const int jobs = np + (l == L ? nspec : 0);
+            const int64_t ncap_s = spec && l == L ? a.tree.ncap[L - 2] : 0;
+            const float* kh_s = spec && l == L ? a.tree.khat[L - 2] + slice * ncap_s * R * D : nullptr;
+            const float* bh_s = spec && l == L ? a.tree.bhat[L - 2] + slice * ncap_s * R : nullptr;
+            // a job's max goes to this level's max, except the spec level's (its candidates are
+            // only the kept top nodes' children, whose max the copy above takes)
+            auto job = [&](int j, const float*& k0, const float*& b0, int& cnt, float*& out, int*& mx) {
+                if (j < np) {
+                    const int64_t c0 = static_cast<int64_t>(par[j]) * b;
+                    cnt = static_cast<int>(min(static_cast<int64_t>(b), nl - c0));
+                    k0 = kh + c0 * R * D;
+                    b0 = bh + c0 * R;
+                    out = sc + static_cast<int64_t>(j) * b;
+                    mx = mxk;
                 } else {
-                    scan_children<D, NVR>(kh + c0 * D, bh + c0, cnt0, b, qv, sc + static_cast<int64_t>(pi) * b);
+                    const int64_t c0 = static_cast<int64_t>(j - np) * b;
+                    cnt = static_cast<int>(min(static_cast<int64_t>(b), n[L - 2] - c0));
+                    k0 = kh_s + c0 * R * D;
+                    b0 = bh_s + c0 * R;
+                    out = sm.spec + c0;
+                    mx = nullptr;
                 }
-                continue;
-            }
-            if (pj < np) {
-                const int64_t c1 = static_cast<int64_t>(par[pj]) * b;
-                const int cnt1 = static_cast<int>(min(static_cast<int64_t>(b), nl - c1));
+            };
+            for (int ji = w; ji < jobs; ji += 2 * kRouteWarps) {
+                const int jj = ji + kRouteWarps;   // a second job in the same round, if any
+                const float *k0, *b0, *k1 = nullptr, *b1 = nullptr;
+                int cnt0, cnt1 = 0;
+                float *o0, *o1 = nullptr;
+                int *m0, *m1 = nullptr;
+                job(ji, k0, b0, cnt0, o0, m0);
+                if (jj < jobs) job(jj, k1, b1, cnt1, o1, m1);
+                if constexpr (!MP) {
+                    if (jj < jobs) scan_children2<D, NVR>(k0, b0, cnt0, k1, b1, cnt1, b, qv, o0, o1, m0, m1);
+                    else scan_children<D, NVR>(k0, b0, cnt0, b, qv, o0, D, 1, true, m0);
+                    continue;
+                }
+                if (jj < jobs)
+                    for (int pl = 0; pl < R; ++pl)
+                        scan_children<D, NVR>(k1 + pl * D, b1 + pl, cnt1, b, qv, o1, R * D, R, pl == 0,
+                                              pl == R - 1 ? m1 : nullptr);
                 for (int pl = 0; pl < R; ++pl)
-                    scan_children<D, NVR>(kh + (c1 * R + pl) * D, bh + c1 * R + pl, cnt1, b, qv,
-                                          sc + static_cast<int64_t>(pj) * b, R * D, R, pl == 0);
+                    scan_children<D, NVR>(k0 + pl * D, b0 + pl, cnt0, b, qv, o0, R * D, R, pl == 0,
+                                          pl == R - 1 ? m0 : nullptr);
             }
-            for (int pl = 0; pl < R; ++pl)
-                scan_children<D, NVR>(kh + (c0 * R + pl) * D, bh + c0 * R + pl, cnt0, b, qv,
-                                      sc + static_cast<int64_t>(pi) * b, R * D, R, pl == 0);
         }
         __syncthreads();
         // ---- top-p cut and compaction of the kept node ids
         const int np_par = np;
         const int nxt = nc <= kParentsSmem ? (cur == 0 ? 1 : 0) : (cur == 2 ? 3 : 2);
         auto node_of = [par, b](int i) { return static_cast<int32_t>(par[i / b] * b + i % b); };
-        if (nc <= 64) {
-            if (w == 0) {
-                const int c = top_p_small(sc, nc, a.p[l - 1], bufs[nxt], node_of);
-                if (lane == 0) sm.redi[0] = c;
+        {
+            const bool big = (nc + 31) / 32 > kScoresSmem / 32;   // ballot words in the workspace
+            np = block_cut(sc, nc, a.p[l - 1], key_ord(*mxk), bufs[nxt], sm.cut, big ? ws_kb : sm.keep_ballot,
+                           big ? reinterpret_cast<int32_t*>(ws_kb) + a.kb_cap : sm.keep_prefix, sm.scan, node_of);
+        }
+        __syncthreads();
+        if (region) {
+            // the kept nodes into CTA 0's bitmaps: the level's kept set (for the count of distinct
+            // nodes read), or at level 1 this head's selected blocks (the gather plan)
+            if (l == L) cluster_wait();   // CTA 0 has cleared the region
+            const uint32_t bm = region + 4u * static_cast<uint32_t>(l == 1 ? head * a.plan.words : a.lvl_off[l - 1]);
+            const int32_t* kept = bufs[nxt];
+            for (int i = tid; i < np; i += kRouteThreads) {
+                const int32_t x = kept[i];
+                dsmem_or(bm + 4u * static_cast<uint32_t>(x >> 5), 1u << (x & 31));
             }
-            __syncthreads();
-            np = sm.redi[0];
-        } else {
-            const bool big = (nc + 31) / 32 > kScoresSmem / 32;
-            np = top_p_select(sc, nc, a.p[l - 1], bufs[nxt], sm, big ? ws_kb : sm.keep_ballot,
-                              big ? reinterpret_cast<int32_t*>(ws_kb) + a.kb_cap : sm.keep_prefix, node_of);
         }
         if constexpr (vsum)
             add_dropped<D, NVR>(sc, par, np_par, b, nl, bufs[nxt], np, a.tree.vhat[l - 1] + slice * ncap * D, sm);
@@ -624,41 +761,83 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
     }
 }
 
+// Distinct tree nodes the group's route read: every top node, the level below the top
+// whole when it was read with the top (kSpecMax), and below that the children of the
+// nodes any head kept one level up (the level bitmaps in the plan region).  Warp 0 of CTA 0.
+__device__ int64_t route_scanned(const RouteArgs& a, const uint32_t* region, int64_t Ntree) {
+    const int lane = threadIdx.x & 31;
+    int64_t n[kMaxLevels];
+    const int L = tree_levels(Ntree, a.B, a.b, a.L_fixed, n);
+    const bool spec = L >= 2 && n[L - 2] <= kSpecMax;
+    int64_t tot = n[L - 1] + (spec ? n[L - 2] : 0);
+    for (int l = spec ? L - 1 : L; l >= 2; --l) {
+        const uint32_t* bm = region + a.lvl_off[l - 1];
+        const int64_t words = (n[l - 1] + 31) / 32, last = n[l - 1] - 1;
+        int64_t c = 0;
+        for (int64_t i = lane; i < words; i += 32) c += __popc(bm[i]);
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        tot += c * a.b;
+        if ((bm[last >> 5] >> (last & 31)) & 1u) tot -= a.b - (n[l - 2] - last * a.b);   // partial last parent
+    }
+    return tot;
+}
 
 // One CTA per (sequence, query head): the whole top-down walk of one decode query.
 // NVR = b rounded up to a power of two (4, 8, 16 or 32).
 // MP: nodes carry several reference-query planes (R > 1); R = 1 compiles the
 // single-plane scan alone.  VS: the tree holds value summaries (R = 1): the nodes the
 // cut drops are summed into a per-query partial.
+// fuse_plan: launched as clusters of G CTAs, the G query heads of one (sequence, KV
+// head) (cluster rank = head).  CTA 0 clears its plan region, the heads OR their kept
+// nodes into it (DSMEM), and after a cluster barrier CTA 0 builds the group's gather
+// plan from its own shared memory.
 template <typename T, int D, int NVR, bool MP, bool VS = false>
 __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     RouteSmem& sm = *reinterpret_cast<RouteSmem*>(smem_raw);
+    uint32_t* region = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RouteSmem));
     const int tid = threadIdx.x;
     const int cta = blockIdx.x;
     const int s = cta / a.Hq, hq = cta % a.Hq;
-    const int kv = hq / (a.Hq / a.Hkv);
+    const int G = a.Hq / a.Hkv;
+    const int kv = hq / G;
     const int64_t slice = static_cast<int64_t>(s) * a.Hkv + kv;
     const int64_t row = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + hq;
+    const bool fused = a.fuse_plan != 0;
+    // the query, the key count and the tree count in one round trip to memory
+    const float q_in = tid < D ? to_f32(static_cast<const T*>(a.Q)[row * D + tid]) : 0.f;
+    const uint32_t rank = fused ? cluster_rank() : 0u;
+    if (fused) {
+        if (rank == 0)
+            for (int i = tid; i < a.region_words; i += kRouteThreads) region[i] = 0u;
+        cluster_arrive();   // waited on by the walk before its first remote write
+    }
     const int64_t N = a.N[s];
     const int64_t Ntree = a.tree.n_tree[s];
-    const bool valid = !(N < 1 || N > a.N_cap || Ntree > N || Ntree < 0);
+    const bool valid = !(N < 1 || N > a.N_cap || Ntree > N || Ntree < 0);   // uniform over the cluster
     if (!valid) {
         if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.sel_count[row] = 0; a.cand[row] = 0; }
+        if (fused) cluster_wait();
     } else {
-        route_walk<T, D, NVR, MP, VS>(a, sm, cta, row, slice, N, Ntree);
+        route_walk<T, D, NVR, MP, VS>(a, sm, cta, row, slice, N, Ntree, fused ? cluster_map(region, 0) : 0u,
+                                      static_cast<int>(rank), q_in);
     }
-    if (a.fuse_plan) {
-        // the last of the group's G query-head CTAs builds the group's gather plan; the
-        // count's release publishes this CTA's selection (ordered before it by the barrier),
-        // its acquire makes the other heads' selections visible to the last CTA
-        __syncthreads();
-        if (tid == 0)
-            sm.plan_last = atomic_add_acq_rel_gpu(&a.grp_done[slice], 1u) == static_cast<uint32_t>(a.Hq / a.Hkv - 1);
-        __syncthreads();
-        if (sm.plan_last) {
-            plan_group(a.plan, static_cast<int>(slice), reinterpret_cast<uint32_t*>(sm.scores), sm.scan, N, Ntree);
-            if (tid == 0) a.grp_done[slice] = 0u;
+    if (fused) {
+        // every head's kept nodes are in CTA 0's region; the other CTAs are done with it
+        cluster_arrive();
+        cluster_wait();
+        if (rank == 0) {
+            if (valid) {
+                plan_emit(a.plan, static_cast<int>(slice), region, sm.scan, N, Ntree);
+                if (tid < 32) {
+                    const int64_t c = route_scanned(a, region, Ntree);
+                    if (tid == 0) a.scanned[slice] = static_cast<int32_t>(c);
+                }
+            } else if (tid == 0) {
+                a.plan.n_items[slice] = 0;
+                a.plan.rows[slice] = 0;
+                a.scanned[slice] = 0;
+            }
         }
     }
 }

@@ -40,7 +40,7 @@ class ZhaConfig(ctypes.Structure):
 
 EXPORTS = ["zha_levels_cap", "zha_tree_bytes", "zha_tree_level", "zha_tree_level_v", "zha_tree_count_offset", "zha_workspace_bytes", "zha_workspace_init", "zha_workspace_stats", "zha_attend_kernel", "zha_build",
            "zha_extend", "zha_append", "zha_route", "zha_attend", "zha_attend_noalloc", "zha_decode", "zha_dense", "zha_get_status",
-           "zha_last_error"]
+           "zha_set_wait_limit", "zha_last_error"]
 
 
 def lib():
@@ -62,7 +62,7 @@ def lib():
         "zha_tree_count_offset": [C, P],
         "zha_workspace_bytes": [C, I32, P],
         "zha_workspace_init": [C, P, SZ, P],
-        "zha_workspace_stats": [C, I32, P, P],
+        "zha_workspace_stats": [C, I32, P, P, P],
         "zha_attend_kernel": [C, I32, P],
         "zha_build": [C, P, P, P, P, P, P],
         "zha_extend": [C, P, P, P, P, P],
@@ -73,6 +73,7 @@ def lib():
         "zha_decode": [C, P, P, P, P, P, P, P, P, P, SZ, P],
         "zha_dense": [C, P, P, P, I32, P, P, P, SZ, P],
         "zha_get_status": [P, I32, P],
+        "zha_set_wait_limit": [ctypes.c_uint64, P],
     }
     for name, args in sig.items():
         fn = getattr(L, name)
@@ -191,12 +192,17 @@ def workspace_bytes(cfg: Config, n_q: int = 1) -> int:
     return v.value
 
 
-def workspace_stats_view(cfg: Config, ws: torch.Tensor, n_q: int = 1) -> tuple[torch.Tensor, torch.Tensor]:
-    """(rows [batch*Hkv] keys gathered per group, cand [batch*n_q*Hq] nodes scored per query head) int32 views."""
-    ro, co = ctypes.c_size_t(), ctypes.c_size_t()
-    _check(lib().zha_workspace_stats(ctypes.byref(cfg.c()), n_q, ctypes.byref(ro), ctypes.byref(co)))
+def workspace_stats_view(cfg: Config, ws: torch.Tensor, n_q: int = 1):
+    """int32 views (rows [batch*Hkv] keys gathered per group, cand [batch*n_q*Hq] nodes scored per
+    query head, scanned [batch*Hkv] distinct nodes the route read per group; with n_q > 1 scanned
+    is cand)."""
+    ro, co, so = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().zha_workspace_stats(ctypes.byref(cfg.c()), n_q, ctypes.byref(ro), ctypes.byref(co),
+                                     ctypes.byref(so)))
     g, c = cfg.batch * cfg.Hkv, cfg.batch * n_q * cfg.Hq
-    return (ws[ro.value:ro.value + 4 * g].view(torch.int32), ws[co.value:co.value + 4 * c].view(torch.int32))
+    sn = c if n_q > 1 else g
+    return (ws[ro.value:ro.value + 4 * g].view(torch.int32), ws[co.value:co.value + 4 * c].view(torch.int32),
+            ws[so.value:so.value + 4 * sn].view(torch.int32))
 
 
 def alloc_tree(cfg: Config, device="cuda") -> torch.Tensor:
@@ -215,8 +221,13 @@ def attend_kernel(cfg: Config, n_q: int = 1) -> str:
 
 def alloc_workspace(cfg: Config, n_q: int = 1, device="cuda", stream=None) -> torch.Tensor:
     ws = torch.empty(workspace_bytes(cfg, n_q), dtype=torch.uint8, device=device)
-    _check(lib().zha_workspace_init(ctypes.byref(cfg.c()), _ptr(ws), ws.numel(), _stream(stream)))
+    workspace_init(cfg, ws, stream)
     return ws
+
+
+def workspace_init(cfg: Config, ws: torch.Tensor, stream=None):
+    """Zeroes a workspace (after allocation, or after a call that raised ZHA_ERR_TIMEOUT)."""
+    _check(lib().zha_workspace_init(ctypes.byref(cfg.c()), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def build(cfg: Config, K, qref, N, tree, stream=None, V=None):
@@ -250,8 +261,10 @@ def attend(cfg: Config, K, V, tree, Q, N, sel, sel_count, O, ws, n_q: int = 1, s
                             _ptr(sel_count), sel_cap, _ptr(O), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def attend_noalloc(cfg: Config, K, V, tree, Q, N, sel, sel_count, O, n_q: int = 1, stream=None):
-    """zha_attend without a workspace: the library's static device scratch (see include/zha.h)."""
+def attend_noalloc(cfg: Config, K, V, tree, Q, N, sel, sel_count, O, stream=None, n_q: int = 1):
+    """zha_attend of decode queries (n_q = 1) without a workspace: the library's static device
+    scratch (see include/zha.h).  n_q is passed through only so that a caller can see the
+    library's own refusal of a chunked prefill."""
     _check(lib().zha_attend_noalloc(ctypes.byref(cfg.c()), _ptr(K), _ptr(V), _ptr(tree), _ptr(Q), n_q, _ptr(N),
                                     _ptr(sel), _ptr(sel_count), sel.shape[-1], _ptr(O), _stream(stream)))
 
@@ -274,3 +287,11 @@ def get_status(clear: bool = True, stream=None) -> int:
 
 def status_names(bits: int) -> list[str]:
     return [STATUS[c] for c in STATUS if c and bits & (1 << c)]
+
+
+def set_wait_limit(ns: int) -> int:
+    """Sets the bound (ns) of the tensor-core decode attention's waits on its other warps'
+    progress; returns the previous bound (see include/zha.h, zha_set_wait_limit)."""
+    prev = ctypes.c_uint64()
+    _check(lib().zha_set_wait_limit(int(ns), ctypes.byref(prev)))
+    return prev.value

@@ -52,7 +52,7 @@ typedef struct CUstream_st *zha_stream_t;
 typedef enum {
     ZHA_OK = 0,
     ZHA_ERR_INVALID_ARG = 1,  /* null pointer, bad size or inconsistent config       */
-    ZHA_ERR_UNSUPPORTED = 2,  /* valid but not built: d not in {64,128}, R > 1, ...    */
+    ZHA_ERR_UNSUPPORTED = 2,  /* valid but not built: d not in {64,128}, R > 16, ...   */
     ZHA_ERR_CAPACITY = 3,     /* device: cache full (N == N_cap) or sel_cap exceeded   */
     ZHA_ERR_CUDA = 4,         /* a CUDA runtime call failed (message in last_error)    */
     ZHA_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up (the call returned)    */
@@ -76,7 +76,7 @@ typedef struct zha_config {
     int32_t Hkv;      /* KV heads; Hq/Hkv in {1, 2, 4}                        */
     int32_t B;        /* leaf block, 1..256 (chunked prefill: 64)             */
     int32_t b;        /* branching factor, 2..32                              */
-    int32_t R;        /* reference queries per node (GPU path: 1)             */
+    int32_t R;        /* reference queries (planes) per node, 1..16           */
     int32_t dtype;    /* zha_dtype of K, V, Q, k_new, v_new                   */
     int32_t batch;    /* sequences                                            */
     int64_t N_cap;    /* rows allocated per (sequence, KV head) in K and V    */
@@ -130,9 +130,14 @@ int zha_workspace_init(const zha_config *cfg, void *ws, size_t ws_bytes, zha_str
  * the path touches: byte offsets of int32 rows[batch*Hkv] (keys gathered per
  * (sequence, KV head) by the last zha_attend / zha_dense plan; with n_q > 1 the
  * number of 64-key blocks the tensor-core attention loaded, each for up to 128
- * query rows) and int32 cand[batch][n_q][Hq] (tree nodes scored over all levels
- * by the last zha_route). */
-int zha_workspace_stats(const zha_config *cfg, int32_t n_q, size_t *rows_offset, size_t *cand_offset);
+ * query rows), int32 cand[batch][n_q][Hq] (tree nodes scored over all levels
+ * for each query head by the last zha_route) and int32 scanned[batch*Hkv]
+ * (decode: the distinct tree nodes the last zha_route read per (sequence, KV
+ * head), over the query heads that share the KV head; 0 when the route could
+ * not count them, for a cache too large for its on-chip bitmaps; with n_q > 1
+ * the offset of cand again, each row reading its own candidates). */
+int zha_workspace_stats(const zha_config *cfg, int32_t n_q, size_t *rows_offset, size_t *cand_offset,
+                        size_t *scanned_offset);
 
 /* Which attention kernel zha_attend (and zha_decode, zha_attend_noalloc) runs for
  * cfg and n_q: *kind = 0 for the CUDA-core decode kernel, 1 for the tensor-core
@@ -237,14 +242,18 @@ int zha_attend(const zha_config *cfg, const void *K, const void *V, const void *
  * device and fragment a pre-reserved pool).  The pages describe no counterpart;
  * it is a convenience of this library.
  *
- * Arguments, layouts and results are those of zha_attend (sel must not be
- * NULL); the caller still owns K, V, tree, Q, N, sel, sel_count and O.  The
+ * Decode only: n_q must be 1 (a chunked prefill, n_q > 1, is refused with
+ * ZHA_ERR_UNSUPPORTED before anything runs), and vsum = 1 is refused likewise.
+ * Otherwise arguments, layouts and results are those of zha_attend with n_q = 1
+ * (sel must not be NULL), bit for bit; the caller still owns K, V, tree, Q, N,
+ * sel, sel_count and O.  The
  * scratch is one static device array of 16 MiB inside the library, present on
  * every GPU that loads the library until the process exits.  A configuration
  * whose scratch (zha_workspace_bytes) exceeds 16 MiB is refused with
  * ZHA_ERR_WORKSPACE before anything runs.  The call allocates nothing.
- * - The first call on a device looks the array's device address up with
- *   cudaGetSymbolAddress; make that first call before any stream capture.
+ * - The first call on a device (in each CUDA context of that device) looks
+ *   the array's device address up with cudaGetSymbolAddress; make that first
+ *   call before any stream capture.
  * - All calls on a device share the array and it keeps the last call's
  *   contents: calls that may overlap on the GPU (two streams, or two host
  *   threads) race on it and must be serialised by the caller.
@@ -271,6 +280,19 @@ int zha_dense(const zha_config *cfg, const void *K, const void *V, const void *Q
  * device: bit (1 << code) for each zha_status code raised on the device since
  * the last clear.  Synchronises `stream`. */
 int zha_get_status(int32_t *status_bits, int32_t clear, zha_stream_t stream);
+
+/* Bound, in nanoseconds, of the tensor-core decode attention's waits on the
+ * progress of its other warps (default 2e9; it applies to kernels launched
+ * after the call, on every device, and returns the previous bound in
+ * *previous when that is not NULL).  A control for testing the failure path:
+ * with 0, a wait that is not already satisfied gives up at once.  A wait that
+ * gives up raises ZHA_ERR_TIMEOUT in the device status; the CTA then stops
+ * work, lets the copies and MMAs it issued itself complete (those waits keep
+ * the 2 s bound), frees its tensor memory and returns, so the call always
+ * ends.  The output of that call is undefined, and so are the merge counters
+ * it leaves in the workspace: re-initialise the workspace (zha_workspace_init)
+ * before reusing it.  The other kernels' waits keep the 2 s bound. */
+int zha_set_wait_limit(uint64_t ns, uint64_t *previous);
 
 /* Message of the calling thread's last failed call ("" if none). */
 const char *zha_last_error(void);

@@ -150,17 +150,15 @@ void oracle_build_v(const void *K, const void *V, int dtype, int64_t N, int d, i
             for (int r = 0; r < R; ++r) {
                 const double *q = qref + ((int64_t)(l - 1) * R + r) * d;
                 for (int64_t c = c0; c < c1; ++c) {
-                    /* The child's best plane is an integer decided by floating point: it is
-                     * decided on the estimates rounded to fp32 (the GPU kernels' precision;
-                     * ties to the lower plane), while its estimate and key stay fp64. */
+                    /* The child's estimate is the max over its planes, taken exactly
+                     * ([HTI] Tree Construction: max over r of t_r); r*(c) is the plane
+                     * that attains it, the lowest one on an exact tie. */
                     double best = -INFINITY;
-                    float bestf = -INFINITY;
                     int br = 0;
                     for (int r2 = 0; r2 < R; ++r2) {
                         int64_t node = off_child + c;
                         double t = scale * dot(q, khat + (node * R + r2) * d, d) + bhat[node * R + r2];
-                        float tf = (float)t;
-                        if (tf > bestf) { bestf = tf; best = t; br = r2; }
+                        if (t > best) { best = t; br = r2; }
                     }
                     z[c - c0] = best;
                     rs[c - c0] = br;

@@ -79,6 +79,9 @@ def test_null_pointers_and_small_workspace_are_refused_on_the_host(lib):
         zha.workspace_bytes(cfg(batch=1, N_cap=4096, vsum=1), 64)
     assert e.value.code == 2
     assert lib.zha_attend_noalloc(cv, 1, 1, 1, 1, 1, 1, 1, 1, 16, 1, None) == 2   # nor the no-alloc call
+    # the no-alloc call is decode only: a chunked prefill (n_q > 1) is refused before anything runs
+    assert lib.zha_attend_noalloc(cc, 1, 1, 1, 1, 64, 1, 1, 1, 16, 1, None) == 2
+    assert "n_q = 1" in lib.zha_last_error().decode()
     off = ctypes.c_size_t()
     assert lib.zha_tree_level_v(cc, 1, ctypes.byref(off)) == 1             # vsum = 0: no vhat
     assert lib.zha_tree_level_v(cv, 1, ctypes.byref(off)) == 0
@@ -95,3 +98,12 @@ def test_null_pointers_and_small_workspace_are_refused_on_the_host(lib):
     assert lib.zha_decode(cc, None, None, None, None, None, None, None, None, 256, need, None) == 1
     assert lib.zha_dense(cc, 1, 1, 1, 1, 1, 1, None, need, None) == 1
     assert "ws" in lib.zha_last_error().decode()
+
+
+def test_wait_limit_setter_round_trips(lib):
+    prev = zha.set_wait_limit(12345)
+    try:
+        assert zha.set_wait_limit(prev) == 12345
+    finally:
+        zha.set_wait_limit(prev)
+    assert prev == 2_000_000_000

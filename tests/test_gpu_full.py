@@ -12,7 +12,12 @@ from tests.zha_parity import Report, assert_status_clean, check_queries, compare
 
 pytestmark = pytest.mark.gpu
 
-CASES = {"decode1m": ([(0, 0), (3, 7)], 2), "decode8m": ([(0, 5), (0, 1)], 2)}
+CASES = {"decode1m": ([(0, 0), (1, 3), (2, 6), (3, 7)], 4), "decode8m": ([(0, 5), (0, 1), (0, 6)], 4)}
+# Least share of the sampled queries whose oracle cut margin exceeds 1e-4 at every level (those
+# must be bit-exact).  The margin is the minimum over the walk's levels, so the deeper 8M tree
+# (five levels against four) leaves fewer queries above it: 19 of 48 in a recorded run, every
+# one of the 48 index sets equal to the oracle's nonetheless.
+MIN_EXACT_SHARE = {"decode1m": 2, "decode8m": 4}   # at least queries // this
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
@@ -43,6 +48,7 @@ def test_decode_full_size_sampled(name):
     zha.get_status(clear=True)
     zha.build(cfg, K, data["qref"], N, tree)
     rep = Report()
+    trees = {}   # the tree depends on N only through its complete blocks: one oracle build per block count
     for i in range(steps):
         q = Q[i].reshape(w.batch, 1, w.Hq, w.d).contiguous()
         zha.append(cfg, K, V, kn[i].contiguous(), vn[i].contiguous(), N, tree)
@@ -53,20 +59,22 @@ def test_decode_full_size_sampled(name):
         o, sl, ct = O_.cpu(), sel.cpu(), cnt.cpu()
         for (s, h) in SAMPLES:
             Kh, Vh = host[(s, h)]
-            ot = oracle_tree(Kh, n_now, cfg, qref[h])
+            key = (s, h, n_now // w.B)
+            if key not in trees:
+                trees[key] = oracle_tree(Kh, n_now, cfg, qref[h])
+            ot = trees[key]
             if i == steps - 1:
                 compare_tree(cfg, tree, ot, s, h)
             hs = slice(h * w.G, (h + 1) * w.G)
             check_queries(cfg, ot, Kh, Vh, n_now - 1, Qh[i, s, hs].float(), sl[s, 0, hs], ct[s, 0, hs],
                           o[s, 0, hs].numpy(), w.p, rep)
+    print(f"{name} sampled: {rep.summary()}; mean keys read per head {np.mean(rep.read_keys):.0f} "
+          f"({np.mean(rep.read_keys) / w.N * 100:.2f}% of the cache)")
     rep.check()
-    assert rep.exact_required >= 1, rep
+    assert rep.exact_required >= rep.queries // MIN_EXACT_SHARE[name], rep
     assert_status_clean()
     del K, V, data, tree, ws
     torch.cuda.empty_cache()
-    print(f"{name} sampled: {rep.exact_required}/{rep.queries} index sets checked bit-exact "
-          f"({rep.low_margin} below the margin), mean keys read per head "
-          f"{np.mean(rep.read_keys):.0f} ({np.mean(rep.read_keys) / w.N * 100:.2f}% of the cache)")
 
 
 def test_prefill_256k_full_size_sampled():

@@ -14,10 +14,11 @@ from hierarchical_tree_indexed_b200 import workloads as W
 from hierarchical_tree_indexed_b200 import zha
 from tests.test_gpu_prefill import Prefill, check_prefill
 from oracle import oracle as O
-from tests.zha_parity import (SUMMARY_ATOL, Decoder, Report, assert_status_clean, check_queries, compare_tree,
-                              oracle_tree)
+from tests.zha_parity import (MARGIN, SUMMARY_ATOL, Decoder, Report, assert_status_clean, check_queries,
+                              compare_tree, oracle_tree)
 
 PLANE_GAP = 1e-5    # a child's two best planes closer than this: the plane choice is a near-tie
+EXCUSED_MAX = 0.10  # at most this fraction of the upper levels' node planes may be near-tied
 
 
 def compare_tree_planes(cfg, tree, ot, s, h):
@@ -25,9 +26,11 @@ def compare_tree_planes(cfg, tree, ot, s, h):
     integer decided by floating point: where two planes of a child are within PLANE_GAP at a
     node's reference query, fp32 and fp64 may pick differently and the pooled key moves, so such
     node planes (and their ancestors) compare only bhat, a continuous function of the estimates.
-    Returns the number of node planes excused."""
-    excused = 0
+    Returns (node planes excused, upper-level node planes, per level the [n] mask of excused
+    nodes, level 1 first)."""
+    excused, upper = 0, 0
     amb_prev = np.zeros((ot.n[0], ot.R), dtype=bool)
+    masks = []
     for l in range(1, ot.L + 1):
         kh, bh = zha.tree_level_view(cfg, tree, l)
         n = ot.n[l - 1]
@@ -37,8 +40,9 @@ def compare_tree_planes(cfg, tree, ot, s, h):
         assert np.max(np.abs(g_b - o_b)) <= SUMMARY_ATOL, f"level {l}: bhat"
         amb = np.zeros((n, ot.R), dtype=bool)
         if l >= 2:
+            upper += n * ot.R
             ck, cb = ot.level(l - 1)
-            q = np.asarray(ot_qref(ot, l))               # [R][d]
+            q = np.asarray(ot.qref[l - 1])               # [R][d]
             for i in range(n):
                 c0, c1 = i * cfg.b, min(i * cfg.b + cfg.b, ot.n[l - 2])
                 est = ot.scale * np.einsum("rd,cpd->rcp", q, ck[c0:c1]) + cb[c0:c1][None]   # [r][child][plane]
@@ -51,13 +55,52 @@ def compare_tree_planes(cfg, tree, ot, s, h):
             dk = np.max(np.abs(g_k - o_k)[ok])
             assert dk <= SUMMARY_ATOL, f"level {l}: khat err {dk:.3g} outside near-tied planes"
         amb_prev = amb
-    return excused
+        masks.append(amb.any(axis=1))
+    return excused, upper, masks
 
 
-def ot_qref(ot, l):
-    return ot.qref[l - 1]
+def node_scores(tree, q):
+    """Every node's score max_r(scale q.khat_r + bhat_r) on a tree, fp64, level 1 first."""
+    qd = np.asarray(q, dtype=np.float64).reshape(-1)
+    return np.max(tree.scale * np.einsum("nrd,d->nr", tree.khat, qd) + tree.bhat, axis=1)
+
+
+def walk_excuser(ot, gt, b):
+    """excuse(route) for check_queries, against the oracle's own tree ot: the GPU's tree gt
+    differs from ot where a child's plane choice was a near-tie, so every node score moves by
+    some delta = |s_gt - s_ot|.  If no node the oracle's walk scored moves by more than delta,
+    every normalised cumulative mass of the walk moves by at most 2 delta (and the score gap at
+    a cut by at most 2 delta), so the index set must still be exact when the cut margin exceeds
+    1e-4 + 2 delta; a query is excused only when it does not.  The scored nodes are rebuilt
+    bottom-up from the route: the kept blocks and the dropped nodes of each level, whose
+    parents (the kept nodes one level up) were scored in turn."""
+    off = np.cumsum([0] + list(ot.n))
+
+    def excuse(rt, q):
+        so, sg = node_scores(ot, q), node_scores(gt, q)
+        pr = np.asarray(rt.pr_node, dtype=np.int64)
+        scored = np.asarray(rt.sel, dtype=np.int64)
+        delta = 0.0
+        for l in range(1, ot.L + 1):
+            lo, hi = off[l - 1], off[l]
+            here = np.concatenate([scored, pr[(pr >= lo) & (pr < hi)] - lo])
+            if len(here):
+                delta = max(delta, float(np.max(np.abs(sg[lo + here] - so[lo + here]))))
+            scored = np.unique(here // b)
+        return rt.min_margin <= MARGIN + 2.0 * delta
+    return excuse
+
 
 pytestmark = pytest.mark.gpu
+
+
+# Reference queries of QREF_GAIN times the generator's N(0, 1/d) per coordinate.  With the
+# generator's own scale every block's softmax pooling is nearly uniform, so all R planes of a
+# node pool nearly the same key and their estimates nearly tie: the plane choice (an integer
+# decided by floating point) then differs between fp32 and fp64 for a large share of nodes and
+# tests little.  Larger reference queries make the planes distinct; the arithmetic tested is the
+# same.  The pages' reference queries are trained, so no scale is the pages'.
+QREF_GAIN = 4.0
 
 
 def planted(batch, Hkv, G, d, N, N_cap, M, n_q, R, run):
@@ -68,50 +111,61 @@ def planted(batch, Hkv, G, d, N, N_cap, M, n_q, R, run):
         for h in range(Hkv):
             cl = W.fill_planted_slice("test", s, h, N, d, M, K[s, h], V[s, h], run=run)
             Q[:, s, h * G:(h + 1) * G] = W.cluster_queries("test", s, h, G, n_q, cl).to(torch.bfloat16)
-    return K, V, Q, W.reference_queries("test", Hkv, R, d)
+    return K, V, Q, W.reference_queries("test", Hkv, R, d) * QREF_GAIN
 
 
 @pytest.mark.parametrize("R", [2, 4, 16])
 def test_planes_route_attend(R):
+    """Routing and attention with R planes, against the oracle's own fp64 tree: index sets
+    bit-exact wherever the cut margin exceeds 1e-4 and the oracle's walk scored no node whose
+    pooled key sits on a near-tied plane choice; then, as a second line, against the oracle run
+    on the GPU's own summaries, where every query beyond the margin must be exact."""
     batch, Hkv, G, d, N = 1, 2, 4, 128, 60013
     K, V, Q, qref = planted(batch, Hkv, G, d, N, N + 64, 24, 2, R, run=4096)
     cfg = zha.Config(d=d, Hq=Hkv * G, Hkv=Hkv, B=64, b=16, batch=batch, N_cap=N + 64, p=0.95, R=R)
     dec = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), [N])
     dec.build()
-    trees = {}
+    trees, gpu_trees, excusers = {}, {}, {}
+    torch.cuda.synchronize()
+    excused, upper = 0, 0
     for h in range(Hkv):
         ot = oracle_tree(K[0, h], N, cfg, qref[h])
         ot.qref = qref[h].double().numpy()
-        trees[h] = ot
-    torch.cuda.synchronize()
-    excused = 0
-    for h, ot in trees.items():
         assert ot.R == R
-        excused += compare_tree_planes(cfg, dec.tree, ot, 0, h)
-    # routing and attention against the oracle run on the GPU's own summaries (the route is a
-    # function of the tree; the tree's own parity is the check above)
-    gpu_trees = {}
-    for h, ot in trees.items():
+        e, u, _ = compare_tree_planes(cfg, dec.tree, ot, 0, h)
+        excused += e
+        upper += u
+        trees[h] = ot
         kk, bb = [], []
         for l in range(1, ot.L + 1):
             kh, bh = zha.tree_level_view(cfg, dec.tree, l)
             kk.append(kh[0, h, :ot.n[l - 1]].double().cpu().numpy())
             bb.append(bh[0, h, :ot.n[l - 1]].double().cpu().numpy())
         gpu_trees[h] = O.Tree(ot.N, ot.B, ot.b, ot.R, ot.d, ot.n, np.concatenate(kk), np.concatenate(bb), ot.scale)
-    trees = gpu_trees
-    rep = Report()
+        excusers[h] = walk_excuser(ot, gpu_trees[h], cfg.b)
+    print(f"R={R}: {excused} of {upper} upper-level node planes compared on bhat only (near-tied child planes)")
+    assert excused <= EXCUSED_MAX * upper, (excused, upper)
+    rep, rep_g = Report(), Report()
     for step in range(Q.shape[0]):
         Qs = Q[step].reshape(batch, 1, Hkv * G, d).contiguous()
         dec.route_attend(Qs.cuda())
         sel, cnt, o = dec.results()
         for hq in range(Hkv * G):
             h = hq // G
-            check_queries(cfg, trees[h], K[0, h], V[0, h], N - 1, Qs[0, 0, hq:hq + 1], [sel[0, 0, hq].numpy()],
-                          [int(cnt[0, 0, hq])], [o[0, 0, hq].numpy()], 0.95, rep)
+            args = (K[0, h], V[0, h], N - 1, Qs[0, 0, hq:hq + 1], [sel[0, 0, hq].numpy()], [int(cnt[0, 0, hq])],
+                    [o[0, 0, hq].numpy()], 0.95)
+            q = Qs[0, 0, hq].float()
+            check_queries(cfg, trees[h], *args, rep, excuse=lambda rt, h=h, q=q: excusers[h](rt, q))
+            # second line: the oracle's routing on the GPU's own summaries (the route is a function
+            # of the tree, so here every query beyond the margin is held to the bit)
+            check_queries(cfg, gpu_trees[h], *args, rep_g)
+    print(f"R={R} against the oracle's tree: {rep.summary()}")
+    print(f"R={R} against the oracle on the GPU's summaries: {rep_g.summary()}")
     rep.check()
+    rep_g.check()
     assert rep.exact_required >= rep.queries // 2, rep
+    assert rep_g.exact_required >= rep_g.queries // 2, rep_g
     assert_status_clean()
-    print(f"R={R}: {excused} node planes compared on bhat only (near-tied child planes)")
 
 
 def test_planes_append_matches_rebuild():

@@ -33,12 +33,21 @@ class Report:
     mismatches_required: int = 0
     mismatches_low_margin: int = 0
     low_margin: int = 0
+    excused: int = 0                # margin > 1e-4, but the walk met a node the caller excused
     max_err_own: float = 0.0        # vs the oracle over the oracle's set (relative in bf16)
     max_err_gpu_set: float = 0.0    # vs the oracle over the GPU's set
     read_keys: list = field(default_factory=list)
 
     def check(self):
         assert self.mismatches_required == 0, f"{self.mismatches_required} index sets differ beyond the margin"
+
+    def summary(self) -> dict:
+        """The counts the parity bar is stated in: index sets required bit-exact (margin > 1e-4) and
+        how many of them differ, and the same for the queries below the margin (reported only)."""
+        return {"queries": self.queries, "exact_required": self.exact_required,
+                "mismatches_required": self.mismatches_required, "low_margin": self.low_margin,
+                "mismatches_low_margin": self.mismatches_low_margin, "excused": self.excused,
+                "max_err_gpu_set": self.max_err_gpu_set, "max_err_own": self.max_err_own}
 
 
 def oracle_tree(K_slice_cpu, N, cfg: zha.Config, qref_slice):
@@ -66,11 +75,13 @@ def out_err(o_gpu: np.ndarray, o_ref: np.ndarray, dtype: str) -> float:
 
 
 def check_queries(cfg: zha.Config, ot: O.Tree, K_slice, V_slice, t, queries, sel_rows, counts, outs,
-                  p, rep: Report, tight_of_v: float | None = None):
+                  p, rep: Report, tight_of_v: float | None = None, excuse=None):
     """queries: [nq][d] (CPU tensors, the exact values the GPU read); sel_rows/counts/outs: GPU results.
     t: the queries' position, or one position per query.  tight_of_v: when given, the tight check
     against the oracle over the GPU's set is |d|_inf <= tight_of_v * max |v| over that set (the
-    tensor-core path rounds the softmax weights to bf16 before P V) instead of 1e-3 of |o|_inf."""
+    tensor-core path rounds the softmax weights to bf16 before P V) instead of 1e-3 of |o|_inf.
+    excuse: when given, excuse(route) -> True lifts the exactness requirement of a query whose
+    oracle walk scored a node the caller cannot compare (counted in rep.excused)."""
     bar = TOL_F32 if cfg.dtype == "f32" else TOL_BF16_REL
     for i in range(len(queries)):
         q = queries[i]
@@ -79,7 +90,9 @@ def check_queries(cfg: zha.Config, ot: O.Tree, K_slice, V_slice, t, queries, sel
         g_sel = np.asarray(sel_rows[i][:counts[i]], dtype=np.int64)
         rep.queries += 1
         same = len(g_sel) == len(rt.sel) and np.array_equal(g_sel, rt.sel)
-        if rt.min_margin > MARGIN:
+        if rt.min_margin > MARGIN and excuse is not None and excuse(rt):
+            rep.excused += 1
+        elif rt.min_margin > MARGIN:
             rep.exact_required += 1
             rep.mismatches_required += 0 if same else 1
         else:
