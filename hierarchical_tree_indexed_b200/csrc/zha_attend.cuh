@@ -109,11 +109,13 @@ __device__ __forceinline__ void consumer_sync() {   // named barrier of the 8 co
 // chunk j belongs to CTA j mod C.  A CTA's chunks inside one group are
 // consecutive in its own order, so it gives at most one partial per group,
 // stored at slot = its index; a group has min(C, chunks it spans) partials.
+// (Item counts stay below 2^31: 32-bit divisions.)
 __device__ __forceinline__ int64_t chunk_items(int64_t I, int C) {
-    return kAttChunk > 0 ? kAttChunk : (I + C - 1) / C;
+    return kAttChunk > 0 ? kAttChunk : (static_cast<uint32_t>(I) + C - 1) / static_cast<uint32_t>(C);
 }
 __device__ __forceinline__ int partials_of(int64_t g0, int64_t g1, int64_t ch, int C) {
-    const int64_t j0 = g0 / ch, j1 = (g1 - 1) / ch;
+    const uint32_t uch = static_cast<uint32_t>(ch);
+    const int64_t j0 = static_cast<uint32_t>(g0) / uch, j1 = static_cast<uint32_t>(g1 - 1) / uch;
     return static_cast<int>(min(static_cast<int64_t>(C), j1 - j0 + 1));
 }
 
@@ -537,7 +539,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attend_kernel(AttendArgs a) {
                 const int s = g / a.Hkv, kv = g % a.Hkv;
                 const int ct = tid;   // 0 .. 255
                 const int64_t pb = static_cast<int64_t>(g) * kSplitMax * G;
-                const int slot0 = static_cast<int>((sm.prefix[g] / ch) % C);   // partial k sits at slot (slot0+k) % C
+                const int slot0 = static_cast<int>((static_cast<uint32_t>(sm.prefix[g]) / static_cast<uint32_t>(ch)) % C);   // partial k sits at slot (slot0+k) % C
                 float* fw = sm.red;                      // [kSplitMax][G] weights (red is free here)
                 float* fl = fw + kSplitMax * G;          // [kSplitMax][G] partial sums
                 for (int x = ct; x < sp * G; x += kAttConsumers * 32) {

@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         if (lane == 0) ctl->prefix[a.groups] = static_cast<int>(I);
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->pre_ready);
-        const int64_t ch = I > 0 ? (I + C - 1) / C : 1;   // items per CTA: one contiguous piece each
+        const int64_t ch = I > 0 ? (static_cast<uint32_t>(I) + C - 1) / static_cast<uint32_t>(C) : 1;   // items per CTA: one contiguous piece each
         int fills = 0;     // pairs posted (lane 0's count is the one used)
         bool ok = true;
         auto acquire = [&](int f) -> bool {
@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         }
         twait(&ctl->pre_ready, 0, ctl);   // the group prefix (first read by an epilogue)
         const int64_t I = ctl->prefix[a.groups];
-        const int64_t ch = I > 0 ? (I + C - 1) / C : 1;
+        const int64_t ch = I > 0 ? (static_cast<uint32_t>(I) + C - 1) / static_cast<uint32_t>(C) : 1;
         uint32_t e = 0, nm = 0;   // epilogues and merges so far
         float2* mbuf = reinterpret_cast<float2*>(reinterpret_cast<unsigned char*>(ctl) + tc_merge_offset(a.groups));
         for (uint32_t g = 0;; ++g) {
@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                     const int sp = ctl->sp;
                     const int s = grp / a.Hkv, kv = grp % a.Hkv;
                     const int64_t pb0 = static_cast<int64_t>(grp) * kSplitMax * G;
-                    const int slot0 = static_cast<int>((ctl->prefix[grp] / ch) % C);   // partial k at slot (slot0+k) % C
+                    const int slot0 = static_cast<int>((static_cast<uint32_t>(ctl->prefix[grp]) / static_cast<uint32_t>(ch)) % C);   // partial k at slot (slot0+k) % C
                     float xr[kTCRegPartials][G];
                     auto load_round = [&](int k0) {
 #pragma unroll

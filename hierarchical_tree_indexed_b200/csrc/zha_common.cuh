@@ -24,13 +24,16 @@ __device__ __forceinline__ void raise_status(int code) { atomicOr(&g_status, 1 <
 // ("Subquadratic Attention with a Hierarchical Tree-Structured Indexer",
 // Tree Construction: a level-l node spans C^l keys, here B*b^(l-1)).
 // Returns L, or -1 when more than kMaxLevels levels would be needed.
+// N < 2^31 (zha_config's N_cap is bounded so), so the arithmetic is 32-bit: a 64-bit
+// division is a long emulated sequence on the GPU, on every router's critical path.
 __host__ __device__ inline int tree_levels(int64_t N, int B, int b, int L_fixed, int64_t* n) {
-    int64_t cur = N / B;
+    uint32_t cur = static_cast<uint32_t>(N > 0 ? N : 0) / static_cast<uint32_t>(B);
+    const uint32_t ub = static_cast<uint32_t>(b);
     int L = 1;
     n[0] = cur;
-    while (L_fixed > 0 ? L < L_fixed : cur > b) {
+    while (L_fixed > 0 ? L < L_fixed : cur > ub) {
         if (L >= kMaxLevels) return -1;
-        cur = (cur + b - 1) / b;
+        cur = (cur + ub - 1) / ub;
         n[L++] = cur;
     }
     return L;

@@ -40,14 +40,22 @@ struct PlanArgs {
 // (bits at and beyond n_1 clear); the current chunk's block is added here.  scan:
 // kPlanThreads/32+1 ints.  N, Ntree: the sequence's key count and tree count, valid
 // (1 <= N <= N_cap, Ntree <= N).
-__device__ void plan_emit(const PlanArgs& a, int g, uint32_t* bits, int* scan, int64_t N, int64_t Ntree) {
+struct NoTail {
+    __device__ void operator()() const {}
+};
+// tail(): run by warp 1 while thread 0 writes the plan's last items (used for bookkeeping
+// that does not touch the plan).
+template <typename Tail = NoTail>
+__device__ void plan_emit(const PlanArgs& a, int g, uint32_t* bits, int* scan, int64_t N, int64_t Ntree,
+                          Tail tail = Tail()) {
     const int tid = threadIdx.x;
     const int G = a.G;
     const uint32_t all = (1u << G) - 1u;
     const int64_t t = N - 1;
-    const int64_t n1 = Ntree / a.B;
+    const uint32_t uB = static_cast<uint32_t>(a.B);   // keys < 2^31: 32-bit divisions
+    const int64_t n1 = static_cast<uint32_t>(Ntree) / uB;
     const int64_t words = (n1 + 31) / 32;
-    const int64_t cb = min(t / a.B, n1);   // C_cur = [cb*B, t]
+    const int64_t cb = min(static_cast<int64_t>(static_cast<uint32_t>(t) / uB), n1);   // C_cur = [cb*B, t]
     if (tid < G && cb < n1) atomicOr(&bits[tid * a.words + (cb >> 5)], 1u << (cb & 31));
     __syncthreads();
     // compaction of the union, ascending.  Warp w takes the words [w*per, (w+1)*per), per a
@@ -120,6 +128,8 @@ __device__ void plan_emit(const PlanArgs& a, int g, uint32_t* bits, int* scan, i
             }
         a.n_items[g] = n;
         a.rows[g] = static_cast<int32_t>(rows);
+    } else if (tid >= 32 && tid < 64) {
+        tail();
     }
     __syncthreads();
 }
@@ -137,7 +147,7 @@ __device__ void plan_group(const PlanArgs& a, int g, uint32_t* bits, int* scan) 
         __syncthreads();
         return;
     }
-    const int64_t n1 = Ntree / a.B;
+    const int64_t n1 = static_cast<uint32_t>(Ntree) / static_cast<uint32_t>(a.B);
     const int64_t words = (n1 + 31) / 32;
     // every head's selected blocks into its bitmap: kPlanThreads / G threads per head load
     // the head's count and their first kPlanSpec entries together (one round trip; entries

@@ -71,6 +71,7 @@ struct CutSmem {
     unsigned long long mmass[kCutMembers];
     unsigned long long above, target;      // mass ordered before the crossing (sub-)bin; the target
     int nm, cbin, sbin;                    // members; crossing bin; crossing sub-bin (-1: not split)
+    int cnt;                               // the kept count (small cuts)
 };
 
 struct RouteSmem {
@@ -259,6 +260,14 @@ __device__ int block_cut(const float* sc, int nc, float p, float mx, int32_t* ou
     constexpr int NT = kRouteThreads;
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     if (mx == -INFINITY || nc <= 0) return 0;   // uniform
+    if (nc <= 64) {   // one warp sorts them (top_p_small)
+        if (w == 0) {
+            const int c = top_p_small(sc, nc, p, out, node_of);
+            if (lane == 0) cs.cnt = c;
+        }
+        __syncthreads();
+        return cs.cnt;
+    }
     const bool keep_all = p >= 1.0f;
     const int ngrp = (nc + 31) / 32;
     int cbin = kCutBins, sbin = -1;
@@ -633,7 +642,7 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
     int cur = 0;   // index into bufs
 
     // virtual parents of the top level: parent i has children [i*b, i*b+b) of level L
-    int np = static_cast<int>((n[L - 1] + b - 1) / b);
+    int np = static_cast<int>((static_cast<uint32_t>(n[L - 1]) + b - 1) / static_cast<uint32_t>(b));
     if (np > kParentsSmem) cur = 2;
     for (int i = tid; i < np; i += kRouteThreads) bufs[cur][i] = i;
     // the level below the top, when small, is scored in the same pass as the top level (its
@@ -648,7 +657,7 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
         const int64_t nl = n[l - 1];
         const int nc = np * b;
         if (np > 0) {   // only the last possible parent can have fewer than b children
-            const int64_t last_parent = (nl - 1) / b;
+            const int64_t last_parent = static_cast<uint32_t>(nl - 1) / static_cast<uint32_t>(b);
             scored += nc - (bufs[cur][np - 1] == last_parent ? b - (nl - last_parent * b) : 0);
         }
         float* sc = nc <= kScoresSmem ? sm.scores : ws_sc;
@@ -724,23 +733,65 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
         const int np_par = np;
         const int nxt = nc <= kParentsSmem ? (cur == 0 ? 1 : 0) : (cur == 2 ? 3 : 2);
         auto node_of = [par, b](int i) { return static_cast<int32_t>(par[i / b] * b + i % b); };
+        // the kept nodes into CTA 0's bitmaps: the level's kept set (for the count of distinct
+        // nodes read), or at level 1 this head's selected blocks (the gather plan)
+        auto publish = [&](int lv, const int32_t* kept, int cnt) {
+            if (!region) return;
+            const uint32_t bm = region + 4u * static_cast<uint32_t>(lv == 1 ? head * a.plan.words : a.lvl_off[lv - 1]);
+            for (int i = tid; i < cnt; i += kRouteThreads) {
+                const int32_t x = kept[i];
+                dsmem_or(bm + 4u * static_cast<uint32_t>(x >> 5), 1u << (x & 31));
+            }
+        };
+        if (!vsum && spec && l == L && nc <= 64 && cur < 2 && nxt < 2) {
+            // ---- the top level and the level below it in one step of warp 0 (both small; the
+            // level below was scored with the top): a block cut and the scores' copy less
+            if (w == 0) {
+                const int k = top_p_small(sc, nc, a.p[L - 1], bufs[nxt], node_of);
+                __syncwarp();
+                const int nc2 = k * b;
+                int k2 = -1;
+                if (nc2 <= 64) {
+                    float* sc2 = sm.scores + 64;
+                    const int32_t* kt = bufs[nxt];
+                    for (int i = lane; i < nc2; i += 32) {
+                        const int64_t c = static_cast<int64_t>(kt[i / b]) * b + i % b;
+                        sc2[i] = c < n[L - 2] ? sm.spec[c] : -INFINITY;
+                    }
+                    __syncwarp();
+                    auto node2 = [kt, b](int i) { return static_cast<int32_t>(kt[i / b] * b + i % b); };
+                    k2 = top_p_small(sc2, nc2, a.p[L - 2], bufs[cur], node2);   // the top's parents are done
+                }
+                if (lane == 0) { sm.redi[0] = k; sm.redi[1] = k2; }
+            }
+            // the top level's max slot is the level two below's: clear it (its scan starts after
+            // the barrier; nothing reads the top's max on this path)
+            if (tid == 32) sm.mxkey[L & 1] = ord_key(-INFINITY);
+            __syncthreads();
+            const int k = sm.redi[0], k2 = sm.redi[1];
+            if (region) cluster_wait();   // CTA 0 has cleared the region
+            publish(L, bufs[nxt], k);
+            if (k2 >= 0) {   // uniform
+                publish(L - 1, bufs[cur], k2);
+                const int64_t n2 = n[L - 2];
+                const int64_t last2 = static_cast<uint32_t>(n2 - 1) / static_cast<uint32_t>(b);
+                if (k > 0) scored += static_cast<int64_t>(k) * b - (bufs[nxt][k - 1] == last2 ? b - (n2 - last2 * b) : 0);
+                np = k2;
+                --l;   // the level below the top is done; bufs[cur] holds its kept nodes
+                continue;
+            }
+            np = k;
+            cur = nxt;
+            continue;
+        }
         {
             const bool big = (nc + 31) / 32 > kScoresSmem / 32;   // ballot words in the workspace
             np = block_cut(sc, nc, a.p[l - 1], key_ord(*mxk), bufs[nxt], sm.cut, big ? ws_kb : sm.keep_ballot,
                            big ? reinterpret_cast<int32_t*>(ws_kb) + a.kb_cap : sm.keep_prefix, sm.scan, node_of);
         }
         __syncthreads();
-        if (region) {
-            // the kept nodes into CTA 0's bitmaps: the level's kept set (for the count of distinct
-            // nodes read), or at level 1 this head's selected blocks (the gather plan)
-            if (l == L) cluster_wait();   // CTA 0 has cleared the region
-            const uint32_t bm = region + 4u * static_cast<uint32_t>(l == 1 ? head * a.plan.words : a.lvl_off[l - 1]);
-            const int32_t* kept = bufs[nxt];
-            for (int i = tid; i < np; i += kRouteThreads) {
-                const int32_t x = kept[i];
-                dsmem_or(bm + 4u * static_cast<uint32_t>(x >> 5), 1u << (x & 31));
-            }
-        }
+        if (region && l == L) cluster_wait();   // CTA 0 has cleared the region
+        publish(l, bufs[nxt], np);
         if constexpr (vsum)
             add_dropped<D, NVR>(sc, par, np_par, b, nl, bufs[nxt], np, a.tree.vhat[l - 1] + slice * ncap * D, sm);
         cur = nxt;
@@ -763,7 +814,7 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
 
 // Distinct tree nodes the group's route read: every top node, the level below the top
 // whole when it was read with the top (kSpecMax), and below that the children of the
-// nodes any head kept one level up (the level bitmaps in the plan region).  Warp 0 of CTA 0.
+// nodes any head kept one level up (the level bitmaps in the plan region).  One warp.
 __device__ int64_t route_scanned(const RouteArgs& a, const uint32_t* region, int64_t Ntree) {
     const int lane = threadIdx.x & 31;
     int64_t n[kMaxLevels];
@@ -773,14 +824,25 @@ __device__ int64_t route_scanned(const RouteArgs& a, const uint32_t* region, int
     for (int l = spec ? L - 1 : L; l >= 2; --l) {
         const uint32_t* bm = region + a.lvl_off[l - 1];
         const int64_t words = (n[l - 1] + 31) / 32, last = n[l - 1] - 1;
-        int64_t c = 0;
+        int c = 0;
         for (int64_t i = lane; i < words; i += 32) c += __popc(bm[i]);
-        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-        tot += c * a.b;
+        c = __reduce_add_sync(0xffffffffu, static_cast<unsigned>(c));
+        tot += static_cast<int64_t>(c) * a.b;
         if ((bm[last >> 5] >> (last & 31)) & 1u) tot -= a.b - (n[l - 2] - last * a.b);   // partial last parent
     }
     return tot;
 }
+
+// Writes the group's count of distinct nodes read (warp 1 of CTA 0, beside the plan's tail).
+struct ScannedTail {
+    const RouteArgs* a;
+    const uint32_t* region;
+    int64_t Ntree, slice;
+    __device__ void operator()() const {
+        const int64_t c = route_scanned(*a, region, Ntree);
+        if ((threadIdx.x & 31) == 0) a->scanned[slice] = static_cast<int32_t>(c);
+    }
+};
 
 // One CTA per (sequence, query head): the whole top-down walk of one decode query.
 // NVR = b rounded up to a power of two (4, 8, 16 or 32).
@@ -828,11 +890,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
         cluster_wait();
         if (rank == 0) {
             if (valid) {
-                plan_emit(a.plan, static_cast<int>(slice), region, sm.scan, N, Ntree);
-                if (tid < 32) {
-                    const int64_t c = route_scanned(a, region, Ntree);
-                    if (tid == 0) a.scanned[slice] = static_cast<int32_t>(c);
-                }
+                plan_emit(a.plan, static_cast<int>(slice), region, sm.scan, N, Ntree,
+                          ScannedTail{&a, region, Ntree, slice});
             } else if (tid == 0) {
                 a.plan.n_items[slice] = 0;
                 a.plan.rows[slice] = 0;
