@@ -68,6 +68,9 @@ def parse():
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling cases)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's N (profiling cases)")
     ap.add_argument("--sweep", default="", help="comma-separated context lengths: tree path vs dense baseline")
+    ap.add_argument("--run", type=int, default=0,
+                    help="keys per planted cluster (0: the calibrated default); with --beta, another in-band calibration")
+    ap.add_argument("--beta", type=float, default=0.0, help="query aim strength (0: the calibrated default)")
     ap.add_argument("--vsum", action="store_true",
                     help="decode with value summaries of the dropped subtrees, and report their error against dense")
     return ap.parse_args()
@@ -86,8 +89,12 @@ def workload(args):
 
 
 def config_dict(w, world: int) -> dict:
+    gen = ""
+    if getattr(args_global, "run", 0) or getattr(args_global, "beta", 0.0):
+        from hierarchical_tree_indexed_b200 import workloads as W
+        gen = f", planted clusters of {args_global.run or W.RUN} keys aimed at with beta {args_global.beta or W.BETA}"
     return {"workload": f"{w.name}: batch {w.batch} per GPU, {w.Hq} query / {w.Hkv} KV heads, d {w.d}, "
-                        f"bf16 K/V, N={w.N}, leaf block {w.B}, branching {w.b}, p={w.p}",
+                        f"bf16 K/V, N={w.N}, leaf block {w.B}, branching {w.b}, p={w.p}{gen}",
             "global_batch": w.batch * world, "seq_len": w.N, "parallelism": f"dp{world}",
             "kv_dtype": w.dtype,
             "l2": L2Flush.NOTE + f"; KV {w.batch * w.Hkv * w.N * w.d * 2 * (2 if w.dtype == 'bf16' else 4) / 2**30:.1f} GiB > L2",
@@ -354,7 +361,12 @@ class DecodeRun:
         from hierarchical_tree_indexed_b200 import zha
         self.w, self.dev, self.zha = w, dev, zha
         # weak scaling: every rank owns a batch of w.batch sequences of its own
-        data = W.planted(w, device=dev, N_cap=N_cap, n_queries=POOL, seq_base=rank.rank * w.batch)
+        gen = {}
+        if getattr(args_global, "run", 0):
+            gen["run"] = args_global.run
+        if getattr(args_global, "beta", 0.0):
+            gen["beta"] = args_global.beta
+        data = W.planted(w, device=dev, N_cap=N_cap, n_queries=POOL, seq_base=rank.rank * w.batch, **gen)
         self.K, self.V, self.Qp, self.knp, self.vnp = data["K"], data["V"], data["Q"], data["k_new"], data["v_new"]
         self.cfg = zha.Config(d=w.d, Hq=w.Hq, Hkv=w.Hkv, B=w.B, b=w.b, batch=w.batch, N_cap=N_cap,
                               dtype=w.dtype, p=w.p, vsum=1 if vsum else 0)
@@ -805,8 +817,13 @@ def value_summary_report(run, args, queries=8, ps=(None, 0.8, 0.5)):
             "note": "mean over (query, head) of |o - o_dense| / |o_dense|, decode queries of the workload"}
 
 
+args_global = None   # the parsed command line (generator overrides read by the workload helpers)
+
+
 def main():
+    global args_global
     args = parse()
+    args_global = args
     from hierarchical_tree_indexed_b200 import dist as D
     rank = D.from_env()
     if args.impl == "reference":

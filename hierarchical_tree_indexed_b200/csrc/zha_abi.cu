@@ -25,6 +25,7 @@
 #include "zha_attend.cuh"
 #include "zha_attend_tc.cuh"
 #include "zha_prefill.cuh"
+#include "zha_score_tc.cuh"
 
 using namespace zha;
 
@@ -526,6 +527,10 @@ int run_plan(const zha_config* c, const WsLayout& wl, const TreeLayout& lay, con
 // partials of every row and the accounting counters.
 struct PfLayout {
     int64_t slices, R, rows, cand_cap, par_cap, nJ_cap, item_cap, n1_cap, pair_cap;
+    int64_t ucap;              // upper nodes scored on the tensor cores per row (0: that path is off)
+    int up_off[kMaxLevels];
+    int chunk_cap;             // 64-node chunks of the upper levels, at most
+    size_t off_up, off_split, off_sbias;
     size_t off_spill_sc, off_spill_par, off_cand, off_totals, off_hdr, off_ctr, off_row_cnt, off_row_pairs, off_row_off;
     size_t off_jcount, off_jcur, off_pairs, off_items, off_tail_ml, off_tail_o, off_sel_ml, off_sel_o, off_steps;
     size_t total;
@@ -571,6 +576,28 @@ int pf_layout(const zha_config* c, int n_q, const TreeLayout& t, PfLayout* p) {
     p->off_tail_o = off;    off = align256(off + sizeof(float) * p->rows * D);
     p->off_sel_ml = off;    off = align256(off + sizeof(float2) * p->pair_cap);
     p->off_sel_o = off;     off = align256(off + sizeof(float) * p->pair_cap * D);
+    // the upper levels' scores of every row, computed on the tensor cores (R = 1, at least two
+    // levels, at most kSUMaxCols upper nodes): column up_off[l-1] + node for level l >= 2
+    p->ucap = 0;
+    p->chunk_cap = 0;
+    for (int l = 0; l < kMaxLevels; ++l) p->up_off[l] = 0;
+    if (t.R == 1 && t.Lcap >= 2) {
+        int64_t u = 0;
+        int ch = 0;
+        for (int l = 2; l <= t.Lcap; ++l) {
+            p->up_off[l - 1] = static_cast<int>(u);
+            u += t.ncap[l - 1];
+            ch += static_cast<int>((t.ncap[l - 1] + kSUNodes - 1) / kSUNodes);
+        }
+        if (u <= kSUMaxCols) {
+            p->ucap = u;
+            p->chunk_cap = ch;
+        }
+    }
+    const size_t tile_bytes = (c->d == 128 ? SULayout<128>::kBBytes : SULayout<64>::kBBytes);
+    p->off_up = off;        off = align256(off + sizeof(float) * p->rows * p->ucap);
+    p->off_split = off;     off = align256(off + tile_bytes * p->slices * p->chunk_cap);
+    p->off_sbias = off;     off = align256(off + sizeof(float) * kSUNodes * p->slices * p->chunk_cap);
     p->total = off;
     return ZHA_OK;
 }
@@ -625,6 +652,34 @@ int make_q_map(const zha_config* c, const void* base, int64_t rows, CUtensorMap*
     return ZHA_OK;
 }
 
+// The upper levels' scores of every chunk row on the tensor cores (score_upper_kernel).
+template <int D>
+int run_score_upper(const zha_config* c, const TreeLayout& lay, const PfLayout& pl, const void* tree, const void* Q,
+                    int n_q, const int32_t* N, void* ws, cudaStream_t st) {
+    SUArgs s{};
+    s.Q = static_cast<const uint16_t*>(Q);
+    s.tree = tree_view(lay, const_cast<void*>(tree));
+    s.N = N;
+    s.up = at<float>(ws, pl.off_up);
+    s.split = at<unsigned char>(ws, pl.off_split);
+    s.bias = at<float>(ws, pl.off_sbias);
+    s.chunk_cap = pl.chunk_cap;
+    s.ucap = pl.ucap;
+    s.N_cap = c->N_cap;
+    for (int l = 0; l < kMaxLevels; ++l) s.up_off[l] = pl.up_off[l];
+    s.n_q = n_q; s.Hq = c->Hq; s.Hkv = c->Hkv; s.G = c->Hq / c->Hkv; s.B = c->B; s.b = c->b; s.L_fixed = c->L_fixed;
+    s.R = static_cast<int>(pl.R);
+    s.slices = static_cast<int>(pl.slices);
+    s.tiles = static_cast<int>((pl.R + kSUTileRows - 1) / kSUTileRows);
+    s.scale = scale_of(c);
+    split_upper_kernel<D><<<static_cast<unsigned>(s.slices * s.chunk_cap), 256, 0, st>>>(s);
+    ZHA_TRY(check_launch("split_upper"));
+    auto kern = score_upper_kernel<D>;
+    ZHA_TRY(allow_smem(kern, SULayout<D>::kSmem));
+    kern<<<static_cast<unsigned>(s.slices * s.tiles), kSUThreads, SULayout<D>::kSmem, st>>>(s);
+    return check_launch("score_upper");
+}
+
 template <int D, int NVR>
 int run_proute_t(const PRouteArgs& a, int64_t rows, cudaStream_t st) {
     auto kern = a.tree.R > 1 ? route_prefill_kernel<uint16_t, D, NVR, true> : route_prefill_kernel<uint16_t, D, NVR, false>;
@@ -651,6 +706,12 @@ int run_proute(const zha_config* c, const TreeLayout& lay, const PfLayout& pl, c
     a.L_fixed = c->L_fixed; a.n_q = n_q;
     a.scale = scale_of(c);
     for (int l = 0; l < kMaxLevels; ++l) a.p[l] = c->p[l];
+    if (pl.ucap > 0) {   // the upper levels on the tensor cores first
+        ZHA_TRY(run_score_upper<D>(c, lay, pl, tree, Q, n_q, N, ws, st));
+        a.up = at<float>(ws, pl.off_up);
+        a.ucap = pl.ucap;
+        for (int l = 0; l < kMaxLevels; ++l) a.up_off[l] = pl.up_off[l];
+    }
     const int64_t rows = static_cast<int64_t>(c->batch) * n_q * c->Hq;
     if (c->b <= 4) return run_proute_t<D, 4>(a, rows, st);
     if (c->b <= 8) return run_proute_t<D, 8>(a, rows, st);

@@ -55,6 +55,9 @@ struct PRouteArgs {
     int32_t* cand;          // [batch][n_q][Hq] nodes scored (accounting)
     float* spill_sc;        // [kPRSpillWarps][cand_cap]
     int32_t* spill_par;     // [kPRSpillWarps][2][par_cap]
+    const float* up;        // the upper levels' scores from score_upper_kernel, [slices][R][ucap]; or null
+    int64_t ucap;
+    int up_off[kMaxLevels]; // column of level l's node 0 (index l - 1), l >= 2
     int64_t cand_cap, par_cap, N_cap;
     int sel_cap, batch, Hq, Hkv, B, b, L_fixed, n_q;
     float scale;
@@ -101,6 +104,12 @@ __global__ void __launch_bounds__(kPRThreads, 2) route_prefill_kernel(PRouteArgs
             }
             continue;
         }
+        // the row's scores at the upper levels, when the tensor cores computed them
+        const float* up_row = nullptr;
+        if (a.up) {
+            const int i = (x % per_seq) / a.Hq;
+            up_row = a.up + (slice * (static_cast<int64_t>(a.n_q) * G) + static_cast<int64_t>(i) * G + hq % G) * a.ucap;
+        }
         float qv[VF];
         load_n<T, VF>(static_cast<const T*>(a.Q) + static_cast<int64_t>(x) * D + lane * VF, qv);
 #pragma unroll
@@ -127,7 +136,15 @@ __global__ void __launch_bounds__(kPRThreads, 2) route_prefill_kernel(PRouteArgs
             const int R = MP ? a.tree.R : 1;
             const float* kh = a.tree.khat[l - 1] + slice * ncap * R * D;
             const float* bh = a.tree.bhat[l - 1] + slice * ncap * R;
-            for (int pi = 0; pi < np; pi += 2) {
+            const bool read_up = up_row && l >= 2;
+            if (read_up) {   // read, not scanned: the kept parents' children
+                const float* us = up_row + a.up_off[l - 1];
+                for (int i = lane; i < nc; i += 32) {
+                    const int64_t c = static_cast<int64_t>(par[i / b]) * b + i % b;
+                    sc[i] = c < nl ? __ldg(us + c) : -INFINITY;
+                }
+            }
+            for (int pi = 0; pi < (read_up ? 0 : np); pi += 2) {
                 const int64_t c0 = static_cast<int64_t>(par[pi]) * b;
                 const int cnt0 = static_cast<int>(min(static_cast<int64_t>(b), nl - c0));
                 if constexpr (!MP) {
