@@ -33,8 +33,10 @@ namespace zha {
 
 constexpr int kRouteThreads = 512;
 constexpr int kRouteWarps = kRouteThreads / 32;
-constexpr int kScoresSmem = 16384;   // candidate scores kept in shared memory up to this count
-constexpr int kParentsSmem = 4096;   // per buffer; larger lists live in the workspace
+// Shared memory is kept small on purpose: the scans' loads go through L1, which shares the SM's
+// memory with it, and a smaller L1 holds fewer loads in flight.
+constexpr int kScoresSmem = 8192;    // candidate scores kept in shared memory up to this count
+constexpr int kParentsSmem = 2048;   // per buffer; larger lists live in the workspace
 
 struct RouteArgs {
     TreeDev tree;
@@ -63,7 +65,8 @@ struct RouteArgs {
 constexpr int kSpecMax = 256;   // the level below the top is scored with the top level when it has at most this many nodes
 constexpr int kCutBins = 256;      // mass bins of 1/8 nat below the level's max score (a crossing bin
                                    // with too many members is split again into 256 sub-bins)
-constexpr int kCutMembers = 256;   // crossing-bin members ranked pairwise in shared memory
+constexpr int kCutMembers = 256;   // crossing-bin members listed in shared memory and ranked pairwise
+constexpr int kCutSplit = 64;      // a crossing bin with more members is split into sub-bins first
 
 struct CutSmem {
     unsigned long long bins[kCutBins];     // zero between cuts
@@ -249,8 +252,8 @@ __device__ __forceinline__ void cut_locate(unsigned long long* bins, unsigned lo
 //      max's are 0 and skipped);
 //   2. warp 0 finds the bin where the cumulative mass reaches the target;
 //   3. the candidates of earlier bins are kept (one ballot word per 32 slots) and the crossing
-//      bin's members listed; when they are too many, their masses are binned again into 256
-//      sub-bins, the crossing sub-bin found, and its members listed instead;
+//      bin's members listed; when they are more than kCutSplit, their masses are binned again
+//      into 256 sub-bins, the crossing sub-bin found, and its members listed instead;
 //   4. member k is kept iff the mass of the members ordered before it, plus the mass ordered
 //      before its (sub-)bin, is below the target (its bit joins the ballot words);
 //   5. a scan of the ballot words' counts places every word's kept ids, in slot order.
@@ -301,7 +304,7 @@ __device__ int block_cut(const float* sc, int nc, float p, float mx, int32_t* ou
     }
     if (!keep_all) {
         __syncthreads();
-        if (cs.nm > kCutMembers) {   // uniform: split the crossing bin
+        if (cs.nm > kCutSplit) {   // uniform: split the crossing bin (pairwise ranks grow as members^2)
             for (int i = t; i < nc; i += NT) {
                 const float s = sc[i];
                 if (s != -INFINITY && cut_bin(s, mx) == cbin) {
