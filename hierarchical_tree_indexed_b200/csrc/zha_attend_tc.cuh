@@ -24,6 +24,10 @@
 // warp 4: TMA producer; warp 5: TMEM owner and MMA issue (one lane).  The
 // online softmax runs in log2 units; O is rescaled lazily, only when a head's
 // running max outgrows its reference by 2^8.
+// Pieces are cut on a cost axis on which every group starts with kTCGroupCost
+// items of virtual cost: a CTA whose piece crosses into another group spends
+// that long in the extra epilogue (its softmax warps stall while the group's
+// partial is written), so it gets fewer keys and the CTAs end together.
 // Every wait is bounded: a timeout raises ZHA_ERR_TIMEOUT, marks the CTA
 // aborted, and all later waits return at once, so the kernel always ends.
 #pragma once
@@ -46,14 +50,15 @@ constexpr uint32_t kTCPBytes = 2 * 16 * 128;                   // P^T: 16 rows x
 constexpr uint32_t kTCOffP = kTCStages * kTCStageBytes;
 constexpr uint32_t kTCOffCtl = kTCOffP + 2 * kTCPBytes;
 constexpr uint32_t kTCTmemCols = 64;                           // S: 2 x 16 columns; O: 16 columns at 32
-constexpr int kTCRegPartials = 8;                              // a merge of at most this many partials runs from registers
+constexpr int kTCGroupCost = 7;                                // a group start on the piece cost axis, in items
 constexpr float kTCRescaleLog2 = 8.0f;                         // lazy rescale: P stays below 2^8 between rescales
 
 struct TcDesc {
     int n0, n1;                // keys of the pair's items (n1 = 0: one item); n0 < 0: no more work
     uint32_t heads0, heads1;   // head masks of the two items
     int group, split;
-    int flags;                 // bit 0: last pair of this CTA's piece of the group; bit 1: first pair
+    int flags;                 // bit 0: last pair of this CTA's piece of the group; bit 1: first pair;
+                               // bit 2: last pair of the CTA's whole piece
     int pad;
 };
 
@@ -66,17 +71,18 @@ struct TcCtl {
     uint64_t o_done[2];            // MMA -> softmax: P V of pair g (and every MMA before it) completed
     uint64_t mx[2];                // softmax warps: pair maxima exchanged
     uint64_t ep[3];                // softmax warps: partial sums exchanged / partial stored / merge decided
-    uint64_t mg[2];                // softmax warps: a merge's (max, sum) gathered / weights computed
+    uint64_t mg[2];                // softmax warps: a merge's (max, sum) gathered (merge in mid-piece) / weights formed
+    uint64_t mgb;                  // bulk copies: a merge's partials landed in the stage buffers
     uint64_t pre_ready;            // producer -> softmax: prefix[] written
     uint64_t fin;                  // MMA lane: every MMA it issued completed
     TcDesc desc[kTCStages];
     uint32_t tmem;
     int abort;
-    int last_flag, sp;
+    int last_flag, sp, sp0;
     uint64_t wait_ns;              // bound of a wait on another warp's progress
     int red[2][4][4];              // [pair parity][warp][head] order-mapped maxima
     float lsum[4][4];              // [warp][head] softmax sums
-    float mL[4];                   // [head] a merge's total sum
+    float mL[4];                   // [head] a merge's total sum, the dropped nodes' partial included
     float mPr[4];                  // [head] a merge's weight of the dropped nodes' partial (value summaries)
     int prefix[1];                 // [groups + 1] first global item of each group; then the merge's
                                    // (max, sum) -> (weight, sum) of every partial, float2 [grid][4]
@@ -98,6 +104,17 @@ __device__ __forceinline__ bool twait(uint64_t* bar, uint32_t parity, TcCtl* ctl
     return false;
 }
 __device__ __forceinline__ bool tc_aborted(TcCtl* ctl) { return *reinterpret_cast<volatile int*>(&ctl->abort) != 0; }
+
+// The piece cost axis: group g's items occupy [cost_start(g), cost_start(g) + n_g), each
+// group preceded by kTCGroupCost items of virtual cost; CTA j covers [j cc, (j + 1) cc).
+// Costs stay below 2^31 (32-bit arithmetic), like the item counts.
+__device__ __forceinline__ uint32_t tc_cost_chunk(int64_t I, int groups, int C) {
+    const uint32_t Ic = static_cast<uint32_t>(I) + static_cast<uint32_t>(kTCGroupCost * groups);
+    return I > 0 ? (Ic + static_cast<uint32_t>(C) - 1) / static_cast<uint32_t>(C) : 1u;
+}
+__device__ __forceinline__ uint32_t tc_cost_start(const int* prefix, int g) {
+    return static_cast<uint32_t>(prefix[g]) + static_cast<uint32_t>(kTCGroupCost * (g + 1));
+}
 
 // Order-preserving map of floats (no NaN) to int, for the integer warp max.
 __device__ __forceinline__ int ord_of(float x) {
@@ -139,6 +156,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         mbar_init(&ctl->ep[2], 1);
         mbar_init(&ctl->mg[0], 4);
         mbar_init(&ctl->mg[1], 4);
+        mbar_init(&ctl->mgb, 1);
         mbar_init(&ctl->pre_ready, 1);
         mbar_init(&ctl->fin, 1);
         fence_mbar_init();
@@ -185,21 +203,29 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         if (lane == 0) ctl->prefix[a.groups] = static_cast<int>(I);
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->pre_ready);
-        const int64_t ch = I > 0 ? (static_cast<uint32_t>(I) + C - 1) / static_cast<uint32_t>(C) : 1;   // items per CTA: one contiguous piece each
+        const uint32_t cc = tc_cost_chunk(I, a.groups, C);   // cost per CTA: one contiguous piece each
         int fills = 0;     // pairs posted (lane 0's count is the one used)
         bool ok = true;
         auto acquire = [&](int f) -> bool {
             return f < kTCStages || twait(&ctl->kv_empty[f % kTCStages], ((f / kTCStages) - 1) & 1, ctl);
         };
-        const int64_t j = blockIdx.x;
-        if (j * ch < I) {
-            const int64_t x_end = min(I, (j + 1) * ch);
+        if (I > 0) {
+            const uint32_t c0 = static_cast<uint32_t>(blockIdx.x) * cc, c1 = c0 + cc;
             int g = 0;
-            for (int64_t x = j * ch; x < x_end && ok;) {
-                while (ctl->prefix[g + 1] <= x) ++g;   // the group holding item x
-                const int64_t g0 = ctl->prefix[g], g1 = ctl->prefix[g + 1];
-                const int64_t seg_end = min(x_end, g1);
-                const int i0 = static_cast<int>(x - g0), nseg = static_cast<int>(seg_end - x);
+            while (g < a.groups && tc_cost_start(ctl->prefix, g) + (ctl->prefix[g + 1] - ctl->prefix[g]) <= c0) ++g;
+            int g_fin = -1;   // the piece's last group with keys in it
+            for (int x = g; x < a.groups && tc_cost_start(ctl->prefix, x) < c1; ++x) {
+                const uint32_t cs = tc_cost_start(ctl->prefix, x);
+                if ((c0 > cs ? static_cast<int>(c0 - cs) : 0) < min(ctl->prefix[x + 1] - ctl->prefix[x], static_cast<int>(c1 - cs)))
+                    g_fin = x;
+            }
+            for (; g < a.groups && tc_cost_start(ctl->prefix, g) < c1 && ok; ++g) {
+                const uint32_t cs = tc_cost_start(ctl->prefix, g);
+                const int ng = ctl->prefix[g + 1] - ctl->prefix[g];
+                const int i0 = c0 > cs ? static_cast<int>(c0 - cs) : 0;
+                const int i1 = min(ng, static_cast<int>(c1 - cs));
+                if (i0 >= i1) continue;
+                const int nseg = i1 - i0;
                 // CTAs start at different points of their segments (the order of the keys does
                 // not matter to the softmax), so concurrent CTAs stream different address patterns
                 const int rot = static_cast<int>((static_cast<uint32_t>(blockIdx.x) * 2654435761u) %
@@ -244,7 +270,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                             d.heads1 = c1 > 0 ? m1 : 0u;
                             d.group = g;
                             d.split = blockIdx.x;
-                            d.flags = (vb + p + 2 >= nseg ? 1 : 0) | (vb + p == 0 ? 2 : 0);
+                            d.flags = (vb + p + 2 >= nseg ? (g == g_fin ? 5 : 1) : 0) | (vb + p == 0 ? 2 : 0);
                             unsigned char* sb = stage(slot);
                             uint64_t* bar = &ctl->kv_full[slot];
                             const uint32_t bytes = (c0 > 0 ? 2 * kTCSpan : 0u) + (c1 > 0 ? 2 * kTCSpan : 0u) + kTCQBytes;
@@ -272,7 +298,6 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                         ++fills;
                     }
                 }
-                x = seg_end;
             }
         }
         if (lane == 0) {
@@ -369,9 +394,8 @@ __global__ void __launch_bounds__(kTCThreads, 1)
             l[h] = 0.f;
         }
         twait(&ctl->pre_ready, 0, ctl);   // the group prefix (first read by an epilogue)
-        const int64_t I = ctl->prefix[a.groups];
-        const int64_t ch = I > 0 ? (static_cast<uint32_t>(I) + C - 1) / static_cast<uint32_t>(C) : 1;
-        uint32_t e = 0, nm = 0;   // epilogues and merges so far
+        const uint32_t cc = tc_cost_chunk(ctl->prefix[a.groups], a.groups, C);
+        uint32_t e = 0, nm = 0, nmg = 0;   // epilogues, merges, merges from global memory
         float2* mbuf = reinterpret_cast<float2*>(reinterpret_cast<unsigned char*>(ctl) + tc_merge_offset(a.groups));
         for (uint32_t g = 0;; ++g) {
             if (tc_aborted(ctl)) break;
@@ -494,54 +518,68 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                 if (lane == 0) mbar_arrive(&ctl->ep[1]);
                 if (i == 0) {
                     twait(&ctl->ep[1], e & 1u, ctl);
-                    const int sp = partials_of(ctl->prefix[grp], ctl->prefix[grp + 1], ch, C);
+                    // the CTAs whose pieces meet the group's items: slots j0 .. j1
+                    const uint32_t cs = tc_cost_start(ctl->prefix, grp);
+                    const int j0 = static_cast<int>(cs / cc);
+                    const int j1 = static_cast<int>((cs + (ctl->prefix[grp + 1] - ctl->prefix[grp]) - 1) / cc);
+                    const int sp = j1 - j0 + 1;
                     const uint32_t done = atomic_add_acq_rel_gpu(&a.counters[grp], 1u);
                     ctl->last_flag = done == static_cast<uint32_t>(sp - 1);
                     ctl->sp = sp;
+                    ctl->sp0 = j0;
                     mbar_arrive(&ctl->ep[2]);
                 }
                 twait(&ctl->ep[2], e & 1u, ctl);
                 if (ctl->last_flag) {
-                    // ---- this CTA closes the group: merge its partials into O.  The (max, sum)
-                    // pairs go to shared memory in parallel; warp h turns them into the weights
-                    // 2^(m_k - M_h) and the total sum; thread i sums dimension i over the
-                    // partials from registers, kTCRegPartials partials per round of loads (the
-                    // first round issued together with the (max, sum) loads).
+                    // ---- this CTA closes the group: merge its partials (slots sp0 .. sp0 + sp - 1,
+                    // one contiguous run of the workspace) into O.  After the CTA's last pair the
+                    // stage buffers are idle, and two bulk copies bring the run's (max, sum) pairs
+                    // and accumulators into them; a merge in mid-piece (rare) gathers the pairs
+                    // into shared memory and reads the accumulators from global memory.  Warp h
+                    // forms head h's weights 2^(m_k - M_h) in place and the total sum; then thread
+                    // i sums dimension i over the partials with shared-memory loads and FMAs only.
+                    // The loops stay rolled: this code runs once per group, from a cold
+                    // instruction cache.
                     const int sp = ctl->sp;
                     const int s = grp / a.Hkv, kv = grp % a.Hkv;
-                    const int64_t pb0 = static_cast<int64_t>(grp) * kSplitMax * G;
-                    const int slot0 = static_cast<int>((static_cast<uint32_t>(ctl->prefix[grp]) / static_cast<uint32_t>(ch)) % C);   // partial k at slot (slot0+k) % C
-                    float xr[kTCRegPartials][G];
-                    auto load_round = [&](int k0) {
+                    const int64_t pb0 = (static_cast<int64_t>(grp) * kSplitMax + ctl->sp0) * G;   // partial k, head h: entry pb0 + k G + h
+                    const int64_t orow0 = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G;
+                    const uint32_t acc_bytes = static_cast<uint32_t>(sp * G * D) * 4u, ml_bytes = static_cast<uint32_t>(sp * G) * 8u;
+                    const bool staged = (d.flags & 4) != 0 && acc_bytes + ml_bytes <= kTCStages * kTCStageBytes;
+                    const float* sacc = reinterpret_cast<const float*>(stage(0));
+                    float2* sml = staged ? reinterpret_cast<float2*>(stage(0) + acc_bytes) : mbuf;
+                    // value summaries: the dropped nodes' partial of each head's query joins the merge
+                    float pa[G];
 #pragma unroll
-                        for (int k = 0; k < kTCRegPartials; ++k)
-#pragma unroll
-                            for (int h = 0; h < G; ++h)
-                                xr[k][h] = k0 + k < sp
-                                    ? __ldcg(a.part_acc + ((pb0 + static_cast<int64_t>((slot0 + k0 + k) % C) * G + h) * D + i))
-                                    : 0.f;
-                    };
-                    load_round(0);
-                    for (int x = i; x < sp * G; x += 128) {
-                        const int k = x / G, h = x % G;
-                        mbuf[k * 4 + h] = __ldcg(&a.part_ml[pb0 + ((slot0 + k) % C) * G + h]);
+                    for (int h = 0; h < G; ++h) pa[h] = a.pr_acc ? a.pr_acc[(orow0 + h) * D + i] : 0.f;
+                    if (staged) {
+                        if (i == 0) {
+                            // the count's acquire made the partials visible to this thread; the
+                            // bulk copies read them through the async proxy
+                            umma::fence_proxy_async_global();
+                            mbar_arrive_expect_tx(&ctl->mgb, acc_bytes + ml_bytes);
+                            bulk_g2s(stage(0), a.part_acc + pb0 * D, acc_bytes, &ctl->mgb);
+                            bulk_g2s(stage(0) + acc_bytes, a.part_ml + pb0, ml_bytes, &ctl->mgb);
+                        }
+                        twait(&ctl->mgb, (nm - nmg) & 1u, ctl);
+                    } else {
+                        for (int x = i; x < sp * G; x += 128) mbuf[x] = __ldcg(&a.part_ml[pb0 + x]);
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&ctl->mg[0]);
+                        twait(&ctl->mg[0], nmg & 1u, ctl);
+                        ++nmg;
                     }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&ctl->mg[0]);
-                    twait(&ctl->mg[0], nm & 1u, ctl);
                     if (warp < G) {
                         const int h = warp;
-                        // value summaries: the dropped nodes' partial of this head's query joins the merge
-                        const float2 pr = a.pr_ml ? a.pr_ml[(static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + h]
-                                                  : make_float2(-INFINITY, 0.f);
-                        float M = -INFINITY;
-                        for (int k = lane; k < sp; k += 32) M = fmaxf(M, mbuf[k * 4 + h].x);
-                        M = fmaxf(warp_max(M), pr.x);
+                        const float2 pr = a.pr_ml ? a.pr_ml[orow0 + h] : make_float2(-INFINITY, 0.f);
+                        float M = pr.x;
+                        for (int k = lane; k < sp; k += 32) M = fmaxf(M, sml[k * G + h].x);
+                        M = warp_max(M);
                         float Ls = 0.f;
                         for (int k = lane; k < sp; k += 32) {
-                            const float2 ml = mbuf[k * 4 + h];
+                            const float2 ml = sml[k * G + h];
                             const float f = M == -INFINITY ? 0.f : exp2f(ml.x - M);
-                            mbuf[k * 4 + h].x = f;
+                            sml[k * G + h].x = f;
                             Ls = fmaf(f, ml.y, Ls);
                         }
                         Ls = warp_sum(Ls);
@@ -556,24 +594,26 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                     twait(&ctl->mg[1], nm & 1u, ctl);
                     float o[G];
 #pragma unroll
-                    for (int h = 0; h < G; ++h) o[h] = 0.f;
-                    for (int k0 = 0; k0 < sp; k0 += kTCRegPartials) {
-                        if (k0 > 0) load_round(k0);
+                    for (int h = 0; h < G; ++h) o[h] = ctl->mPr[h] * pa[h];
+                    if (staged) {
+#pragma unroll 4
+                        for (int k = 0; k < sp; ++k)
 #pragma unroll
-                        for (int k = 0; k < kTCRegPartials; ++k)
-                            if (k0 + k < sp)
+                            for (int h = 0; h < G; ++h) o[h] = fmaf(sml[k * G + h].x, sacc[(k * G + h) * D + i], o[h]);
+                    } else {
+#pragma unroll 4
+                        for (int k = 0; k < sp; ++k)
 #pragma unroll
-                                for (int h = 0; h < G; ++h) o[h] = fmaf(mbuf[(k0 + k) * 4 + h].x, xr[k][h], o[h]);
+                            for (int h = 0; h < G; ++h)
+                                o[h] = fmaf(sml[k * G + h].x, __ldcg(a.part_acc + (pb0 + k * G + h) * D + i), o[h]);
                     }
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
                         const float Ls = ctl->mL[h];
-                        const int64_t orow = (static_cast<int64_t>(s) * a.n_q + (a.n_q - 1)) * a.Hq + kv * G + h;
-                        if (a.pr_acc) o[h] = fmaf(ctl->mPr[h], a.pr_acc[orow * D + i], o[h]);
-                        a.O[orow * D + i] = Ls > 0.f ? o[h] / Ls : 0.f;
+                        a.O[(orow0 + h) * D + i] = Ls > 0.f ? o[h] / Ls : 0.f;
                     }
-                    if (i == 0) a.counters[grp] = 0u;
                     ++nm;
+                    if (i == 0) a.counters[grp] = 0u;
                 }
                 ++e;
             }

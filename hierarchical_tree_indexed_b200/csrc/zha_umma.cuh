@@ -84,6 +84,11 @@ __device__ __forceinline__ void fence_after_sync() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Orders this thread's view of global memory (generic proxy) before its later bulk copies
+// (async proxy) that read it.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 // 32 consecutive fp32 columns of this warp's 32 TMEM lanes (lane = thread's
 // row), waiting for the load to land before returning.
