@@ -70,6 +70,7 @@ constexpr int kCutSplit = 64;      // a crossing bin with more members is split 
 
 struct CutSmem {
     unsigned long long bins[kCutBins];     // zero between cuts
+    uint32_t bw[2][kCutBins];              // a pass's masses as 32-bit words (low, high); zero between cuts
     unsigned long long mkey[kCutMembers];  // crossing-bin members: order key and mass
     unsigned long long mmass[kCutMembers];
     unsigned long long above, target;      // mass ordered before the crossing (sub-)bin; the target
@@ -257,9 +258,15 @@ __device__ __forceinline__ void cut_locate(unsigned long long* bins, unsigned lo
 //   4. member k is kept iff the mass of the members ordered before it, plus the mass ordered
 //      before its (sub-)bin, is below the target (its bit joins the ballot words);
 //   5. a scan of the ballot words' counts places every word's kept ids, in slot order.
+// A pass adds each candidate's 64-bit mass to its bin as two 32-bit shared atomics (the low
+// word, then the high word plus the low word's carry, only when not zero): thousands of
+// candidates can share a bin, and contended 32-bit shared atomics are cheaper.  The words are
+// gathered into cs.bins before the crossing bin is looked for.
+// priv: when not null, kRouteWarps private pairs of word rows (shared memory otherwise idle),
+// so that each warp's atomics go to its own words.
 template <typename NodeOf>
 __device__ int block_cut(const float* sc, int nc, float p, float mx, int32_t* out, CutSmem& cs, uint32_t* kball,
-                         int32_t* kpre, int* scan, NodeOf node_of) {
+                         int32_t* kpre, int* scan, NodeOf node_of, unsigned long long* priv = nullptr) {
     constexpr int NT = kRouteThreads;
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     if (mx == -INFINITY || nc <= 0) return 0;   // uniform
@@ -274,15 +281,47 @@ __device__ int block_cut(const float* sc, int nc, float p, float mx, int32_t* ou
     const bool keep_all = p >= 1.0f;
     const int ngrp = (nc + 31) / 32;
     int cbin = kCutBins, sbin = -1;
+    uint32_t* wlo = priv ? reinterpret_cast<uint32_t*>(priv) + w * 2 * kCutBins : cs.bw[0];   // this warp's words
+    uint32_t* whi = wlo + kCutBins;
+    auto add_mass = [&](int bn, unsigned long long m) {
+        const uint32_t lo = static_cast<uint32_t>(m), hi = static_cast<uint32_t>(m >> 32);
+        const uint32_t old = atomicAdd(&wlo[bn], lo);
+        const uint32_t hc = hi + (old + lo < old ? 1u : 0u);   // the low word's carry
+        if (hc) atomicAdd(&whi[bn], hc);
+    };
+    auto private_zero = [&]() {   // before a pass: this warp's words
+        if (priv)
+            for (int x = lane; x < 2 * kCutBins; x += 32) wlo[x] = 0u;
+        __syncwarp();
+    };
+    auto gather = [&]() {   // after a pass and a barrier: the words into cs.bins (shared words left zero), a barrier
+        for (int x = t; x < kCutBins; x += NT) {
+            unsigned long long v = 0ull;
+            if (priv) {
+                for (int k = 0; k < kRouteWarps; ++k) {
+                    const uint32_t* pw = reinterpret_cast<const uint32_t*>(priv) + k * 2 * kCutBins;
+                    v += (static_cast<unsigned long long>(pw[kCutBins + x]) << 32) + pw[x];
+                }
+            } else {
+                v = (static_cast<unsigned long long>(cs.bw[1][x]) << 32) + cs.bw[0][x];
+                cs.bw[0][x] = 0u;
+                cs.bw[1][x] = 0u;
+            }
+            cs.bins[x] = v;
+        }
+        __syncthreads();
+    };
     if (!keep_all) {
+        private_zero();
         for (int i = t; i < nc; i += NT) {
             const float s = sc[i];
             if (s == -INFINITY) continue;
             const unsigned long long m = score_mass(s, mx);
-            if (m) atomicAdd(&cs.bins[cut_bin(s, mx)], m);
+            if (m) add_mass(cut_bin(s, mx), m);
         }
         if (t == 0) { cs.nm = 0; cs.target = 0; cs.sbin = -1; }
         __syncthreads();
+        gather();
         if (w == 0) cut_locate(cs.bins, 0ull, p, &cs.target, &cs.cbin, &cs.above);
         __syncthreads();
         cbin = cs.cbin;
@@ -305,14 +344,16 @@ __device__ int block_cut(const float* sc, int nc, float p, float mx, int32_t* ou
     if (!keep_all) {
         __syncthreads();
         if (cs.nm > kCutSplit) {   // uniform: split the crossing bin (pairwise ranks grow as members^2)
+            private_zero();
             for (int i = t; i < nc; i += NT) {
                 const float s = sc[i];
                 if (s != -INFINITY && cut_bin(s, mx) == cbin) {
                     const unsigned long long m = score_mass(s, mx);
-                    if (m) atomicAdd(&cs.bins[cut_sub(s, mx, cbin)], m);
+                    if (m) add_mass(cut_sub(s, mx, cbin), m);
                 }
             }
             __syncthreads();
+            gather();
             if (t == 0) cs.nm = 0;
             if (w == 0) cut_locate(cs.bins, cs.above, p, &cs.target, &cs.sbin, &cs.above);
             __syncthreads();
@@ -624,7 +665,11 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
     (void)N;
     if (tid < D) sm.q[tid] = q_in * a.scale;   // q_in: element tid of the query (loaded by the caller)
     if (tid < 2) sm.mxkey[tid] = ord_key(-INFINITY);
-    for (int i = tid; i < kCutBins; i += kRouteThreads) sm.cut.bins[i] = 0ull;
+    for (int i = tid; i < kCutBins; i += kRouteThreads) {
+        sm.cut.bins[i] = 0ull;
+        sm.cut.bw[0][i] = 0u;
+        sm.cut.bw[1][i] = 0u;
+    }
     constexpr bool vsum = VS && !MP;   // value summaries (R = 1)
     if constexpr (vsum) {
         if (tid < D) sm.pr_acc[tid] = 0.f;
@@ -789,8 +834,12 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
         }
         {
             const bool big = (nc + 31) / 32 > kScoresSmem / 32;   // ballot words in the workspace
+            // with the scores in the workspace, sm.scores holds the warps' private bins
+            static_assert(kRouteWarps * 2 * kCutBins * sizeof(uint32_t) <= sizeof(float) * kScoresSmem,
+                          "private bin words fit the score buffer");
             np = block_cut(sc, nc, a.p[l - 1], key_ord(*mxk), bufs[nxt], sm.cut, big ? ws_kb : sm.keep_ballot,
-                           big ? reinterpret_cast<int32_t*>(ws_kb) + a.kb_cap : sm.keep_prefix, sm.scan, node_of);
+                           big ? reinterpret_cast<int32_t*>(ws_kb) + a.kb_cap : sm.keep_prefix, sm.scan, node_of,
+                           sc != sm.scores ? reinterpret_cast<unsigned long long*>(sm.scores) : nullptr);
         }
         __syncthreads();
         if (region && l == L) cluster_wait();   // CTA 0 has cleared the region
