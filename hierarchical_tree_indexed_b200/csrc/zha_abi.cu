@@ -369,10 +369,21 @@ bool plan_fits_route(const zha_config* c, const TreeLayout& lay, const WsLayout&
     return need + 1024 <= static_cast<size_t>(di.smem_optin);
 }
 
+// The cluster's CTAs help each other with levels too large for shared memory where that can
+// pay: clusters (the plan fused) that leave at least half the SMs idle, over trees whose leaf
+// level alone exceeds the router's shared score buffer.
+bool route_help_pays(const RouteArgs& a, int ctas, int G) {
+    DevInfo di;
+    if (!a.fuse_plan || G < 2 || a.tree.R > 1 || a.pr_ml || dev_info(&di) != ZHA_OK) return false;
+    return 2 * ctas <= di.sms && a.tree.ncap[0] > kScoresSmem;
+}
+
 template <typename T, int D, int NVR>
 int run_route_t(const RouteArgs& a, int ctas, int G, cudaStream_t st) {
     auto kern = a.tree.R > 1 ? route_decode_kernel<T, D, NVR, true>
-                : a.pr_ml ? route_decode_kernel<T, D, NVR, false, true> : route_decode_kernel<T, D, NVR, false>;
+                : a.pr_ml ? route_decode_kernel<T, D, NVR, false, true>
+                : route_help_pays(a, ctas, G) ? route_decode_kernel<T, D, NVR, false, false, true>
+                : route_decode_kernel<T, D, NVR, false>;
     const size_t smem = sizeof(RouteSmem) + (a.fuse_plan ? 4 * static_cast<size_t>(a.region_words) : 0);
     ZHA_TRY(allow_smem(kern, smem));
     cudaLaunchConfig_t lc = {};

@@ -78,6 +78,27 @@ struct CutSmem {
     int cnt;                               // the kept count (small cuts)
 };
 
+// A level's scan offered to the other CTAs of the cluster (decode, the plan fused): the owner
+// publishes where the jobs (kept parents) and their outputs are, then claims jobs from `claim`
+// like its helpers.  Shared addresses are this CTA's; a helper maps them to the owner's.
+// Only levels whose scores live in the workspace (more than kScoresSmem candidates) are
+// offered: below that the claims' round trips cost more than the help saves (measured at 1M).
+struct HelpSmem {
+    uint32_t claim;            // (level << 24) | next job; jobs are claimed two at a time; 0: none
+    uint32_t done;             // jobs of the offered level finished, helpers' included
+    uint32_t walk_done;        // this CTA's walk is over: its helpers may leave
+    int level, np, b;
+    int64_t nl;                // nodes of the offered level
+    const float* kh;           // the level's summaries and biases of this slice (global memory)
+    const float* bh;
+    float* sc_global;          // the scores, when they live in the workspace,
+    uint32_t sc_smem;          //   else in this CTA's shared memory
+    uint32_t par_smem;         // the kept parents in shared memory,
+    const int32_t* par_global; //   or in the workspace
+    uint32_t mx_smem;          // the level's max score slot (order-mapped int)
+    uint32_t q_smem;           // the scaled query
+};
+
 struct RouteSmem {
     float scores[kScoresSmem];
     int32_t parents[2][kParentsSmem];
@@ -94,6 +115,7 @@ struct RouteSmem {
     int scan[kRouteWarps + 1];
     float redf[kRouteWarps];
     int redi[kRouteWarps];
+    HelpSmem help;                     // last: the buffers above keep their offsets
 };
 
 // Order-preserving map of a float (no NaN) to int, and back: the max of scores as an int max.
@@ -651,13 +673,78 @@ __device__ void add_dropped(const float* sc, const int32_t* par, int np_par, int
     __syncthreads();
 }
 
+// The scan of a level offered to the cluster (single plane): the descriptor is published
+// (seqlock: level 0 while the fields change, the level after them, then the claim word with
+// release order at cluster scope), the CTA's warps claim jobs two at a time like its helpers,
+// and thread 0 waits (bounded) until every job is done, the helpers' included.  The caller's
+// barrier follows.
+template <int D, int NVR>
+__device__ __forceinline__ void scan_offered(RouteSmem& sm, const float* kh, const float* bh, const int32_t* par,
+                                          bool par_in_smem, int np, int b, int64_t nl, float* sc, int* mxk, int l,
+                                          uint32_t head) {
+    constexpr int VF = D / 32;
+    const int tid = threadIdx.x, lane = tid & 31;
+    if (tid == 0) {
+        HelpSmem& hs = sm.help;
+        hs.level = 0;
+        fence_acq_rel_cluster();
+        hs.np = np;
+        hs.b = b;
+        hs.nl = nl;
+        hs.kh = kh;
+        hs.bh = bh;
+        hs.sc_global = sc;
+        hs.sc_smem = 0u;
+        hs.par_smem = par_in_smem ? smem_addr(par) : 0u;
+        hs.par_global = par_in_smem ? nullptr : par;
+        hs.mx_smem = smem_addr(mxk);
+        hs.q_smem = smem_addr(sm.q);
+        hs.done = 0u;
+        fence_acq_rel_cluster();
+        hs.level = l;
+        dsmem_st_release_u32(cluster_map(&hs.claim, head), static_cast<uint32_t>(l) << 24);
+    }
+    __syncthreads();
+    float qv[VF];
+#pragma unroll
+    for (int e = 0; e < VF; ++e) qv[e] = sm.q[lane * VF + e];
+    for (;;) {
+        uint32_t jw = 0u;
+        if (lane == 0) jw = atomicAdd(&sm.help.claim, 2u);
+        jw = __shfl_sync(0xffffffffu, jw, 0);
+        const int ji = static_cast<int>(jw & 0xffffffu);
+        if ((jw >> 24) != static_cast<uint32_t>(l) || ji >= np) break;
+        const int64_t c0 = static_cast<int64_t>(par[ji]) * b;
+        const int cnt0 = static_cast<int>(min(static_cast<int64_t>(b), nl - c0));
+        if (ji + 1 < np) {
+            const int64_t c1 = static_cast<int64_t>(par[ji + 1]) * b;
+            const int cnt1 = static_cast<int>(min(static_cast<int64_t>(b), nl - c1));
+            scan_children2<D, NVR>(kh + c0 * D, bh + c0, cnt0, kh + c1 * D, bh + c1, cnt1, b, qv,
+                                   sc + static_cast<int64_t>(ji) * b, sc + static_cast<int64_t>(ji + 1) * b, mxk, mxk);
+        } else {
+            scan_children<D, NVR>(kh + c0 * D, bh + c0, cnt0, b, qv, sc + static_cast<int64_t>(ji) * b, D, 1, true, mxk);
+        }
+        __syncwarp();
+        if (lane == 0) atomicAdd(&sm.help.done, ji + 1 < np ? 2u : 1u);
+    }
+    if (tid == 0) {
+        const uint32_t da = cluster_map(&sm.help.done, head);
+        const uint64_t t0 = global_timer_ns();
+        while (dsmem_ld_acquire_u32(da) < static_cast<uint32_t>(np))
+            if (global_timer_ns() - t0 > kWaitLongNs) {
+                raise_status(ZHA_ERR_TIMEOUT);
+                break;
+            }
+    }
+}
+
 // The top-down walk of one decode query (the body of route_decode_kernel).  With
 // `region` != 0 (fuse_plan) the kept nodes of every level are OR'd into the bitmaps of
 // the cluster's CTA 0 (shared::cluster address of its plan region): level 1 into head
 // `head`'s plan bitmap, level l >= 2 into the level's bitmap of kept nodes.  The walk
 // then waits on the cluster barrier that CTA 0 arrived on after clearing the region,
 // once, right after the top level's cut (before its first remote write).
-template <typename T, int D, int NVR, bool MP, bool VS>
+template <typename T, int D, int NVR, bool MP, bool VS, bool HELP>
 __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, int cta, int64_t row, int64_t slice,
                                            int64_t N, int64_t Ntree, uint32_t region, int head, float q_in) {
     constexpr int VF = D / 32;   // fp32 summary elements per lane
@@ -754,8 +841,7 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
                     mx = nullptr;
                 }
             };
-            for (int ji = w; ji < jobs; ji += 2 * kRouteWarps) {
-                const int jj = ji + kRouteWarps;   // a second job in the same round, if any
+            auto two_jobs = [&](int ji, int jj) {   // jobs ji and jj (jj >= jobs: none)
                 const float *k0, *b0, *k1 = nullptr, *b1 = nullptr;
                 int cnt0, cnt1 = 0;
                 float *o0, *o1 = nullptr;
@@ -765,7 +851,7 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
                 if constexpr (!MP) {
                     if (jj < jobs) scan_children2<D, NVR>(k0, b0, cnt0, k1, b1, cnt1, b, qv, o0, o1, m0, m1);
                     else scan_children<D, NVR>(k0, b0, cnt0, b, qv, o0, D, 1, true, m0);
-                    continue;
+                    return;
                 }
                 if (jj < jobs)
                     for (int pl = 0; pl < R; ++pl)
@@ -774,6 +860,17 @@ __device__ __forceinline__ void route_walk(const RouteArgs& a, RouteSmem& sm, in
                 for (int pl = 0; pl < R; ++pl)
                     scan_children<D, NVR>(k0 + pl * D, b0 + pl, cnt0, b, qv, o0, R * D, R, pl == 0,
                                           pl == R - 1 ? m0 : nullptr);
+            };
+            // a large level below the top is offered to the cluster's CTAs whose walks are over
+            bool offered = false;
+            if constexpr (HELP && !MP && !vsum) {
+                if (region != 0u && l < L && sc != sm.scores) {   // uniform
+                    scan_offered<D, NVR>(sm, kh, bh, par, cur < 2, np, b, nl, sc, mxk, l, static_cast<uint32_t>(head));
+                    offered = true;
+                }
+            }
+            if (!offered) {
+                for (int ji = w; ji < jobs; ji += 2 * kRouteWarps) two_jobs(ji, ji + kRouteWarps);   // two per round
             }
         }
         __syncthreads();
@@ -901,11 +998,131 @@ struct ScannedTail {
 // MP: nodes carry several reference-query planes (R > 1); R = 1 compiles the
 // single-plane scan alone.  VS: the tree holds value summaries (R = 1): the nodes the
 // cut drops are summed into a per-query partial.
+// After its own walk, a CTA of the cluster scans jobs that the others offer (HelpSmem) until
+// every other CTA's walk is over.  A warp claims two jobs at a time over DSMEM, reads the
+// owner's descriptor and query the first time it meets an offer, scores the jobs into its own
+// (now idle) score buffer, copies the scores where the owner keeps them, raises the owner's level
+// max, and adds to its done count with release order.  Every wait is bounded.
+template <int D, int NVR>
+__device__ void route_help(RouteSmem& sm, uint32_t rank, uint32_t G) {
+    constexpr int VF = D / 32;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    if (threadIdx.x == 0) dsmem_st_release_u32(cluster_map(&sm.help.walk_done, rank), 1u);
+    float* scratch = sm.scores + w * 64;
+    int c_rank = -1, c_level = -1, c_np = 0, c_b = 1;
+    int64_t c_nl = 0;
+    const float *c_kh = nullptr, *c_bh = nullptr;
+    float* c_scg = nullptr;
+    const int32_t* c_parg = nullptr;
+    uint32_t c_scs = 0u, c_pars = 0u, c_mx = 0u, c_done = 0u;
+    float qv[VF];
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        bool all_over = true, worked = false;
+        for (uint32_t r = 0; r < G; ++r) {
+            if (r == rank) continue;
+            const uint32_t claim_r = cluster_map(&sm.help.claim, r);
+            uint32_t wd = 0u, cw = 0u;
+            if (lane == 0) {
+                wd = dsmem_ld_acquire_u32(cluster_map(&sm.help.walk_done, r));
+                cw = dsmem_ld_u32(claim_r);
+            }
+            wd = __shfl_sync(0xffffffffu, wd, 0);
+            cw = __shfl_sync(0xffffffffu, cw, 0);
+            if (!wd) all_over = false;
+            if (cw == 0u) continue;   // nothing offered yet
+            if (static_cast<int>(r) == c_rank && static_cast<int>(cw >> 24) == c_level &&
+                static_cast<int>(cw & 0xffffffu) >= c_np)
+                continue;   // that offer is taken up
+            uint32_t jw = 0u;
+            if (lane == 0) jw = dsmem_atom_add_u32(claim_r, 2u);
+            jw = __shfl_sync(0xffffffffu, jw, 0);
+            fence_acq_rel_cluster();   // the descriptor written before the claim word
+            const int jl = static_cast<int>(jw >> 24), ji = static_cast<int>(jw & 0xffffffu);
+            if (static_cast<int>(r) != c_rank || jl != c_level) {
+                const uint32_t hb = cluster_map(&sm.help, r);
+                auto fld = [&](const void* f) {
+                    return hb + static_cast<uint32_t>(reinterpret_cast<const char*>(f) - reinterpret_cast<const char*>(&sm.help));
+                };
+                // seqlock read: the level before and after the fields must both be the claim's,
+                // else the claim is a stale one of an offer the owner has closed
+                int lv = 0;
+                if (lane == 0) lv = static_cast<int>(dsmem_ld_u32(fld(&sm.help.level)));
+                lv = __shfl_sync(0xffffffffu, lv, 0);
+                if (lv != jl) continue;
+                c_np = static_cast<int>(dsmem_ld_u32(fld(&sm.help.np)));
+                c_b = static_cast<int>(dsmem_ld_u32(fld(&sm.help.b)));
+                c_nl = static_cast<int64_t>(dsmem_ld_u64(fld(&sm.help.nl)));
+                c_kh = reinterpret_cast<const float*>(dsmem_ld_u64(fld(&sm.help.kh)));
+                c_bh = reinterpret_cast<const float*>(dsmem_ld_u64(fld(&sm.help.bh)));
+                c_scg = reinterpret_cast<float*>(dsmem_ld_u64(fld(&sm.help.sc_global)));
+                c_parg = reinterpret_cast<const int32_t*>(dsmem_ld_u64(fld(&sm.help.par_global)));
+                const uint32_t scs = dsmem_ld_u32(fld(&sm.help.sc_smem)), pars = dsmem_ld_u32(fld(&sm.help.par_smem));
+                c_scs = scs ? cluster_map_addr(scs, r) : 0u;
+                c_pars = pars ? cluster_map_addr(pars, r) : 0u;
+                c_mx = cluster_map_addr(dsmem_ld_u32(fld(&sm.help.mx_smem)), r);
+                c_done = cluster_map(&sm.help.done, r);
+                const uint32_t qa = cluster_map_addr(dsmem_ld_u32(fld(&sm.help.q_smem)), r);
+#pragma unroll
+                for (int e = 0; e < VF; ++e) qv[e] = dsmem_ld_f32(qa + 4u * static_cast<uint32_t>(lane * VF + e));
+                fence_acq_rel_cluster();
+                if (lane == 0) lv = static_cast<int>(dsmem_ld_u32(fld(&sm.help.level)));
+                lv = __shfl_sync(0xffffffffu, lv, 0);
+                if (lv != jl) {
+                    c_rank = -1;
+                    continue;
+                }
+                c_rank = static_cast<int>(r);
+                c_level = jl;
+            }
+            if (ji >= c_np) continue;
+            worked = true;
+            const int nj = ji + 1 < c_np ? 2 : 1;
+            auto par_of = [&](int j) {
+                return c_pars ? static_cast<int32_t>(dsmem_ld_u32(c_pars + 4u * static_cast<uint32_t>(j))) : c_parg[j];
+            };
+            const int64_t p0 = par_of(ji), p1 = nj > 1 ? par_of(ji + 1) : 0;
+            const int64_t c0 = p0 * c_b, c1 = p1 * c_b;
+            const int cnt0 = static_cast<int>(min(static_cast<int64_t>(c_b), c_nl - c0));
+            const int cnt1 = nj > 1 ? static_cast<int>(min(static_cast<int64_t>(c_b), c_nl - c1)) : 0;
+            if (lane == 0) sm.redi[w] = ord_key(-INFINITY);
+            __syncwarp();
+            if (nj > 1)
+                scan_children2<D, NVR>(c_kh + c0 * D, c_bh + c0, cnt0, c_kh + c1 * D, c_bh + c1, cnt1, c_b, qv, scratch,
+                                       scratch + 32, &sm.redi[w], &sm.redi[w]);
+            else
+                scan_children<D, NVR>(c_kh + c0 * D, c_bh + c0, cnt0, c_b, qv, scratch, D, 1, true, &sm.redi[w]);
+            __syncwarp();
+            for (int x = lane; x < nj * c_b; x += 32) {   // the owner's slots ji b .. (ji + nj) b
+                const float v = scratch[(x / c_b) * 32 + x % c_b];
+                const int64_t dst = static_cast<int64_t>(ji) * c_b + x;
+                if (c_scg) c_scg[dst] = v;
+                else dsmem_st_f32(c_scs + 4u * static_cast<uint32_t>(dst), v);
+            }
+            __syncwarp();
+            if (lane == 0) {
+                dsmem_red_max_s32(c_mx, sm.redi[w]);
+                dsmem_red_add_release_u32(c_done, static_cast<uint32_t>(nj));
+            }
+        }
+        if (all_over) break;
+        if (!worked) __nanosleep(256);   // polling: leave the owners' shared memory some quiet
+        bool expired = false;
+        if (lane == 0) expired = !worked && global_timer_ns() - t0 > kWaitLongNs;
+        if (__shfl_sync(0xffffffffu, expired, 0)) {
+            if (lane == 0) raise_status(ZHA_ERR_TIMEOUT);
+            break;
+        }
+    }
+}
+
 // fuse_plan: launched as clusters of G CTAs, the G query heads of one (sequence, KV
 // head) (cluster rank = head).  CTA 0 clears its plan region, the heads OR their kept
 // nodes into it (DSMEM), and after a cluster barrier CTA 0 builds the group's gather
 // plan from its own shared memory.
-template <typename T, int D, int NVR, bool MP, bool VS = false>
+// HELP: the cluster's CTAs help each other scan levels too large for shared memory (chosen by
+// the host where the launch leaves SMs idle; the code is not compiled into the other variants).
+template <typename T, int D, int NVR, bool MP, bool VS = false, bool HELP = false>
 __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     RouteSmem& sm = *reinterpret_cast<RouteSmem*>(smem_raw);
@@ -924,7 +1141,14 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
     if (fused) {
         if (rank == 0)
             for (int i = tid; i < a.region_words; i += kRouteThreads) region[i] = 0u;
-        cluster_arrive();   // waited on by the walk before its first remote write
+        if constexpr (HELP)
+            if (tid == 0) {
+                sm.help.claim = 0u;
+                sm.help.done = 0u;
+                sm.help.walk_done = 0u;
+                sm.help.level = 0;
+            }
+        cluster_arrive();   // waited on by the walk before its first remote write (or help)
     }
     const int64_t N = a.N[s];
     const int64_t Ntree = a.tree.n_tree[s];
@@ -933,8 +1157,10 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_decode_kernel(RouteArg
         if (tid == 0) { raise_status(ZHA_ERR_INVALID_ARG); a.sel_count[row] = 0; a.cand[row] = 0; }
         if (fused) cluster_wait();
     } else {
-        route_walk<T, D, NVR, MP, VS>(a, sm, cta, row, slice, N, Ntree, fused ? cluster_map(region, 0) : 0u,
-                                      static_cast<int>(rank), q_in);
+        route_walk<T, D, NVR, MP, VS, HELP>(a, sm, cta, row, slice, N, Ntree, fused ? cluster_map(region, 0) : 0u,
+                                            static_cast<int>(rank), q_in);
+        if constexpr (HELP && !MP && !VS)
+            if (fused && G > 1) route_help<D, NVR>(sm, rank, static_cast<uint32_t>(G));
     }
     if (fused) {
         // every head's kept nodes are in CTA 0's region; the other CTAs are done with it

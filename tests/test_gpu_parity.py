@@ -157,6 +157,33 @@ def test_large_candidate_sets(p):
     assert_status_clean()
 
 
+def test_offered_level_exact_ties():
+    """A leaf level of 9,999 candidates per head (all keys zero, p = 1 above it), more than the
+    router's shared score buffer holds: the decode router offers its scan to the other CTAs of
+    the cluster (one KV head, four query heads, a launch that leaves SMs idle) and the scores come
+    from whichever CTA claimed each parent.  Every score is equal, so p = 0.5 must keep exactly the
+    5,000 lowest blocks (an odd count, so that the cut does not fall exactly on p)."""
+    d, G = 128, 4
+    N = 9999 * 64
+    K = torch.zeros((1, 1, N, d), dtype=torch.bfloat16)
+    V = torch.randn((1, 1, N, d), generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    qref = W.reference_queries("test", 1, 1, d)
+    Q = torch.randn((1, 1, G, d), generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    p = [0.5, 1.0, 1.0, 1.0]
+    cfg = zha.Config(d=d, Hq=G, Hkv=1, B=64, b=16, batch=1, N_cap=N, p=p)
+    dec = Decoder(cfg, K.cuda(), V.cuda(), qref.cuda(), [N])
+    dec.build()
+    for _ in range(3):   # the claims interleave differently from run to run; the result may not
+        dec.route_attend(Q.cuda())
+        sel, cnt, _ = dec.results()
+        for h in range(G):
+            assert int(cnt[0, 0, h]) == 5000
+            assert torch.equal(sel[0, 0, h, :5000], torch.arange(5000, dtype=torch.int32))
+    ot = oracle_tree(K[0, 0], N, cfg, qref[0])
+    assert list(O.route(Q[0, 0, 0], ot, p).sel) == list(range(5000))
+    assert_status_clean()
+
+
 def test_thousands_of_exact_ties_keep_the_lowest_ids():
     """All keys zero: every summary, hence every score, is equal.  p = 0.5 at level 1 (p = 1 above)
     keeps the lowest half of the 4687 leaf blocks, ties going to the lower id."""
