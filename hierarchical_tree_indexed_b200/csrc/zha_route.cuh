@@ -86,13 +86,13 @@ struct CutSmem {
 struct HelpSmem {
     uint32_t claim;            // (level << 24) | next job; jobs are claimed two at a time; 0: none
     uint32_t done;             // jobs of the offered level finished, helpers' included
-    uint32_t walk_done;        // this CTA's walk is over: its helpers may leave
+    uint32_t walk_done;        // this CTA's walk is over: it offers nothing more
     int level, np, b;
     int64_t nl;                // nodes of the offered level
     const float* kh;           // the level's summaries and biases of this slice (global memory)
     const float* bh;
-    float* sc_global;          // the scores, when they live in the workspace,
-    uint32_t sc_smem;          //   else in this CTA's shared memory
+    float* sc_global;          // the scores, when they live in the workspace (the levels offered),
+    uint32_t sc_smem;          //   else in this CTA's shared memory (helpers handle both)
     uint32_t par_smem;         // the kept parents in shared memory,
     const int32_t* par_global; //   or in the workspace
     uint32_t mx_smem;          // the level's max score slot (order-mapped int)
